@@ -1,0 +1,151 @@
+"""Python side of the fp64 CPU oracle (test infrastructure only).
+
+Only the tests, the smoke check and the CPU-baseline leg of the benchmark use
+this module. It builds ``tfmoe_oracle.c`` with gcc into ``libtfmoe_oracle.so``
+beside it (on first use, or through :func:`build`) and calls it via ctypes.
+It imports nothing from the CUDA package.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Dict, Optional
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "tfmoe_oracle.c")
+LIB = os.path.join(HERE, "libtfmoe_oracle.so")
+
+_u16p = ctypes.POINTER(ctypes.c_uint16)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
+_f32p = ctypes.POINTER(ctypes.c_float)
+_f64p = ctypes.POINTER(ctypes.c_double)
+_i32p = ctypes.POINTER(ctypes.c_int32)
+
+
+class _Layer(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int32), ("intermediate", ctypes.c_int32),
+                ("num_experts", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("router_w", _u16p), ("router_bias", _f32p),
+                ("gate_codes", _u8p), ("up_codes", _u8p),
+                ("gate_scales", _u8p), ("up_scales", _u8p),
+                ("gate_global", _f32p), ("up_global", _f32p),
+                ("down_codes", _u8p), ("down_scales", _u8p), ("down_global", _f32p)]
+
+
+class _Outputs(ctypes.Structure):
+    _fields_ = [("out", _u16p), ("out64", _f64p), ("S", _f64p), ("logits", _f32p),
+                ("ids", _i32p), ("g", _f64p), ("G", _f32p), ("U", _f32p),
+                ("a", _u16p), ("y", _f64p)]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (IEEE semantics: no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+        tmp = LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+                               "-shared", "-fPIC", "-std=c11", SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, LIB)
+    return LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        _lib.oracle_e2m1.restype = ctypes.c_double
+        _lib.oracle_e2m1.argtypes = [ctypes.c_uint]
+        _lib.oracle_e4m3.restype = ctypes.c_double
+        _lib.oracle_e4m3.argtypes = [ctypes.c_uint]
+        _lib.oracle_round_bf16.restype = ctypes.c_uint16
+        _lib.oracle_round_bf16.argtypes = [ctypes.c_double]
+        _lib.oracle_bf16_to_double.restype = ctypes.c_double
+        _lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+        _lib.oracle_forward.restype = ctypes.c_int
+        _lib.oracle_forward.argtypes = [ctypes.POINTER(_Layer), _u16p, ctypes.c_int32,
+                                        ctypes.c_int32, ctypes.POINTER(_Outputs)]
+        _lib.oracle_max_threads.restype = ctypes.c_int
+    return _lib
+
+
+def e2m1(code: int) -> float:
+    return lib().oracle_e2m1(code)
+
+
+def e4m3(byte: int) -> float:
+    return lib().oracle_e4m3(byte)
+
+
+def round_bf16(v: float) -> int:
+    return int(lib().oracle_round_bf16(v))
+
+
+def bf16_to_float(bits: int) -> float:
+    return lib().oracle_bf16_to_double(bits)
+
+
+def max_threads() -> int:
+    return int(lib().oracle_max_threads())
+
+
+def _ptr(a: Optional[np.ndarray], t):
+    if a is None:
+        return ctypes.cast(None, t)
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(t)
+
+
+def forward(layer: Dict[str, Optional[np.ndarray]], x: np.ndarray, *, top_k: int,
+            nthreads: int = 0, intermediates: bool = False) -> Dict[str, np.ndarray]:
+    """Run the oracle on host arrays in the canonical layout.
+
+    ``x`` is bf16 bits [T][H]. Returns out (bf16 bits), out64, S, and with
+    ``intermediates`` also logits, ids, g, G, U, a and y.
+    """
+    E, H = layer["router_w"].shape
+    I = layer["gate_codes"].shape[1]
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    T = x.shape[0]
+    assert x.shape == (T, H)
+    keep = []
+
+    def arr(name, dtype):
+        a = np.ascontiguousarray(layer[name], dtype=dtype)
+        keep.append(a)
+        return a
+
+    L = _Layer(H, I, E, top_k,
+               _ptr(arr("router_w", np.uint16), _u16p),
+               _ptr(None if layer.get("router_bias") is None else arr("router_bias", np.float32), _f32p),
+               _ptr(arr("gate_codes", np.uint8), _u8p), _ptr(arr("up_codes", np.uint8), _u8p),
+               _ptr(arr("gate_scales", np.uint8), _u8p), _ptr(arr("up_scales", np.uint8), _u8p),
+               _ptr(arr("gate_global", np.float32), _f32p), _ptr(arr("up_global", np.float32), _f32p),
+               _ptr(arr("down_codes", np.uint8), _u8p), _ptr(arr("down_scales", np.uint8), _u8p),
+               _ptr(arr("down_global", np.float32), _f32p))
+    P = T * top_k
+    res = {"out": np.zeros((T, H), np.uint16), "out64": np.zeros((T, H), np.float64),
+           "S": np.zeros((T, H), np.float64)}
+    if intermediates:
+        res.update(logits=np.zeros((T, E), np.float32), ids=np.zeros((T, top_k), np.int32),
+                   g=np.zeros((T, top_k), np.float64), G=np.zeros((T, top_k, I), np.float32),
+                   U=np.zeros((T, top_k, I), np.float32), a=np.zeros((T, top_k, I), np.uint16),
+                   y=np.zeros((T, top_k, H), np.float64))
+    O = _Outputs(_ptr(res["out"], _u16p), _ptr(res["out64"], _f64p), _ptr(res["S"], _f64p),
+                 _ptr(res.get("logits"), _f32p), _ptr(res.get("ids"), _i32p),
+                 _ptr(res.get("g"), _f64p), _ptr(res.get("G"), _f32p), _ptr(res.get("U"), _f32p),
+                 _ptr(res.get("a"), _u16p), _ptr(res.get("y"), _f64p))
+    rc = lib().oracle_forward(ctypes.byref(L), _ptr(x, _u16p), T, nthreads, ctypes.byref(O))
+    if rc != 0:
+        raise RuntimeError(f"oracle_forward failed with code {rc}")
+    del keep, P
+    return res
+
+
+def tolerance(S: np.ndarray) -> np.ndarray:
+    """Per-element bound |gpu - oracle| <= 4e-3 * S + 1e-3, S = sum |a*w| (g-weighted)."""
+    return 4e-3 * S + 1e-3

@@ -1,0 +1,294 @@
+/*
+ * tfmoe_oracle.c -- plain fp64 CPU oracle for the forward pass of one
+ * mixture-of-experts FFN layer with NVFP4 weights and BF16 activations
+ * (W4A16).
+ *
+ * TEST INFRASTRUCTURE. Only the tests, the smoke check and the CPU-baseline
+ * leg of the benchmark load this library. The CUDA library never links,
+ * includes or calls it, and the two share no source.
+ *
+ * What it computes, and where each step comes from:
+ *
+ *  - W4A16: weights are NVFP4 (4-bit floats carrying a scale), inputs stay
+ *    BF16 and the arithmetic is done at higher precision, not on FP4
+ *    operands [TensorFold 1.0.12 GLM-5.3-Flash post, section "NVFP4 is
+ *    neither uniform 4-bit nor all-FP4 compute"].
+ *  - Only the experts a token routes to are evaluated; their weights are what
+ *    a decode step must stream [DGX Spark GB10 bandwidth-budget page, section
+ *    "Mechanism: decode is bandwidth-bound, prefill is compute-bound"].
+ *  - The per-layer sequence router -> top-k -> plan -> routed experts ->
+ *    weighted combine is the MoE chain of [TensorFold issue #627, comment
+ *    "Where the 0.35 ms per step goes"].
+ *  - Bit layouts: E2M1 and E4M3 follow the OCP Microscaling (MX) format
+ *    definitions; one E4M3 scale per 16 consecutive reduction elements and one
+ *    fp32 per-tensor multiplier per (expert, projection).
+ *  - The reference is 64-bit, as the error budget of [TensorFold issue #627,
+ *    "Description"] is stated against a float64 reference.
+ *
+ * Rounding points (the only places precision is lost on purpose):
+ *   router logit      = fp32( fp64 sum of bf16*bf16 products ) (+ fp32 bias)
+ *   gate G, up U      = fp32( fp64 sum over K of x * deq(w) )
+ *   a = bf16_RNE( silu(G) * U )   evaluated in fp64 from the fp32 G, U
+ *   y = fp64 sum over K of a * deq(w)      (not rounded)
+ *   out = bf16_RNE( sum over slots s=0..k-1 of g_s * y_s )   in fp64
+ *
+ * Parity pins live in the repository's CPU test-suite; every function below
+ * is pinned there (format tables, a hand-worked block, closed-form chains,
+ * routing invariants and a brute-force dense-equivalent computation).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <omp.h>
+
+/* ------------------------------------------------------------------ */
+/* Number formats                                                       */
+/* ------------------------------------------------------------------ */
+
+/* E2M1: bit 3 sign, bits 2..1 exponent (bias 1), bit 0 mantissa.
+ * Exponent 0 is subnormal: 0.5 * m. Otherwise (1 + m/2) * 2^(e-1). */
+double oracle_e2m1(unsigned code)
+{
+    unsigned s = (code >> 3) & 1u, e = (code >> 1) & 3u, m = code & 1u;
+    double mag = (e == 0) ? 0.5 * (double)m : (1.0 + 0.5 * (double)m) * ldexp(1.0, (int)e - 1);
+    return s ? -mag : mag;
+}
+
+/* E4M3 ("fn" variant): bit 7 sign, bits 6..3 exponent (bias 7), bits 2..0
+ * mantissa. Exponent 0 is subnormal (m/8) * 2^-6. Exponent 15 with mantissa 7
+ * is NaN; there is no infinity, so the largest value is 448. */
+double oracle_e4m3(unsigned byte)
+{
+    unsigned s = (byte >> 7) & 1u, e = (byte >> 3) & 15u, m = byte & 7u;
+    if (e == 15u && m == 7u) return NAN;
+    double mag = (e == 0) ? ((double)m / 8.0) * ldexp(1.0, -6)
+                          : (1.0 + (double)m / 8.0) * ldexp(1.0, (int)e - 7);
+    return s ? -mag : mag;
+}
+
+double oracle_bf16_to_double(uint16_t bits)
+{
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Round a double to the nearest bfloat16 (ties to even), directly from the
+ * double: bf16 keeps 8 significant bits and fp32's exponent range, so the
+ * quantum is 2^(e-8) for |v| in [2^(e-1), 2^e), and 2^-133 below 2^-126. */
+uint16_t oracle_round_bf16(double v)
+{
+    if (isnan(v)) return 0x7FC0u;
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    double a = fabs(v);
+    if (isinf(a)) return (uint16_t)(sign | 0x7F80u);
+    if (a == 0.0) return sign;
+    int e;
+    (void)frexp(a, &e);               /* a = f * 2^e, f in [0.5, 1) */
+    int q_exp = e - 8;
+    if (q_exp < -133) q_exp = -133;
+    double r = ldexp(rint(ldexp(a, -q_exp)), q_exp);   /* rint: nearest, ties to even */
+    if (r >= ldexp(1.0, 128)) return (uint16_t)(sign | 0x7F80u);
+    float f = (float)r;               /* exact: r has <= 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(sign | ((u >> 16) & 0x7FFFu));
+}
+
+/* One weight row of an NVFP4 matrix, decoded to fp64:
+ * deq[c] = E2M1(code c) * E4M3(scale of block c/16) * global.
+ * Element c sits in byte c/2, low nibble when c is even. */
+static void dequant_row(const uint8_t *codes, const uint8_t *scales, float global, int K, double *deq)
+{
+    for (int c = 0; c < K; ++c) {
+        uint8_t byte = codes[c / 2];
+        unsigned nib = (c % 2 == 0) ? (byte & 0x0Fu) : (byte >> 4);
+        deq[c] = oracle_e2m1(nib) * oracle_e4m3(scales[c / 16]) * (double)global;
+    }
+}
+
+static double silu(double z) { return z / (1.0 + exp(-z)); }
+
+/* ------------------------------------------------------------------ */
+/* The layer                                                            */
+/* ------------------------------------------------------------------ */
+
+typedef struct {
+    int32_t hidden, intermediate, num_experts, top_k;
+    const uint16_t *router_w;      /* bf16 [E][H] */
+    const float *router_bias;      /* fp32 [E] or NULL */
+    const uint8_t *gate_codes, *up_codes;     /* [E][I][H/2] */
+    const uint8_t *gate_scales, *up_scales;   /* [E][I][H/16] */
+    const float *gate_global, *up_global;     /* [E] */
+    const uint8_t *down_codes;                /* [E][H][I/2] */
+    const uint8_t *down_scales;               /* [E][H][I/16] */
+    const float *down_global;                 /* [E] */
+} oracle_layer;
+
+/* Outputs. Every pointer except out may be NULL. Per-pair arrays are indexed
+ * by pair = t*k + s, s the slot (0 = highest logit). */
+typedef struct {
+    uint16_t *out;      /* bf16 [T][H] */
+    double *out64;      /* [T][H] value before the final rounding */
+    double *S;          /* [T][H] sum_s g_s * sum_j |a_s[j] * deq(Wd)[h][j]| */
+    float *logits;      /* [T][E] */
+    int32_t *ids;       /* [T][k] */
+    double *g;          /* [T][k] */
+    float *G, *U;       /* [T][k][I] */
+    uint16_t *a;        /* bf16 [T][k][I] */
+    double *y;          /* [T][k][H] */
+} oracle_outputs;
+
+/* Router logits, top-k (ties to the lower expert index) and the softmax
+ * weights over the selected logits for token row x. */
+static void route_token(const oracle_layer *L, const uint16_t *x, float *logits, int32_t *ids, double *g)
+{
+    const int H = L->hidden, E = L->num_experts, k = L->top_k;
+    for (int e = 0; e < E; ++e) {
+        double acc = 0.0;
+        for (int h = 0; h < H; ++h)
+            acc += oracle_bf16_to_double(x[h]) * oracle_bf16_to_double(L->router_w[(size_t)e * H + h]);
+        float l = (float)acc;
+        if (L->router_bias) l = l + L->router_bias[e];
+        logits[e] = l;
+    }
+    char *taken = (char *)calloc((size_t)E, 1);
+    for (int s = 0; s < k; ++s) {
+        int best = -1;
+        for (int e = 0; e < E; ++e)
+            if (!taken[e] && (best < 0 || logits[e] > logits[best])) best = e;
+        ids[s] = best;
+        taken[best] = 1;
+    }
+    free(taken);
+    double lmax = (double)logits[ids[0]], den = 0.0;
+    for (int s = 0; s < k; ++s) den += exp((double)logits[ids[s]] - lmax);
+    for (int s = 0; s < k; ++s) g[s] = exp((double)logits[ids[s]] - lmax) / den;
+}
+
+int oracle_forward(const oracle_layer *L, const uint16_t *x, int32_t T, int32_t nthreads,
+                   const oracle_outputs *O)
+{
+    if (!L || !O || T < 0) return 1;
+    const int H = L->hidden, I = L->intermediate, E = L->num_experts, k = L->top_k;
+    if (H <= 0 || I <= 0 || E <= 0 || k <= 0 || k > E || H % 16 || I % 16) return 1;
+    if (T == 0) return 0;
+    if (nthreads <= 0) nthreads = omp_get_max_threads();
+    const size_t P = (size_t)T * k;
+
+    float *logits = (float *)malloc(sizeof(float) * (size_t)T * E);
+    int32_t *ids = (int32_t *)malloc(sizeof(int32_t) * P);
+    double *g = (double *)malloc(sizeof(double) * P);
+    uint16_t *a = (uint16_t *)malloc(sizeof(uint16_t) * P * I);
+    double *y = (double *)malloc(sizeof(double) * P * H);
+    double *yabs = (double *)malloc(sizeof(double) * P * H);
+    double *xd = (double *)malloc(sizeof(double) * (size_t)T * H);
+    int32_t *count = (int32_t *)calloc((size_t)E, sizeof(int32_t));
+    int32_t *start = (int32_t *)malloc(sizeof(int32_t) * ((size_t)E + 1));
+    int32_t *pairs = (int32_t *)malloc(sizeof(int32_t) * P);
+    if (!logits || !ids || !g || !a || !y || !yabs || !xd || !count || !start || !pairs) return 2;
+
+    /* Step 1: routing, token by token. */
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1)
+    for (int t = 0; t < T; ++t)
+        route_token(L, x + (size_t)t * H, logits + (size_t)t * E, ids + (size_t)t * k, g + (size_t)t * k);
+
+    for (size_t i = 0; i < (size_t)T * H; ++i) xd[i] = oracle_bf16_to_double(x[i]);
+
+    /* Step 2: per-expert pair lists, in (token, slot) order. */
+    for (size_t p = 0; p < P; ++p) count[ids[p]]++;
+    start[0] = 0;
+    for (int e = 0; e < E; ++e) start[e + 1] = start[e] + count[e];
+    {
+        int32_t *fill = (int32_t *)calloc((size_t)E, sizeof(int32_t));
+        for (size_t p = 0; p < P; ++p) { int e = ids[p]; pairs[start[e] + fill[e]++] = (int32_t)p; }
+        free(fill);
+    }
+
+    /* Step 3: gate and up projections with the SwiGLU activation, one
+     * expert at a time, rows in parallel. */
+    for (int e = 0; e < E; ++e) {
+        if (count[e] == 0) continue;
+#pragma omp parallel num_threads(nthreads)
+        {
+            double *dg = (double *)malloc(sizeof(double) * H);
+            double *du = (double *)malloc(sizeof(double) * H);
+#pragma omp for schedule(static)
+            for (int j = 0; j < I; ++j) {
+                size_t row = (size_t)e * I + j;
+                dequant_row(L->gate_codes + row * (H / 2), L->gate_scales + row * (H / 16), L->gate_global[e], H, dg);
+                dequant_row(L->up_codes + row * (H / 2), L->up_scales + row * (H / 16), L->up_global[e], H, du);
+                for (int q = start[e]; q < start[e + 1]; ++q) {
+                    int p = pairs[q], t = p / k;
+                    const double *xr = xd + (size_t)t * H;
+                    double sg = 0.0, su = 0.0;
+                    for (int h = 0; h < H; ++h) { sg += xr[h] * dg[h]; su += xr[h] * du[h]; }
+                    float G = (float)sg, U = (float)su;
+                    if (O->G) O->G[(size_t)p * I + j] = G;
+                    if (O->U) O->U[(size_t)p * I + j] = U;
+                    a[(size_t)p * I + j] = oracle_round_bf16(silu((double)G) * (double)U);
+                }
+            }
+            free(dg);
+            free(du);
+        }
+    }
+
+    /* Step 4: down projection, rows in parallel; y stays in fp64. */
+    for (int e = 0; e < E; ++e) {
+        if (count[e] == 0) continue;
+#pragma omp parallel num_threads(nthreads)
+        {
+            double *dd = (double *)malloc(sizeof(double) * I);
+#pragma omp for schedule(static)
+            for (int h = 0; h < H; ++h) {
+                size_t row = (size_t)e * H + h;
+                dequant_row(L->down_codes + row * (I / 2), L->down_scales + row * (I / 16), L->down_global[e], I, dd);
+                for (int q = start[e]; q < start[e + 1]; ++q) {
+                    int p = pairs[q];
+                    const uint16_t *ar = a + (size_t)p * I;
+                    double s = 0.0, sa = 0.0;
+                    for (int j = 0; j < I; ++j) {
+                        double term = oracle_bf16_to_double(ar[j]) * dd[j];
+                        s += term;
+                        sa += fabs(term);
+                    }
+                    y[(size_t)p * H + h] = s;
+                    yabs[(size_t)p * H + h] = sa;
+                }
+            }
+            free(dd);
+        }
+    }
+
+    /* Step 5: weighted combine in slot order, rounded once to bf16. */
+#pragma omp parallel for num_threads(nthreads) schedule(static)
+    for (int t = 0; t < T; ++t) {
+        for (int h = 0; h < H; ++h) {
+            double acc = 0.0, bound = 0.0;
+            for (int s = 0; s < k; ++s) {
+                size_t p = (size_t)t * k + s;
+                acc += g[p] * y[p * H + h];
+                bound += g[p] * yabs[p * H + h];
+            }
+            size_t o = (size_t)t * H + h;
+            if (O->out) O->out[o] = oracle_round_bf16(acc);
+            if (O->out64) O->out64[o] = acc;
+            if (O->S) O->S[o] = bound;
+        }
+    }
+
+    if (O->logits) memcpy(O->logits, logits, sizeof(float) * (size_t)T * E);
+    if (O->ids) memcpy(O->ids, ids, sizeof(int32_t) * P);
+    if (O->g) memcpy(O->g, g, sizeof(double) * P);
+    if (O->a) memcpy(O->a, a, sizeof(uint16_t) * P * I);
+    if (O->y) memcpy(O->y, y, sizeof(double) * P * H);
+
+    free(logits); free(ids); free(g); free(a); free(y); free(yabs); free(xd);
+    free(count); free(start); free(pairs);
+    return 0;
+}
+
+int oracle_max_threads(void) { return omp_get_max_threads(); }
