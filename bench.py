@@ -1,0 +1,450 @@
+#!/usr/bin/env python
+"""Throughput of the NVFP4 W4A16 MoE FFN layer forward (libtfmoe) on B200.
+
+Default workload (N=1): the decode layer shape -- H=2048, I=768, E=128, top-8,
+T=8 tokens per forward -- three seeded layers (seeds 1, 2, 3) rotated so that
+consecutive forwards read different weights (each forward touches ~137 MB; a
+layer is re-read only after two other layers' ~274 MB, which exceeds the
+126 MB L2). A step is one forward of the whole layer (router, top-k, permute,
+gate/up + SwiGLU, down, combine) over one batch; eight distinct seeded
+activation batches rotate per layer. Forwards are replayed from CUDA graphs of
+up to 100 consecutive forwards.
+
+Printed JSON line (rank 0): value = tokens/s over all ranks, e2e = the same
+metric through tfmoe_forward_host with pinned host buffers (copies inside the
+timed region), roofline of the dominant kernel measured live with CUDA events,
+cpu_baseline = the fp64 oracle on a bounded sample on this host's cores.
+
+--impl reference times the fp64 CPU oracle (the only reference this layer has)
+on the same workload, one token per step.
+
+Multi-GPU (torchrun): replicas only -- every rank runs its own layers on its
+own GPU with no data-path collective (weak scaling); the timed region is
+bracketed by barriers and the max over ranks is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "NVFP4 MoE layer tok/s; decode HBM GB/s, prefill TFLOP/s vs B200 peak"
+NVFP4_BYTES_PER_WEIGHT = 0.5625        # 4-bit code + one E4M3 byte per 16 weights
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+WORKLOADS = {
+    # name: (layer shape index, tokens per forward, seeds)
+    "decode": (1, 8, (1, 2, 3)),
+    "decode_t1": (1, 1, (1, 2, 3)),
+    "tiny": (0, 4, (0,)),
+    "zipf": (2, 256, (4,)),
+    "prefill": (3, 8192, (5,)),
+    "sweep_t1": (4, 1, (6,)),
+    "sweep_t32": (4, 32, (6,)),
+    "sweep_t256": (4, 256, (6,)),
+    "sweep_t2048": (4, 2048, (6,)),
+    "sweep_t7234": (4, 7234, (6,)),
+}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, interval_ms: int = 10):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 f"-lms={interval_ms}", "-i", str(gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.05)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [v.strip() for v in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("gemv.cu", "common.cuh", "internal.h"):
+        h.update(open(os.path.join(ROOT, "nvfp4_weight_only_route_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(stage: str):
+    """DRAM bytes per launch from a committed ncu capture, if it matches the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    ent = d.get(stage)
+    if not ent or ent.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def oracle_cpu_sample(shape, layers, xs, seconds: float):
+    """Time the fp64 oracle on whole decode batches (or single tokens for big shapes)."""
+    from oracle import oracle
+    oracle.build()
+    tokens, n, t0 = 0, 0, time.perf_counter()
+    while True:
+        L = layers[n % len(layers)]
+        x = xs[n % len(xs)]
+        if shape.H * shape.I * shape.k * x.shape[0] > 2 ** 27:
+            x = x[n % x.shape[0]: n % x.shape[0] + 1]
+        oracle.forward(L, x, top_k=shape.k)
+        tokens += x.shape[0]
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return tokens / el, oracle.max_threads(), f"{n} oracle forwards, {tokens} tokens, {el:.1f} s"
+
+
+def dist_setup(n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    return rank, world, local, pg
+
+
+def barrier(pg, torch):
+    if pg is not None:
+        pg.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(pg, torch, v: float) -> float:
+    if pg is None:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from nvfp4_weight_only_route_b200 import synth
+    from oracle import oracle
+    oracle.build()
+    shape_idx, T, seeds = WORKLOADS[args.workload]
+    shape = synth.SHAPES[shape_idx]
+    layers = [synth.make_layer(shape, s) for s in seeds]
+    xs = [synth.make_x(shape, s, T, stream=r) for s in seeds for r in range(2)]
+
+    def step(i):
+        x = xs[i % len(xs)]
+        j = (i // len(xs)) % x.shape[0]
+        oracle.forward(layers[i % len(layers)], x[j:j + 1], top_k=shape.k)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    el = time.perf_counter() - t0
+    value = args.steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: H={shape.H} I={shape.I} E={shape.E} top-{shape.k} T={T}, seeds {list(seeds)}",
+                   "reference": "fp64 CPU oracle, one token of the workload per step"},
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": oracle.max_threads(), "kind": "oracle",
+                         "sample": f"{args.steps} steps of one token each"},
+        "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["tfmoe", "reference"], default="tfmoe")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
+    ap.add_argument("--flags", type=int, default=0, help="descriptor flags (1 = force GEMV, 2 = force MMA)")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", type=int, default=100, help="forwards per CUDA graph (0 = no graphs)")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+
+    from nvfp4_weight_only_route_b200 import synth, tfmoe
+    rank, world, local, pg = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    hbm_peak, bf16_peak, bf16_sustained, peak_src = load_peaks()
+
+    shape_idx, T, seeds = WORKLOADS[args.workload]
+    shape = synth.SHAPES[shape_idx]
+    H, I, E, k = shape.H, shape.I, shape.E, shape.k
+    n_x = 8 if T <= 256 else 2
+    layers_np, layers, xs = [], [], []
+    for s in seeds:
+        lnp = synth.make_layer(shape, s + 1000 * rank) if rank else synth.make_layer(shape, s)
+        layers_np.append(lnp)
+        L = tfmoe.MoELayer(H, I, E, k, T, has_router_bias=lnp["router_bias"] is not None, flags=args.flags)
+        L.load_weights(tfmoe.layer_to_device(lnp, dev))
+        layers.append(L)
+        xs.append([torch.from_numpy(synth.make_x(shape, s, T, stream=r + 100 * rank).view(np.int16)).to(dev)
+                   for r in range(n_x)])
+    torch.cuda.synchronize()
+    out = torch.empty((T, H), dtype=torch.int16, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def fwd(i):
+        L = layers[i % len(layers)]
+        x = xs[i % len(layers)][(i // len(layers)) % n_x]
+        tfmoe.check(L.forward_raw(x.data_ptr(), T, out.data_ptr(), stream.cuda_stream))
+        return L
+
+    # ---- parity gate against the oracle (rank 0), sampled tokens for large T
+    parity = "skipped"
+    if rank == 0:
+        from oracle import oracle
+        worst = 0.0
+        for li, L in enumerate(layers):
+            with torch.cuda.stream(stream):
+                fwd(li)
+            stream.synchronize()
+            tfmoe.check(L.sync_status(stream))
+            got = out.cpu().numpy().view(np.uint16)
+            ids_g = L.buffer_tensor(tfmoe.BUF_TOPK_IDS, torch.int32, (T, k)).cpu().numpy()
+            x_np = xs[li][0].cpu().numpy().view(np.uint16)
+            idx = np.arange(T) if T <= 64 else np.unique(np.linspace(0, T - 1, 16).astype(int))
+            ref = oracle.forward(layers_np[li], x_np[idx], top_k=k, intermediates=True)
+            if not np.array_equal(ids_g[idx], ref["ids"]):
+                raise SystemExit("parity gate: routing differs from the oracle")
+            g64 = (got[idx].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            half_ulp = 0.5 * 2.0 ** (np.floor(np.log2(np.maximum(np.maximum(np.abs(g64), np.abs(ref["out64"])), 2.0 ** -126))) - 7)
+            tol = 4e-3 * ref["S"] + 1e-3 + half_ulp
+            err = np.abs(g64 - ref["out64"])
+            if not np.all(err <= tol):
+                raise SystemExit(f"parity gate: output outside tolerance (worst {float(np.max(err / tol)):.3f})")
+            worst = max(worst, float(np.max(err / tol)))
+        parity = f"ok: ids bit-exact, worst |err|/tol {worst:.3f} on {len(layers)} layer(s)"
+
+    # ---- routing statistics for the algorithmic byte / flop counts
+    active, gemv_experts, launches_per_fwd = [], [], 0
+    n_inputs = len(layers) * n_x
+    for i in range(n_inputs):
+        with torch.cuda.stream(stream):
+            L = fwd(i)
+        stream.synchronize()
+        launches_per_fwd = L.last_launch_count()
+        cnt = L.buffer_tensor(tfmoe.BUF_EXPERT_COUNTS, torch.int32, (E,)).cpu().numpy()
+        reg = L.buffer_tensor(tfmoe.BUF_REGIME, torch.int32, (E,)).cpu().numpy()
+        active.append(int(np.sum(cnt > 0)))
+        gemv_experts.append(int(np.sum(reg == 1)))
+    mean_active = float(np.mean(active))
+    mean_gemv = float(np.mean(gemv_experts))
+    weight_bytes_expert = 3 * H * I * NVFP4_BYTES_PER_WEIGHT
+    bytes_per_fwd = mean_active * weight_bytes_expert + E * H * 2 + T * H * 2 * 2
+    flops_per_fwd = 2.0 * T * k * 3 * H * I + 2.0 * T * H * E
+
+    # ---- CUDA graphs of consecutive forwards, all captured before timing. Each graph
+    # starts at input index 0 and holds a whole number of input cycles when it can.
+    cycle = len(layers) * n_x
+    G = 0
+    if args.graph > 0:
+        G = max(cycle, (args.graph // cycle) * cycle) if args.steps >= cycle else args.steps
+        G = min(G, args.steps)
+    graphs = {}
+
+    def make_graph(n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for j in range(n):
+                fwd(j)
+        return g
+
+    def run_steps(n, start):
+        if G == 0:
+            with torch.cuda.stream(stream):
+                for j in range(n):
+                    fwd(start + j)
+            return
+        done = 0
+        while done < n:
+            m = min(G, n - done)
+            graphs[m].replay()
+            done += m
+
+    if G:
+        sizes = {G} if args.steps >= G else set()
+        if args.steps % G:
+            sizes.add(args.steps % G)
+        w_full, w_rem = divmod(args.warmup, G)
+        if w_rem:
+            sizes.add(w_rem)
+        for m in sorted(sizes):
+            graphs[m] = make_graph(m)
+            graphs[m].replay()          # first replay of every graph happens before timing
+        stream.synchronize()
+    run_steps(args.warmup, 0)
+    stream.synchronize()
+
+    # ---- timed region
+    sampler = ClockSampler(local) if rank == 0 else None
+    barrier(pg, torch)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        run_steps(args.steps, args.warmup)
+        ev1.record(stream)
+    stream.synchronize()
+    barrier(pg, torch)
+    clocks = sampler.stop() if sampler else None
+    ms_local = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(pg, torch, ms_local)
+    value = world * T * args.steps / (ms / 1e3)
+
+    # ---- per-stage timing (profiled forwards, not graph-captured) for the roofline
+    prof_steps = min(args.steps, 200)
+    for L in layers:
+        L.profile(True)
+        L.profile_read(reset=True)
+    for i in range(prof_steps):
+        with torch.cuda.stream(stream):
+            fwd(i)
+    stage_ms = {}
+    for L in layers:
+        for name, (ms_tot, calls) in L.profile_read(reset=True).items():
+            a, c = stage_ms.get(name, (0.0, 0))
+            stage_ms[name] = (a + ms_tot, c + calls)
+        L.profile(False)
+    stage_avg_us = {n: (v[0] / v[1] * 1e3 if v[1] else 0.0) for n, v in stage_ms.items()}
+    dominant = max(stage_avg_us, key=stage_avg_us.get)
+    if dominant in ("gemv_gate_up", "gemv_down"):
+        rows = 2 * I * H if dominant == "gemv_gate_up" else H * I
+        alg = mean_gemv * rows * NVFP4_BYTES_PER_WEIGHT
+        achieved = alg / (stage_avg_us[dominant] * 1e-6) / 1e9
+        roofline = {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": achieved / hbm_peak, "traffic": ncu_traffic(dominant),
+                    "algorithmic_bytes_per_launch": alg, "avg_launch_us": stage_avg_us[dominant],
+                    "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback"}
+    else:
+        roofline = {"bound": "tensor", "kernel": dominant, "achieved": None, "peak": bf16_peak, "unit": "TFLOP/s",
+                    "frac": None, "traffic": ncu_traffic(dominant), "avg_launch_us": stage_avg_us[dominant]}
+    layer_gbs = bytes_per_fwd / (ms / args.steps * 1e-3) / 1e9
+    layer_tflops = flops_per_fwd / (ms / args.steps * 1e-3) / 1e12
+
+    # ---- end to end through the host-buffer entry point (pinned memory)
+    x_host = [xs[li][r].cpu().pin_memory() for li in range(len(layers)) for r in range(min(n_x, 2))]
+    out_host = torch.empty((T, H), dtype=torch.int16).pin_memory()
+    e2e_steps = min(args.steps, 500)
+    barrier(pg, torch)
+    t0 = time.perf_counter()
+    for i in range(e2e_steps):
+        L = layers[i % len(layers)]
+        L.forward_host(x_host[i % len(x_host)], out_host, T=T, stream=stream)
+    el = time.perf_counter() - t0
+    el = max_over_ranks(pg, torch, el)
+    e2e = {"value": world * T * e2e_steps / el, "unit": "tok/s", "h2d_bytes_per_step": T * H * 2,
+           "d2h_bytes_per_step": T * H * 2, "steps": e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample = oracle_cpu_sample(shape, layers_np, [x.cpu().numpy().view(np.uint16) for x in xs[0]],
+                                             args.cpu_seconds)
+        cpu = {"value": v, "unit": "tok/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 activations, nvfp4 weights, fp32 accumulate", "data": "synthetic",
+            "config": {"workload": f"{args.workload}: H={H} I={I} E={E} top-{k} T={T} tokens/forward, "
+                                   f"seeds {list(seeds)} rotated", "global_batch": T * world,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2: rotating seeded layers / full weight sets exceed 126 MB",
+                       "flags": args.flags, "graph_forwards": G},
+            "roofline": roofline,
+            "layer": {"algorithmic_bytes_per_forward": bytes_per_fwd, "hbm_gbs": layer_gbs,
+                      "hbm_frac": layer_gbs / hbm_peak, "hbm_frac_of_8tbs": layer_gbs / 8000.0,
+                      "flops_per_forward": flops_per_fwd, "tflops": layer_tflops,
+                      "tensor_frac": layer_tflops / bf16_peak, "active_experts_mean": mean_active,
+                      "stage_avg_us": stage_avg_us},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_fwd * args.steps,
+            "clocks": clocks,
+            "parity": parity,
+        }
+        print(json.dumps(line), flush=True)
+    for g in graphs.values():
+        del g
+    graphs.clear()
+    for L in layers:
+        L.close()
+    if pg is not None:
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,210 @@
+/*
+ * tfmoe.h -- C ABI of libtfmoe: the forward pass of one mixture-of-experts FFN
+ * layer with NVFP4 weights and BF16 activations (W4A16) on one NVIDIA B200
+ * (sm_100a).
+ *
+ * What the layer computes (the operation every entry point below serves):
+ *
+ *   logits[t,e] = fp32( sum_h x[t,h] * Wr[e,h] ) (+ bias[e])        router
+ *   ids[t,0..k) = the k largest logits, ties to the lower expert index
+ *   g[t,s]      = softmax over the k selected logits                 weights
+ *   G = fp32(x . deq(Wgate_e)), U = fp32(x . deq(Wup_e))              per routed pair
+ *   a = bf16( silu(G) * U )                                           SwiGLU
+ *   y = a . deq(Wdown_e)^T                                            down projection
+ *   out[t,h] = bf16( sum_s g[t,s] * y_s[h] )                          weighted combine
+ *
+ *   deq(W)[r,c] = E2M1(code[r,c]) * E4M3(scale[r, c/16]) * global
+ *
+ * Passages this follows:
+ *  - W4A16, i.e. 4-bit-float weights with attached scales computed against
+ *    BF16 inputs rather than as all-FP4 arithmetic: TensorFold 1.0.12
+ *    GLM-5.3-Flash post, section "NVFP4 is neither uniform 4-bit nor all-FP4
+ *    compute".
+ *  - Only the routed experts' weights are read per token; decode streams
+ *    those weights, prefill is one large matrix multiply: DGX Spark GB10
+ *    bandwidth-budget page, section "Mechanism: decode is bandwidth-bound,
+ *    prefill is compute-bound".
+ *  - The chain router -> top-k -> plan -> routed experts -> weighted combine:
+ *    TensorFold issue #627, comment "Where the 0.35 ms per step goes" and
+ *    the per-launch kernel table (router, topk, add_moe_norm).
+ *  - E2M1 and E4M3 bit layouts: OCP Microscaling (MX) format definitions.
+ *
+ * Threading: handles are not thread-safe; use one handle per host thread or
+ * serialise. tfmoe_last_error() is thread-local.
+ */
+#ifndef TFMOE_H
+#define TFMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TFMOE_API __attribute__((visibility("default")))
+#else
+#define TFMOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TFMOE_OK = 0,
+    TFMOE_ERR_INVALID_ARG = 1,   /* a null pointer, a size out of range, T > max_tokens ... */
+    TFMOE_ERR_OOM = 2,           /* device allocation failed in create / load_weights */
+    TFMOE_ERR_CUDA = 3,          /* a CUDA call or kernel launch failed; see tfmoe_last_error() */
+    TFMOE_ERR_NOT_LOADED = 4,    /* forward before load_weights */
+    TFMOE_ERR_UNSUPPORTED = 5,   /* valid arguments this build does not handle (e.g. H % 128 != 0) */
+    TFMOE_ERR_TIMEOUT = 6,       /* a bounded device-side wait gave up (reported by tfmoe_sync_status) */
+    TFMOE_ERR_DEVICE = 7         /* a kernel's own check set the device error word */
+} tfmoe_status;
+
+typedef struct tfmoe_layer tfmoe_layer;   /* opaque */
+
+/* Descriptor flags. */
+#define TFMOE_FLAG_FORCE_GEMV    0x1u  /* every expert uses the CUDA-core GEMV regime */
+#define TFMOE_FLAG_FORCE_MMA     0x2u  /* every expert uses the tcgen05 tensor-core regime */
+#define TFMOE_FLAG_DEBUG_CHECKS  0x4u  /* kernels bounds-check ids/rows and set the error word */
+
+/*
+ * Layer shape. Requirements (else TFMOE_ERR_INVALID_ARG):
+ *   hidden H and intermediate I positive multiples of 16; 1 <= top_k <= num_experts;
+ *   max_tokens >= 1.
+ * This build additionally needs H % 128 == 0, I % 64 == 0 and num_experts <= 256
+ * (else TFMOE_ERR_UNSUPPORTED).
+ */
+typedef struct {
+    int32_t hidden;            /* H */
+    int32_t intermediate;      /* I: expert FFN width */
+    int32_t num_experts;       /* E */
+    int32_t top_k;             /* k */
+    int32_t max_tokens;        /* the largest T tfmoe_forward will accept; sizes the workspace */
+    int32_t has_router_bias;   /* 1: router_bias is read and added to the logits */
+    uint32_t flags;            /* TFMOE_FLAG_* */
+    int32_t gemv_max_tokens;   /* experts routed <= this many tokens use the GEMV regime;
+                                  <= 0 selects the built-in crossover */
+} tfmoe_layer_desc;
+
+/*
+ * Weights in the canonical layout: DEVICE pointers, row-major, caller-owned,
+ * read only during tfmoe_load_weights (which copies and repacks them).
+ * NVFP4 element c of a row sits in byte c/2 of that row, in the low nibble
+ * when c is even; one E4M3 scale byte per 16 consecutive elements of a row
+ * (the reduction dimension); one fp32 multiplier per expert and projection.
+ */
+typedef struct {
+    const uint16_t *router_w;       /* bf16 [E][H] */
+    const float    *router_bias;    /* fp32 [E]; read only when has_router_bias */
+    const uint8_t  *gate_codes;     /* [E][I][H/2] */
+    const uint8_t  *up_codes;       /* [E][I][H/2] */
+    const uint8_t  *gate_scales;    /* e4m3 [E][I][H/16] */
+    const uint8_t  *up_scales;      /* e4m3 [E][I][H/16] */
+    const float    *gate_global;    /* [E] */
+    const float    *up_global;      /* [E] */
+    const uint8_t  *down_codes;     /* [E][H][I/2] */
+    const uint8_t  *down_scales;    /* e4m3 [E][H][I/16] */
+    const float    *down_global;    /* [E] */
+} tfmoe_weights;
+
+/* Create a layer handle on the current CUDA device and allocate its
+ * workspace (sized by max_tokens) and weight storage. On error *out is NULL
+ * and nothing stays allocated. */
+TFMOE_API tfmoe_status tfmoe_create(const tfmoe_layer_desc *desc, tfmoe_layer **out);
+
+/* Copy the caller's canonical weights into library-owned device memory,
+ * repacked into the tiled kernel layout (row tiles of 128, K tiles of 64,
+ * gate and up rows interleaved). Synchronous: returns after the copy is
+ * complete; the caller may free its tensors afterwards. May be called again
+ * to replace the weights. */
+TFMOE_API tfmoe_status tfmoe_load_weights(tfmoe_layer *layer, const tfmoe_weights *w);
+
+/*
+ * out[T][H] = layer(x[T][H]); x and out are DEVICE pointers to bf16, rows of
+ * H contiguous elements, caller-owned; out must not overlap x.
+ * Stream-ordered on `cuda_stream` (a cudaStream_t; NULL = legacy default
+ * stream): returns after enqueueing, never synchronises the host, never
+ * allocates, and reads no device value on the host, so it may be captured
+ * in a CUDA graph. 0 <= T <= max_tokens; T == 0 launches nothing. One handle
+ * has one workspace: do not run two forwards of the same handle
+ * concurrently on different streams.
+ * Argument errors return before anything is enqueued. Launch errors return
+ * TFMOE_ERR_CUDA; faults inside kernels surface at the next synchronisation
+ * (for example tfmoe_sync_status).
+ */
+TFMOE_API tfmoe_status tfmoe_forward(tfmoe_layer *layer, const uint16_t *x, int32_t T,
+                           uint16_t *out, void *cuda_stream);
+
+/*
+ * Same computation with HOST buffers: x_host[T][H] is copied to the
+ * device, the layer runs, and the result is copied into out_host[T][H];
+ * all on `cuda_stream`, and the call returns after the result has arrived
+ * in out_host. Page-locked host buffers make the copies asynchronous to other
+ * host work; pageable buffers work too.
+ */
+TFMOE_API tfmoe_status tfmoe_forward_host(tfmoe_layer *layer, const uint16_t *x_host, int32_t T,
+                                uint16_t *out_host, void *cuda_stream);
+
+/* Synchronise `cuda_stream`, then report a pending CUDA error or the device
+ * error word that kernels with TFMOE_FLAG_DEBUG_CHECKS set (and clear it). */
+TFMOE_API tfmoe_status tfmoe_sync_status(tfmoe_layer *layer, void *cuda_stream);
+
+/* Free everything the handle owns. NULL is accepted. Synchronises the device. */
+TFMOE_API void tfmoe_destroy(tfmoe_layer *layer);
+
+/* Message of the last failing call on this host thread ("" if none). */
+TFMOE_API const char *tfmoe_last_error(void);
+
+/*
+ * Intermediate buffers of the last forward, for inspection (tests, tools).
+ * Returns a DEVICE pointer into the handle's workspace and its size in
+ * bytes; contents are valid after the forward has completed on its stream.
+ * Layouts (P = T*k pairs, rows of the permuted order r = 0..P-1, grouped by
+ * expert in ascending (expert, token, slot) order):
+ */
+typedef enum {
+    TFMOE_BUF_LOGITS = 0,     /* fp32 [T][E] router logits (bias included) */
+    TFMOE_BUF_TOPK_IDS = 1,   /* int32 [T][k] selected experts, slot 0 = largest logit */
+    TFMOE_BUF_TOPK_WEIGHTS = 2, /* fp32 [T][k] softmax weights over the selected logits */
+    TFMOE_BUF_EXPERT_COUNTS = 3, /* int32 [E] tokens routed to each expert */
+    TFMOE_BUF_EXPERT_OFFSETS = 4, /* int32 [E+1] exclusive prefix sum of the counts */
+    TFMOE_BUF_PERM = 5,       /* int32 [P] pair index t*k+s held by permuted row r */
+    TFMOE_BUF_INV = 6,        /* int32 [P] permuted row of pair t*k+s */
+    TFMOE_BUF_ACT = 7,        /* bf16 [P][I] SwiGLU output a, permuted rows */
+    TFMOE_BUF_EXPERT_OUT = 8, /* fp32 [P][H] down-projection output y, permuted rows */
+    TFMOE_BUF_REGIME = 9      /* int32 [E] 0 = not routed, 1 = GEMV regime, 2 = MMA regime */
+} tfmoe_buffer;
+
+TFMOE_API tfmoe_status tfmoe_get_buffer(tfmoe_layer *layer, tfmoe_buffer which, void **dev_ptr, size_t *bytes);
+
+/* Number of kernel launches the last tfmoe_forward enqueued. */
+TFMOE_API int32_t tfmoe_last_launch_count(tfmoe_layer *layer);
+
+/*
+ * Per-stage timing. While enabled, tfmoe_forward records a CUDA event pair on
+ * its stream around each stage below and, before returning, waits for the
+ * last one and adds the elapsed times to per-stage totals (so a profiled
+ * forward blocks the host and must not be graph-captured). tfmoe_profile_read
+ * copies the totals (milliseconds) and per-stage call counts into arrays of
+ * TFMOE_STAGE_COUNT entries and, if reset != 0, zeroes them.
+ */
+typedef enum {
+    TFMOE_STAGE_ROUTER = 0,       /* router logits */
+    TFMOE_STAGE_TOPK = 1,         /* top-k + softmax weights */
+    TFMOE_STAGE_PERMUTE = 2,      /* per-expert counts, offsets, permutation, regimes */
+    TFMOE_STAGE_GEMV_GATE_UP = 3, /* GEMV regime: gate/up projections + SwiGLU */
+    TFMOE_STAGE_GEMV_DOWN = 4,    /* GEMV regime: down projection */
+    TFMOE_STAGE_MMA_GATE_UP = 5,  /* tensor-core regime: gate/up projections + SwiGLU */
+    TFMOE_STAGE_MMA_DOWN = 6,     /* tensor-core regime: down projection */
+    TFMOE_STAGE_COMBINE = 7,      /* weighted combine */
+    TFMOE_STAGE_GATHER = 8,       /* tensor-core regime: activation row gather */
+    TFMOE_STAGE_COUNT = 9
+} tfmoe_stage;
+
+TFMOE_API tfmoe_status tfmoe_profile_enable(tfmoe_layer *layer, int32_t enable);
+TFMOE_API tfmoe_status tfmoe_profile_read(tfmoe_layer *layer, float *ms_total, int32_t *calls, int32_t reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TFMOE_H */

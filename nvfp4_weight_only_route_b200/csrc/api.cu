@@ -1,0 +1,360 @@
+// api.cu -- the C ABI of libtfmoe (declared in include/tfmoe.h): argument
+// validation, device memory ownership, and the stream-ordered launch chain
+// router -> top-k -> permute -> expert projections -> combine.
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "common.cuh"
+#include "internal.h"
+
+using namespace tfmoe;
+
+struct tfmoe_layer {
+    Layer impl;
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+tfmoe_status fail(tfmoe_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+tfmoe_status fail(tfmoe_status st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+tfmoe_status ok() { g_last_error.clear(); return TFMOE_OK; }
+
+tfmoe_status cuda_fail(cudaError_t e, const char *where) {
+    return fail(e == cudaErrorMemoryAllocation ? TFMOE_ERR_OOM : TFMOE_ERR_CUDA, "%s: %s (%s)", where,
+                cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Lays out `n` sub-buffers in one block; returns the total size.
+struct Carver {
+    size_t off = 0;
+    template <class T>
+    size_t take(T **slot, size_t count, uint8_t *base) {
+        off = align_up(off, 256);
+        if (base) *slot = reinterpret_cast<T *>(base + off);
+        const size_t at = off;
+        off += sizeof(T) * count;
+        return at;
+    }
+};
+
+void carve_workspace(Layer &L, uint8_t *base, size_t *total) {
+    const size_t T = L.desc.max_tokens, E = L.desc.num_experts, k = L.desc.top_k;
+    const size_t H = L.desc.hidden, I = L.desc.intermediate, P = T * k;
+    Workspace &w = L.ws;
+    Carver c;
+    c.take(&w.logits, T * E, base);
+    c.take(&w.ids, P, base);
+    c.take(&w.topk_w, P, base);
+    c.take(&w.counts, E, base);
+    c.take(&w.offsets, E + 1, base);
+    c.take(&w.perm, P, base);
+    c.take(&w.inv, P, base);
+    c.take(&w.regime, E, base);
+    c.take(&w.gemv_list, E, base);
+    c.take(&w.mma_list, E, base);
+    c.take(&w.list_sizes, 4, base);
+    c.take(&w.err_word, 1, base);
+    c.take(&w.act, P * I, base);
+    c.take(&w.y, P * H, base);
+    c.take(&w.x_stage, T * H, base);
+    c.take(&w.out_stage, T * H, base);
+    *total = align_up(c.off, 256);
+}
+
+void carve_weights(Layer &L, uint8_t *base, size_t *total) {
+    const size_t E = L.desc.num_experts, H = L.desc.hidden, I = L.desc.intermediate;
+    Weights &w = L.w;
+    Carver c;
+    c.take(&w.router_w, E * H, base);
+    c.take(&w.router_bias, E, base);
+    c.take(&w.gu_codes, E * 2 * I * H / 2, base);
+    c.take(&w.gu_scales, E * 2 * I * H / 16, base);
+    c.take(&w.d_codes, E * H * I / 2, base);
+    c.take(&w.d_scales, E * H * I / 16, base);
+    c.take(&w.gate_global, E, base);
+    c.take(&w.up_global, E, base);
+    c.take(&w.down_global, E, base);
+    *total = align_up(c.off, 256);
+}
+
+struct DeviceGuard {
+    int prev = -1;
+    bool changed = false;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) changed = (cudaSetDevice(dev) == cudaSuccess);
+    }
+    ~DeviceGuard() { if (changed) cudaSetDevice(prev); }
+};
+
+}  // namespace
+
+extern "C" {
+
+const char *tfmoe_last_error(void) { return g_last_error.c_str(); }
+
+tfmoe_status tfmoe_create(const tfmoe_layer_desc *desc, tfmoe_layer **out)
+{
+    if (!out) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_create: out is NULL");
+    *out = nullptr;
+    if (!desc) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_create: desc is NULL");
+    const tfmoe_layer_desc d = *desc;
+    if (d.hidden <= 0 || d.intermediate <= 0 || d.hidden % 16 || d.intermediate % 16)
+        return fail(TFMOE_ERR_INVALID_ARG, "hidden (%d) and intermediate (%d) must be positive multiples of 16",
+                    d.hidden, d.intermediate);
+    if (d.num_experts <= 0 || d.top_k <= 0 || d.top_k > d.num_experts)
+        return fail(TFMOE_ERR_INVALID_ARG, "need 1 <= top_k (%d) <= num_experts (%d)", d.top_k, d.num_experts);
+    if (d.max_tokens <= 0) return fail(TFMOE_ERR_INVALID_ARG, "max_tokens (%d) must be >= 1", d.max_tokens);
+    if ((d.flags & TFMOE_FLAG_FORCE_GEMV) && (d.flags & TFMOE_FLAG_FORCE_MMA))
+        return fail(TFMOE_ERR_INVALID_ARG, "FORCE_GEMV and FORCE_MMA are exclusive");
+    if (d.flags & ~(TFMOE_FLAG_FORCE_GEMV | TFMOE_FLAG_FORCE_MMA | TFMOE_FLAG_DEBUG_CHECKS))
+        return fail(TFMOE_ERR_INVALID_ARG, "unknown flag bits 0x%x", d.flags);
+    if (d.hidden % 128 || d.intermediate % 64)
+        return fail(TFMOE_ERR_UNSUPPORTED, "this build needs hidden %% 128 == 0 and intermediate %% 64 == 0 (got %d, %d)",
+                    d.hidden, d.intermediate);
+    if (d.num_experts > 256 || d.top_k > 32)
+        return fail(TFMOE_ERR_UNSUPPORTED, "this build supports num_experts <= 256 and top_k <= 32");
+    if ((long long)d.max_tokens * d.top_k > (1LL << 30))
+        return fail(TFMOE_ERR_UNSUPPORTED, "max_tokens * top_k too large");
+
+    const char *fail_env = getenv("TFMOE_FAIL_ALLOC");
+    if (fail_env && atoi(fail_env) != 0)
+        return fail(TFMOE_ERR_OOM, "tfmoe_create: allocation failure injected by TFMOE_FAIL_ALLOC");
+
+    tfmoe_layer *h = new (std::nothrow) tfmoe_layer();
+    if (!h) return fail(TFMOE_ERR_OOM, "tfmoe_create: host allocation failed");
+    Layer &L = h->impl;
+    L.desc = d;
+    L.gemv_max_tokens = d.gemv_max_tokens > 0 ? d.gemv_max_tokens : kDefaultGemvMaxTokens;
+    cudaError_t e = cudaGetDevice(&L.device);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&L.num_sms, cudaDevAttrMultiProcessorCount, L.device);
+    if (e != cudaSuccess) { delete h; return cuda_fail(e, "tfmoe_create: device query"); }
+
+    carve_workspace(L, nullptr, &L.ws_bytes);
+    carve_weights(L, nullptr, &L.w_bytes);
+    e = cudaMalloc(&L.ws_block, L.ws_bytes);
+    if (e == cudaSuccess) e = cudaMalloc(&L.w_block, L.w_bytes);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        if (L.ws_block) cudaFree(L.ws_block);
+        delete h;
+        return cuda_fail(e, "tfmoe_create: cudaMalloc");
+    }
+    carve_workspace(L, static_cast<uint8_t *>(L.ws_block), &L.ws_bytes);
+    carve_weights(L, static_cast<uint8_t *>(L.w_block), &L.w_bytes);
+    e = cudaMemset(L.ws.err_word, 0, sizeof(int32_t));
+    if (e == cudaSuccess) e = gemv_setup(L);
+    if (e != cudaSuccess) {
+        cudaFree(L.ws_block);
+        cudaFree(L.w_block);
+        delete h;
+        return cuda_fail(e, "tfmoe_create: setup");
+    }
+    *out = h;
+    return ok();
+}
+
+tfmoe_status tfmoe_load_weights(tfmoe_layer *layer, const tfmoe_weights *w)
+{
+    if (!layer || !w) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_load_weights: NULL argument");
+    Layer &L = layer->impl;
+    const void *req[] = {w->router_w, w->gate_codes, w->up_codes, w->gate_scales, w->up_scales, w->gate_global,
+                         w->up_global, w->down_codes, w->down_scales, w->down_global};
+    for (const void *p : req)
+        if (!p) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_load_weights: a required weight pointer is NULL");
+    if (L.desc.has_router_bias && !w->router_bias)
+        return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_load_weights: has_router_bias but router_bias is NULL");
+    const void *vec[] = {w->router_w, w->gate_codes, w->up_codes, w->down_codes};
+    for (const void *p : vec)
+        if (!aligned16(p)) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_load_weights: codes/router must be 16-byte aligned");
+    const void *sc[] = {w->gate_scales, w->up_scales, w->down_scales};
+    for (const void *p : sc)
+        if (reinterpret_cast<uintptr_t>(p) & 3u)
+            return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_load_weights: scales must be 4-byte aligned");
+
+    DeviceGuard dg(L.device);
+    const size_t E = L.desc.num_experts, H = L.desc.hidden;
+    cudaStream_t s;
+    cudaError_t e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return cuda_fail(e, "tfmoe_load_weights: stream");
+    e = cudaMemcpyAsync(L.w.router_w, w->router_w, E * H * 2, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess && L.desc.has_router_bias)
+        e = cudaMemcpyAsync(L.w.router_bias, w->router_bias, E * 4, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(L.w.gate_global, w->gate_global, E * 4, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(L.w.up_global, w->up_global, E * 4, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(L.w.down_global, w->down_global, E * 4, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess) e = launch_repack(L, *w, s);
+    cudaError_t e2 = cudaStreamSynchronize(s);
+    cudaStreamDestroy(s);
+    if (e == cudaSuccess) e = e2;
+    if (e != cudaSuccess) { L.loaded = false; return cuda_fail(e, "tfmoe_load_weights"); }
+    L.loaded = true;
+    return ok();
+}
+
+tfmoe_status tfmoe_forward(tfmoe_layer *layer, const uint16_t *x, int32_t T, uint16_t *out, void *cuda_stream)
+{
+    if (!layer) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward: layer is NULL");
+    Layer &L = layer->impl;
+    L.last_launches = 0;
+    if (!L.loaded) return fail(TFMOE_ERR_NOT_LOADED, "tfmoe_forward: weights not loaded");
+    if (T < 0 || T > L.desc.max_tokens)
+        return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward: T=%d outside [0, max_tokens=%d]", T, L.desc.max_tokens);
+    if (T == 0) return ok();
+    if (!x || !out) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward: x or out is NULL");
+    if (!aligned16(x) || !aligned16(out))
+        return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward: x and out must be 16-byte aligned");
+    const size_t bytes = (size_t)T * L.desc.hidden * 2;
+    const uintptr_t xa = reinterpret_cast<uintptr_t>(x), oa = reinterpret_cast<uintptr_t>(out);
+    if (xa < oa + bytes && oa < xa + bytes) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward: out overlaps x");
+
+    DeviceGuard dg(L.device);
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    int n = 0;
+    cudaError_t e = launch_router(L, x, T, s, &n);
+    if (e == cudaSuccess) e = launch_permute(L, T, s, &n);
+    if (e == cudaSuccess) e = launch_gemv(L, x, T, s, &n);
+    if (e == cudaSuccess) e = launch_combine(L, T, out, s, &n);
+    L.last_launches = n;
+    if (e != cudaSuccess) return cuda_fail(e, "tfmoe_forward: launch");
+    if (L.profiling) {
+        e = cudaStreamSynchronize(s);
+        for (int st = 0; st < TFMOE_STAGE_COUNT && e == cudaSuccess; ++st) {
+            if (!L.prof_used[st]) continue;
+            float ms = 0.f;
+            e = cudaEventElapsedTime(&ms, L.prof_ev[st][0], L.prof_ev[st][1]);
+            L.prof_ms[st] += ms;
+            L.prof_calls[st] += 1;
+            L.prof_used[st] = false;
+        }
+        if (e != cudaSuccess) return cuda_fail(e, "tfmoe_forward: profiling events");
+    }
+    return ok();
+}
+
+tfmoe_status tfmoe_forward_host(tfmoe_layer *layer, const uint16_t *x_host, int32_t T, uint16_t *out_host,
+                                void *cuda_stream)
+{
+    if (!layer) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward_host: layer is NULL");
+    Layer &L = layer->impl;
+    if (!L.loaded) return fail(TFMOE_ERR_NOT_LOADED, "tfmoe_forward_host: weights not loaded");
+    if (T < 0 || T > L.desc.max_tokens)
+        return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward_host: T=%d outside [0, max_tokens=%d]", T, L.desc.max_tokens);
+    if (T == 0) { L.last_launches = 0; return ok(); }
+    if (!x_host || !out_host) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward_host: NULL buffer");
+    DeviceGuard dg(L.device);
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    const size_t bytes = (size_t)T * L.desc.hidden * 2;
+    cudaError_t e = cudaMemcpyAsync(L.ws.x_stage, x_host, bytes, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "tfmoe_forward_host: copy in");
+    tfmoe_status st = tfmoe_forward(layer, L.ws.x_stage, T, L.ws.out_stage, cuda_stream);
+    if (st != TFMOE_OK) return st;
+    e = cudaMemcpyAsync(out_host, L.ws.out_stage, bytes, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "tfmoe_forward_host: copy out");
+    return ok();
+}
+
+tfmoe_status tfmoe_sync_status(tfmoe_layer *layer, void *cuda_stream)
+{
+    if (!layer) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_sync_status: layer is NULL");
+    Layer &L = layer->impl;
+    DeviceGuard dg(L.device);
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream));
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "tfmoe_sync_status");
+    int32_t word = 0;
+    e = cudaMemcpy(&word, L.ws.err_word, sizeof word, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && word != 0) e = cudaMemset(L.ws.err_word, 0, sizeof(int32_t));
+    if (e != cudaSuccess) return cuda_fail(e, "tfmoe_sync_status: error word");
+    if (word & DEV_ERR_WAIT_TIMEOUT) return fail(TFMOE_ERR_TIMEOUT, "a device-side wait timed out (word 0x%x)", word);
+    if (word) return fail(TFMOE_ERR_DEVICE, "device error word 0x%x (1 bad expert id, 2 bad row, 8 non-finite logit)", word);
+    return ok();
+}
+
+void tfmoe_destroy(tfmoe_layer *layer)
+{
+    if (!layer) return;
+    Layer &L = layer->impl;
+    {
+        DeviceGuard dg(L.device);
+        for (auto &pair : L.prof_ev)
+            for (auto &ev : pair)
+                if (ev) cudaEventDestroy(ev);
+        if (L.ws_block) cudaFree(L.ws_block);
+        if (L.w_block) cudaFree(L.w_block);
+    }
+    delete layer;
+}
+
+tfmoe_status tfmoe_get_buffer(tfmoe_layer *layer, tfmoe_buffer which, void **dev_ptr, size_t *bytes)
+{
+    if (!layer || !dev_ptr || !bytes) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_get_buffer: NULL argument");
+    Layer &L = layer->impl;
+    const size_t T = L.desc.max_tokens, E = L.desc.num_experts, k = L.desc.top_k;
+    const size_t H = L.desc.hidden, I = L.desc.intermediate, P = T * k;
+    switch (which) {
+    case TFMOE_BUF_LOGITS: *dev_ptr = L.ws.logits; *bytes = T * E * 4; break;
+    case TFMOE_BUF_TOPK_IDS: *dev_ptr = L.ws.ids; *bytes = P * 4; break;
+    case TFMOE_BUF_TOPK_WEIGHTS: *dev_ptr = L.ws.topk_w; *bytes = P * 4; break;
+    case TFMOE_BUF_EXPERT_COUNTS: *dev_ptr = L.ws.counts; *bytes = E * 4; break;
+    case TFMOE_BUF_EXPERT_OFFSETS: *dev_ptr = L.ws.offsets; *bytes = (E + 1) * 4; break;
+    case TFMOE_BUF_PERM: *dev_ptr = L.ws.perm; *bytes = P * 4; break;
+    case TFMOE_BUF_INV: *dev_ptr = L.ws.inv; *bytes = P * 4; break;
+    case TFMOE_BUF_ACT: *dev_ptr = L.ws.act; *bytes = P * I * 2; break;
+    case TFMOE_BUF_EXPERT_OUT: *dev_ptr = L.ws.y; *bytes = P * H * 4; break;
+    case TFMOE_BUF_REGIME: *dev_ptr = L.ws.regime; *bytes = E * 4; break;
+    default: return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_get_buffer: unknown buffer %d", (int)which);
+    }
+    return ok();
+}
+
+int32_t tfmoe_last_launch_count(tfmoe_layer *layer) { return layer ? layer->impl.last_launches : 0; }
+
+tfmoe_status tfmoe_profile_enable(tfmoe_layer *layer, int32_t enable)
+{
+    if (!layer) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_profile_enable: layer is NULL");
+    Layer &L = layer->impl;
+    DeviceGuard dg(L.device);
+    if (enable && !L.prof_ev[0][0]) {
+        for (auto &pair : L.prof_ev)
+            for (auto &ev : pair) {
+                cudaError_t e = cudaEventCreate(&ev);
+                if (e != cudaSuccess) return cuda_fail(e, "tfmoe_profile_enable");
+            }
+    }
+    L.profiling = enable != 0;
+    return ok();
+}
+
+tfmoe_status tfmoe_profile_read(tfmoe_layer *layer, float *ms_total, int32_t *calls, int32_t reset)
+{
+    if (!layer || !ms_total || !calls) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_profile_read: NULL argument");
+    Layer &L = layer->impl;
+    for (int st = 0; st < TFMOE_STAGE_COUNT; ++st) {
+        ms_total[st] = L.prof_ms[st];
+        calls[st] = L.prof_calls[st];
+        if (reset) { L.prof_ms[st] = 0.f; L.prof_calls[st] = 0; }
+    }
+    return ok();
+}
+
+}  // extern "C"

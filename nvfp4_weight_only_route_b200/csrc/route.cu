@@ -1,0 +1,350 @@
+// route.cu -- router logits, top-k + softmax weights, and the expert
+// permutation ("plan") of the MoE layer.
+//
+// Router and top-k are the first two launches of the MoE chain in
+// TensorFold issue #627 (per-launch kernel table: router, topk); the pages'
+// fused one-block router was slower because it serialised a row's expert dot
+// products on one SM (issue #627, comment on tf_nemo_route_row), so the
+// logits here keep a wide grid: one warp per (expert, token group) for
+// decode-sized T, a 64x64 register-tiled kernel for large T.
+//
+// Logits are the fp64 sum of exact bf16*bf16 products rounded once to fp32,
+// then plus the fp32 bias: this makes the top-k ids bit-reproducible against
+// a float64 reference (issue #627, "Description": error stated against a
+// 64-bit reference).
+#include "common.cuh"
+#include "internal.h"
+
+namespace tfmoe {
+namespace {
+
+constexpr int kSmallTokens = 8;     // tokens per warp in the small-T router kernel
+
+// One warp per (expert, group of <= 8 tokens). Lane l covers 8 consecutive
+// columns per 256-column step.
+__global__ void __launch_bounds__(128) router_small_kernel(
+    const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, const float *__restrict__ bias,
+    float *__restrict__ logits, int T, int H, int E, int32_t *err_word, int debug)
+{
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int n_groups = (T + kSmallTokens - 1) / kSmallTokens;
+    if (warp >= E * n_groups) return;
+    const int e = warp % E;
+    const int t0 = (warp / E) * kSmallTokens;
+    const int nt = min(kSmallTokens, T - t0);
+    double acc[kSmallTokens];
+#pragma unroll
+    for (int i = 0; i < kSmallTokens; ++i) acc[i] = 0.0;
+    const uint16_t *wrow = wr + (size_t)e * H;
+    for (int c = lane * 8; c < H; c += 256) {
+        uint4 wv = *reinterpret_cast<const uint4 *>(wrow + c);
+        double w[8];
+        const uint32_t wu[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            w[2 * i] = (double)bf16_bits_to_float(wu[i] & 0xFFFFu);
+            w[2 * i + 1] = (double)bf16_bits_to_float(wu[i] >> 16);
+        }
+#pragma unroll
+        for (int t = 0; t < kSmallTokens; ++t) {
+            if (t < nt) {
+                uint4 xv = *reinterpret_cast<const uint4 *>(x + (size_t)(t0 + t) * H + c);
+                const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    acc[t] = fma((double)bf16_bits_to_float(xu[i] & 0xFFFFu), w[2 * i], acc[t]);
+                    acc[t] = fma((double)bf16_bits_to_float(xu[i] >> 16), w[2 * i + 1], acc[t]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < kSmallTokens; ++t) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+    }
+    if (lane < nt) {
+        double v = acc[0];
+#pragma unroll
+        for (int t = 1; t < kSmallTokens; ++t)
+            if (lane == t) v = acc[t];
+        float l = (float)v;
+        if (bias) l = l + bias[e];
+        if (debug && !isfinite(l)) atomicOr(err_word, DEV_ERR_NONFINITE);
+        logits[(size_t)(t0 + lane) * E + e] = l;
+    }
+}
+
+// 64 tokens x 64 experts per CTA, 256 threads, 4x4 fp64 accumulators per
+// thread, K staged through shared memory in steps of 32 (converted to fp64).
+constexpr int RT_T = 64, RT_E = 64, RT_K = 32;
+__global__ void __launch_bounds__(256) router_tiled_kernel(
+    const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, const float *__restrict__ bias,
+    float *__restrict__ logits, int T, int H, int E, int32_t *err_word, int debug)
+{
+    __shared__ double xs[RT_K][RT_T + 1];
+    __shared__ double ws[RT_K][RT_E + 1];
+    const int t_base = blockIdx.x * RT_T, e_base = blockIdx.y * RT_E;
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    double acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+    for (int k0 = 0; k0 < H; k0 += RT_K) {
+        // 64 rows x 32 columns of x and of wr: 2048 elements each, 8 per thread.
+        for (int i = threadIdx.x; i < RT_T * RT_K / 8; i += 256) {
+            const int row = i / (RT_K / 8), col = (i % (RT_K / 8)) * 8;
+            const int t = t_base + row, e = e_base + row;
+            uint4 xv = make_uint4(0, 0, 0, 0), wv = make_uint4(0, 0, 0, 0);
+            if (t < T) xv = *reinterpret_cast<const uint4 *>(x + (size_t)t * H + k0 + col);
+            if (e < E) wv = *reinterpret_cast<const uint4 *>(wr + (size_t)e * H + k0 + col);
+            const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w}, wu[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                xs[col + 2 * j][row] = (double)bf16_bits_to_float(xu[j] & 0xFFFFu);
+                xs[col + 2 * j + 1][row] = (double)bf16_bits_to_float(xu[j] >> 16);
+                ws[col + 2 * j][row] = (double)bf16_bits_to_float(wu[j] & 0xFFFFu);
+                ws[col + 2 * j + 1][row] = (double)bf16_bits_to_float(wu[j] >> 16);
+            }
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int kk = 0; kk < RT_K; ++kk) {
+            double xv[4], wv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) xv[i] = xs[kk][ty + 16 * i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) wv[j] = ws[kk][tx + 16 * j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fma(xv[i], wv[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int t = t_base + ty + 16 * i;
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int e = e_base + tx + 16 * j;
+            if (e >= E) continue;
+            float l = (float)acc[i][j];
+            if (bias) l = l + bias[e];
+            if (debug && !isfinite(l)) atomicOr(err_word, DEV_ERR_NONFINITE);
+            logits[(size_t)t * E + e] = l;
+        }
+    }
+}
+
+// One warp per token: k rounds of a warp arg-max over (logit desc, index asc),
+// then softmax over the selected logits (max-subtracted, fp32).
+constexpr int kMaxEPerLane = 8;   // E <= 256
+__global__ void __launch_bounds__(256) topk_kernel(
+    const float *__restrict__ logits, int32_t *__restrict__ ids, float *__restrict__ wts,
+    int T, int E, int k)
+{
+    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (t >= T) return;
+    float v[kMaxEPerLane];
+    const float *row = logits + (size_t)t * E;
+#pragma unroll
+    for (int i = 0; i < kMaxEPerLane; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = (e < E) ? row[e] : -INFINITY;
+    }
+    uint32_t taken = 0;
+    float sel_first = 0.f, my_sel = 0.f;
+    int my_id = -1;
+    for (int s = 0; s < k; ++s) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < kMaxEPerLane; ++i) {
+            const int e = lane + 32 * i;
+            if (e < E && !(taken & (1u << i)) && (v[i] > bv || (v[i] == bv && e < bi) || bi == 0x7fffffff)) {
+                bv = v[i];
+                bi = e;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        if (s == 0) sel_first = bv;
+        if (lane == s) { my_sel = bv; my_id = bi; }
+    }
+    // softmax over the k selected logits (slot order), fp32
+    const float ex = (lane < k) ? expf(my_sel - sel_first) : 0.f;
+    float den = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (lane < k) {
+        ids[(size_t)t * k + lane] = my_id;
+        wts[(size_t)t * k + lane] = ex / den;
+    }
+}
+
+// Single CTA of 32 warps. Pairs p = t*k + s are split into 32 contiguous
+// segments, one per warp. Pass 1 counts per (segment, expert); a scan turns
+// the counts into per-expert offsets and per-segment bases; pass 2 places each
+// pair at base + its rank among same-expert pairs of the segment, so rows are
+// ordered by (expert, pair index) -- a stable counting sort.
+constexpr int kPermWarps = 32;
+__global__ void __launch_bounds__(1024) permute_kernel(
+    const int32_t *__restrict__ ids, int P, int E, int gemv_max_tokens, uint32_t flags,
+    int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
+    int32_t *__restrict__ inv, int32_t *__restrict__ regime, int32_t *__restrict__ gemv_list,
+    int32_t *__restrict__ mma_list, int32_t *__restrict__ list_sizes, int32_t *err_word, int debug)
+{
+    extern __shared__ int32_t sm[];
+    int32_t *cnt = sm;                       // [32][E]
+    int32_t *tot = sm + kPermWarps * E;      // [E]
+    int32_t *off = tot + E;                  // [E+1]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) cnt[i] = 0;
+    __syncthreads();
+    const int seg = (P + kPermWarps - 1) / kPermWarps;
+    const int p_begin = min(P, warp * seg), p_end = min(P, p_begin + seg);
+    int32_t *my_cnt = cnt + warp * E;
+    for (int p0 = p_begin; p0 < p_end; p0 += 32) {
+        const int p = p0 + lane;
+        int e = (p < p_end) ? ids[p] : -1;
+        if (e >= E || (e < 0 && p < p_end)) {
+            if (debug) atomicOr(err_word, DEV_ERR_BAD_EXPERT);
+            e = -1;
+        }
+        const uint32_t m = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && lane == __ffs(m) - 1) my_cnt[e] += __popc(m);
+        __syncwarp();
+    }
+    __syncthreads();
+    // per-expert totals and per-segment bases (exclusive over segments)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = 0;
+        for (int w = 0; w < kPermWarps; ++w) {
+            const int c = cnt[w * E + e];
+            cnt[w * E + e] = run;
+            run += c;
+        }
+        tot[e] = run;
+    }
+    __syncthreads();
+    if (warp == 0) {   // exclusive scan of tot over experts, E <= 256: 8 per lane
+        int local[8], s = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane * 8 + i;
+            local[i] = (e < E) ? tot[e] : 0;
+            s += local[i];
+        }
+        int incl = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - s;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane * 8 + i;
+            if (e < E) off[e] = run;
+            run += local[i];
+        }
+        if (lane == 31) off[E] = incl;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) cnt[i] += off[i % E];
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets[e] = off[e];
+    __syncthreads();
+    for (int p0 = p_begin; p0 < p_end; p0 += 32) {
+        const int p = p0 + lane;
+        int e = (p < p_end) ? ids[p] : -1;
+        if (e >= E) e = -1;
+        const uint32_t m = __match_any_sync(0xffffffffu, e);
+        if (e >= 0) {
+            const int rank = __popc(m & ((1u << lane) - 1u));
+            const int r = my_cnt[e] + rank;
+            perm[r] = p;
+            inv[p] = r;
+        }
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(m) - 1) my_cnt[e] += __popc(m);
+        __syncwarp();
+    }
+    // regimes and compacted expert lists (ascending expert order)
+    if (warp == 0) {
+        int n_gemv = 0, n_mma = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            const int m = (e < E) ? tot[e] : 0;
+            int reg = 0;
+            if (m > 0) {
+                if (flags & TFMOE_FLAG_FORCE_GEMV) reg = 1;
+                else if (flags & TFMOE_FLAG_FORCE_MMA) reg = 2;
+                else reg = (m <= gemv_max_tokens) ? 1 : 2;
+            }
+            if (e < E) { regime[e] = reg; counts[e] = m; }
+            const uint32_t bg = __ballot_sync(0xffffffffu, reg == 1);
+            const uint32_t bm = __ballot_sync(0xffffffffu, reg == 2);
+            const uint32_t lt = (1u << lane) - 1u;
+            if (reg == 1) gemv_list[n_gemv + __popc(bg & lt)] = e;
+            if (reg == 2) mma_list[n_mma + __popc(bm & lt)] = e;
+            n_gemv += __popc(bg);
+            n_mma += __popc(bm);
+        }
+        if (lane == 0) { list_sizes[0] = n_gemv; list_sizes[1] = n_mma; }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_router(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches)
+{
+    const int H = L.desc.hidden, E = L.desc.num_experts, k = L.desc.top_k;
+    const int debug = (L.desc.flags & TFMOE_FLAG_DEBUG_CHECKS) ? 1 : 0;
+    const float *bias = L.desc.has_router_bias ? L.w.router_bias : nullptr;
+    {
+    StageTimer timer(L, TFMOE_STAGE_ROUTER, s);
+    if (T <= 2 * kSmallTokens) {
+        const int warps = E * ((T + kSmallTokens - 1) / kSmallTokens);
+        router_small_kernel<<<(warps + 3) / 4, 128, 0, s>>>(x, L.w.router_w, bias, L.ws.logits, T, H, E,
+                                                           L.ws.err_word, debug);
+    } else {
+        dim3 grid((T + RT_T - 1) / RT_T, (E + RT_E - 1) / RT_E);
+        router_tiled_kernel<<<grid, 256, 0, s>>>(x, L.w.router_w, bias, L.ws.logits, T, H, E,
+                                                  L.ws.err_word, debug);
+    }
+    }
+    {
+        StageTimer timer(L, TFMOE_STAGE_TOPK, s);
+        topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(L.ws.logits, L.ws.ids, L.ws.topk_w, T, E, k);
+    }
+    *launches += 2;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_permute(Layer &L, int T, cudaStream_t s, int *launches)
+{
+    StageTimer timer(L, TFMOE_STAGE_PERMUTE, s);
+    const int E = L.desc.num_experts, P = T * L.desc.top_k;
+    const int debug = (L.desc.flags & TFMOE_FLAG_DEBUG_CHECKS) ? 1 : 0;
+    const size_t smem = sizeof(int32_t) * ((size_t)kPermWarps * E + 2 * E + 1);
+    permute_kernel<<<1, 1024, smem, s>>>(L.ws.ids, P, E, L.gemv_max_tokens, L.desc.flags, L.ws.counts,
+                                          L.ws.offsets, L.ws.perm, L.ws.inv, L.ws.regime, L.ws.gemv_list,
+                                          L.ws.mma_list, L.ws.list_sizes, L.ws.err_word, debug);
+    *launches += 1;
+    return cudaGetLastError();
+}
+
+}  // namespace tfmoe

@@ -38,7 +38,7 @@ class _Layer(ctypes.Structure):
 class _Outputs(ctypes.Structure):
     _fields_ = [("out", _u16p), ("out64", _f64p), ("S", _f64p), ("logits", _f32p),
                 ("ids", _i32p), ("g", _f64p), ("G", _f32p), ("U", _f32p),
-                ("a", _u16p), ("y", _f64p)]
+                ("a", _u16p), ("y", _f64p), ("yabs", _f64p)]
 
 
 def build(force: bool = False) -> str:
@@ -134,11 +134,11 @@ def forward(layer: Dict[str, Optional[np.ndarray]], x: np.ndarray, *, top_k: int
         res.update(logits=np.zeros((T, E), np.float32), ids=np.zeros((T, top_k), np.int32),
                    g=np.zeros((T, top_k), np.float64), G=np.zeros((T, top_k, I), np.float32),
                    U=np.zeros((T, top_k, I), np.float32), a=np.zeros((T, top_k, I), np.uint16),
-                   y=np.zeros((T, top_k, H), np.float64))
+                   y=np.zeros((T, top_k, H), np.float64), yabs=np.zeros((T, top_k, H), np.float64))
     O = _Outputs(_ptr(res["out"], _u16p), _ptr(res["out64"], _f64p), _ptr(res["S"], _f64p),
                  _ptr(res.get("logits"), _f32p), _ptr(res.get("ids"), _i32p),
                  _ptr(res.get("g"), _f64p), _ptr(res.get("G"), _f32p), _ptr(res.get("U"), _f32p),
-                 _ptr(res.get("a"), _u16p), _ptr(res.get("y"), _f64p))
+                 _ptr(res.get("a"), _u16p), _ptr(res.get("y"), _f64p), _ptr(res.get("yabs"), _f64p))
     rc = lib().oracle_forward(ctypes.byref(L), _ptr(x, _u16p), T, nthreads, ctypes.byref(O))
     if rc != 0:
         raise RuntimeError(f"oracle_forward failed with code {rc}")

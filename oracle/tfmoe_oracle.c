@@ -139,6 +139,7 @@ typedef struct {
     float *G, *U;       /* [T][k][I] */
     uint16_t *a;        /* bf16 [T][k][I] */
     double *y;          /* [T][k][H] */
+    double *yabs;       /* [T][k][H] sum_j |a[j] * deq(Wd)[h][j]| */
 } oracle_outputs;
 
 /* Router logits, top-k (ties to the lower expert index) and the softmax
@@ -285,6 +286,7 @@ int oracle_forward(const oracle_layer *L, const uint16_t *x, int32_t T, int32_t 
     if (O->g) memcpy(O->g, g, sizeof(double) * P);
     if (O->a) memcpy(O->a, a, sizeof(uint16_t) * P * I);
     if (O->y) memcpy(O->y, y, sizeof(double) * P * H);
+    if (O->yabs) memcpy(O->yabs, yabs, sizeof(double) * P * H);
 
     free(logits); free(ids); free(g); free(a); free(y); free(yabs); free(xd);
     free(count); free(start); free(pairs);

@@ -1,0 +1,237 @@
+"""CUDA path vs the fp64 oracle, through the C ABI (needs a B200).
+
+Routing must match bit-exactly; every output element must satisfy
+|gpu - oracle| <= 4e-3 * S + 1e-3 with S = sum_s g_s * sum_j |a_s[j] * w[h,j]|.
+Small layers are compared in full; the full-size prefill and large layers
+on a seeded sample of tokens (each token's output depends only on its own row).
+"""
+import numpy as np
+import pytest
+
+from nvfp4_weight_only_route_b200 import synth
+
+from gpu_harness import GpuRun, check_intermediates, check_output, check_routing
+
+pytestmark = pytest.mark.gpu
+
+REGIMES = {"gemv": 1}          # flag values: FORCE_GEMV = 1
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from nvfp4_weight_only_route_b200 import build
+    build.build()
+
+
+def _full_check(oracle_mod, layer, x, H, I, E, k, flags, max_tokens=None):
+    T = x.shape[0]
+    run = GpuRun(layer, H, I, E, k, max_tokens or max(T, 1), flags=flags)
+    try:
+        g = run.forward(x)
+    finally:
+        run.close()
+    o = oracle_mod.forward(layer, x, top_k=k, intermediates=True)
+    check_routing(g, o, E, k)
+    check_intermediates(g, o, k)
+    return check_output(g["out"], o)
+
+
+@pytest.mark.parametrize("regime", sorted(REGIMES))
+def test_tiny_layer(oracle_mod, regime):
+    s = synth.SHAPES[0]
+    layer = synth.make_layer(s, 0)
+    x = synth.make_x(s, 0, 4)
+    _full_check(oracle_mod, layer, x, s.H, s.I, s.E, s.k, REGIMES[regime])
+
+
+@pytest.mark.parametrize("regime", sorted(REGIMES))
+@pytest.mark.parametrize("seed", [1, 2, 3])
+def test_decode_layer(oracle_mod, seed, regime):
+    s = synth.SHAPES[1]
+    layer = synth.make_layer(s, seed)
+    for T in s.T:
+        x = synth.make_x(s, seed, T)
+        _full_check(oracle_mod, layer, x, s.H, s.I, s.E, s.k, REGIMES[regime])
+
+
+@pytest.mark.parametrize("regime", sorted(REGIMES))
+def test_batched_decode_zipf(oracle_mod, regime):
+    s = synth.SHAPES[2]
+    layer = synth.make_layer(s, 4)
+    x = synth.make_x(s, 4, 256)
+    _full_check(oracle_mod, layer, x, s.H, s.I, s.E, s.k, REGIMES[regime])
+
+
+@pytest.mark.parametrize("regime", sorted(REGIMES))
+@pytest.mark.parametrize("H,I,E,k,T", [
+    (384, 192, 6, 3, 1),       # 3 row tiles, 3 K tiles, ragged everything
+    (384, 192, 6, 3, 37),
+    (256, 320, 5, 2, 100),
+    (128, 64, 4, 1, 9),        # smallest supported tile counts
+    (512, 128, 8, 8, 13),      # k == E: every expert selected
+])
+def test_ragged_shapes(oracle_mod, regime, H, I, E, k, T):
+    shape = synth.custom_shape(H, I, E, k, global_scale=0.05, router_std=1.0)
+    layer = synth.make_layer(shape, 100 + T)
+    x = synth.make_x(shape, 100 + T, T)
+    _full_check(oracle_mod, layer, x, H, I, E, k, REGIMES[regime])
+
+
+@pytest.mark.parametrize("regime", sorted(REGIMES))
+def test_single_expert_holds_every_token(oracle_mod, regime):
+    H, I, E, k, T = 256, 128, 8, 2, 40
+    shape = synth.custom_shape(H, I, E, k, global_scale=0.05, router_std=0.02)
+    layer = synth.make_layer(shape, 7)
+    bias = np.zeros(E, np.float32)
+    bias[5] = 1000.0
+    layer["router_bias"] = bias
+    x = synth.make_x(shape, 7, T)
+    _full_check(oracle_mod, layer, x, H, I, E, k, REGIMES[regime])
+
+
+@pytest.mark.parametrize("regime", sorted(REGIMES))
+def test_exact_logit_ties(oracle_mod, regime):
+    H, I, E, k, T = 256, 128, 8, 3, 16
+    shape = synth.custom_shape(H, I, E, k, global_scale=0.05, router_std=1.0)
+    layer = synth.make_layer(shape, 8)
+    rw = layer["router_w"].copy()
+    rw[2] = rw[6] = rw[1]                 # three identical router rows: exact ties
+    layer["router_w"] = rw
+    x = synth.make_x(shape, 8, T)
+    o = oracle_mod.forward(layer, x, top_k=k, intermediates=True)
+    assert any(len({1, 2, 6} & set(r.tolist())) >= 2 for r in o["ids"]), "fixture should produce ties"
+    _full_check(oracle_mod, layer, x, H, I, E, k, REGIMES[regime])
+
+
+def test_zero_tokens_launches_nothing(oracle_mod):
+    import torch
+    s = synth.SHAPES[0]
+    run = GpuRun(synth.make_layer(s, 0), s.H, s.I, s.E, s.k, 4)
+    try:
+        x = torch.zeros((1, s.H), dtype=torch.int16, device="cuda")
+        out = torch.full((1, s.H), 7, dtype=torch.int16, device="cuda")
+        run.layer.forward(x, out, T=0)
+        assert run.layer.last_launch_count() == 0
+        assert int(out[0, 0]) == 7
+    finally:
+        run.close()
+
+
+def test_max_tokens_and_over_limit(oracle_mod):
+    import torch
+    from nvfp4_weight_only_route_b200 import tfmoe
+    s = synth.SHAPES[0]
+    layer = synth.make_layer(s, 0)
+    x = synth.make_x(s, 0, 6)
+    _full_check(oracle_mod, layer, x, s.H, s.I, s.E, s.k, 0, max_tokens=6)
+    run = GpuRun(layer, s.H, s.I, s.E, s.k, 6)
+    try:
+        xt = torch.zeros((7, s.H), dtype=torch.int16, device="cuda")
+        out = torch.zeros((7, s.H), dtype=torch.int16, device="cuda")
+        with pytest.raises(tfmoe.TfmoeError) as ei:
+            run.layer.forward(xt, out, T=7)
+        assert ei.value.status == tfmoe.ERR_INVALID_ARG
+        with pytest.raises(tfmoe.TfmoeError) as ei:
+            run.layer.forward(xt, xt, T=2)          # out overlaps x
+        assert ei.value.status == tfmoe.ERR_INVALID_ARG
+        with pytest.raises(tfmoe.TfmoeError) as ei:   # misaligned x
+            tfmoe.check(run.layer.forward_raw(xt.data_ptr() + 2, 1, out.data_ptr(), 0))
+        assert ei.value.status == tfmoe.ERR_INVALID_ARG
+    finally:
+        run.close()
+
+
+def test_forward_before_load_is_rejected():
+    import torch
+    from nvfp4_weight_only_route_b200 import tfmoe
+    L = tfmoe.MoELayer(128, 64, 4, 1, 4)
+    try:
+        x = torch.zeros((1, 128), dtype=torch.int16, device="cuda")
+        with pytest.raises(tfmoe.TfmoeError) as ei:
+            L.forward(x, torch.zeros_like(x))
+        assert ei.value.status == tfmoe.ERR_NOT_LOADED
+    finally:
+        L.close()
+
+
+def test_deterministic_bytes(oracle_mod):
+    s = synth.SHAPES[2]
+    layer = synth.make_layer(s, 4)
+    x = synth.make_x(s, 4, 256)
+    run = GpuRun(layer, s.H, s.I, s.E, s.k, 256)
+    try:
+        a = run.forward(x, intermediates=False)["out"]
+        b = run.forward(x, intermediates=False)["out"]
+    finally:
+        run.close()
+    assert a.tobytes() == b.tobytes()
+
+
+def test_forward_host_matches_device(oracle_mod):
+    import torch
+    s = synth.SHAPES[1]
+    layer = synth.make_layer(s, 1)
+    x = synth.make_x(s, 1, 8)
+    run = GpuRun(layer, s.H, s.I, s.E, s.k, 8)
+    try:
+        dev = run.forward(x, intermediates=False)["out"]
+        xh = torch.from_numpy(x.view(np.int16)).pin_memory()
+        oh = torch.empty((8, s.H), dtype=torch.int16).pin_memory()
+        run.layer.forward_host(xh, oh)
+        assert np.array_equal(oh.numpy().view(np.uint16), dev)
+    finally:
+        run.close()
+
+
+def test_debug_checks_report_clean(oracle_mod):
+    s = synth.SHAPES[1]
+    layer = synth.make_layer(s, 2)
+    x = synth.make_x(s, 2, 8)
+    run = GpuRun(layer, s.H, s.I, s.E, s.k, 8, flags=4)
+    try:
+        g = run.forward(x)
+    finally:
+        run.close()
+    o = oracle_mod.forward(layer, x, top_k=s.k, intermediates=True)
+    check_routing(g, o, s.E, s.k)
+    check_output(g["out"], o)
+
+
+def _sampled_check(oracle_mod, run, layer, x, k, n_sample, seed):
+    T = x.shape[0]
+    g = run.forward(x, intermediates=True)
+    rng = np.random.default_rng(seed)
+    idx = np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=min(T, n_sample), replace=False)]))
+    o = oracle_mod.forward(layer, x[idx], top_k=k, intermediates=True)
+    assert np.array_equal(g["ids"][idx], o["ids"])
+    assert np.array_equal(g["logits"][idx], o["logits"])
+    # every pair's row is where the permutation says, and the counts add up
+    assert g["counts"].sum() == T * k and np.array_equal(np.sort(g["perm"]), np.arange(T * k))
+    assert np.array_equal(g["inv"][g["perm"]], np.arange(T * k))
+    return check_output(g["out"][idx], o)
+
+
+def test_prefill_layer_sampled(oracle_mod):
+    s = synth.SHAPES[3]
+    layer = synth.make_layer(s, 5)
+    x = synth.make_x(s, 5, 8192)
+    run = GpuRun(layer, s.H, s.I, s.E, s.k, 8192)
+    try:
+        _sampled_check(oracle_mod, run, layer, x, s.k, 24, 5)
+    finally:
+        run.close()
+
+
+def test_large_layer_sweep_sampled(oracle_mod):
+    s = synth.SHAPES[4]
+    layer = synth.make_layer(s, 6)
+    run = GpuRun(layer, s.H, s.I, s.E, s.k, max(s.T))
+    try:
+        for T in s.T:
+            x = synth.make_x(s, 6, T)
+            _sampled_check(oracle_mod, run, layer, x, s.k, 8, T)
+    finally:
+        run.close()
