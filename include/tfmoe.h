@@ -203,6 +203,41 @@ typedef enum {
 TFMOE_API tfmoe_status tfmoe_profile_enable(tfmoe_layer *layer, int32_t enable);
 TFMOE_API tfmoe_status tfmoe_profile_read(tfmoe_layer *layer, float *ms_total, int32_t *calls, int32_t reset);
 
+/*
+ * Routing without any allocation (the pages describe no such entry point;
+ * it exists for callers of this library that cannot allocate device memory:
+ * code running while another component owns the whole memory budget through a
+ * fixed pool, real-time loops that must not pay cudaMalloc's latency or its
+ * implicit device synchronisation, and hosts whose rules forbid allocating
+ * after start-up). It computes what tfmoe_forward computes for routing -- the
+ * router logits (fp64-accumulated, rounded to fp32, plus the optional bias),
+ * the top_k expert ids (ties to the lower index) and the softmax weights over
+ * the selected logits -- without a tfmoe_layer handle and without calling
+ * cudaMalloc, cudaFree or any allocating routine.
+ *
+ * The fp32 logits live in a fixed scratch array compiled into the library:
+ * TFMOE_ROUTE_NOALLOC_MAX_LOGITS floats (4 MiB) on every GPU that loads it,
+ * held until the process exits. T * num_experts above that limit returns
+ * TFMOE_ERR_INVALID_ARG and launches nothing; split the batch instead.
+ * Every call on a device shares that one array and leaves its logits in it:
+ * calls whose work overlaps on the GPU (two streams, or two host threads)
+ * race on it and must be serialised by the caller. Each call overwrites every
+ * logit it reads, so nothing needs clearing between calls.
+ * The first call on each device looks up the array's device address with
+ * that device current; make that first call before any stream capture.
+ *
+ * Arguments (DEVICE pointers, caller-owned): x bf16 [T][hidden] and router_w
+ * bf16 [num_experts][hidden], both 16-byte aligned; router_bias fp32
+ * [num_experts] or NULL; outputs ids_out int32 [T][top_k] and weights_out fp32
+ * [T][top_k]. hidden must be a positive multiple of 32, 1 <= top_k <= 32,
+ * top_k <= num_experts <= 256. Stream-ordered on cuda_stream; T == 0 is a no-op.
+ */
+#define TFMOE_ROUTE_NOALLOC_MAX_LOGITS (1 << 20)
+TFMOE_API tfmoe_status tfmoe_route_noalloc(const uint16_t *x, int32_t T, int32_t hidden,
+                                           const uint16_t *router_w, const float *router_bias,
+                                           int32_t num_experts, int32_t top_k,
+                                           int32_t *ids_out, float *weights_out, void *cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

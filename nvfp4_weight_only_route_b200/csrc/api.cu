@@ -107,6 +107,19 @@ struct DeviceGuard {
 
 }  // namespace
 
+namespace tfmoe {
+tfmoe_status record_error(tfmoe_status st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+tfmoe_status record_ok() { return ok(); }
+}  // namespace tfmoe
+
 extern "C" {
 
 const char *tfmoe_last_error(void) { return g_last_error.c_str(); }

@@ -96,4 +96,8 @@ cudaError_t launch_combine(Layer &L, int T, uint16_t *out, cudaStream_t s, int *
 cudaError_t launch_repack(const Layer &L, const tfmoe_weights &src, cudaStream_t s);
 cudaError_t gemv_setup(Layer &L);
 
+// Sets the thread-local message returned by tfmoe_last_error() and returns st.
+tfmoe_status record_error(tfmoe_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+tfmoe_status record_ok();
+
 }  // namespace tfmoe

@@ -12,6 +12,8 @@
 // then plus the fp32 bias: this makes the top-k ids bit-reproducible against
 // a float64 reference (issue #627, "Description": error stated against a
 // 64-bit reference).
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -348,3 +350,84 @@ cudaError_t launch_permute(Layer &L, int T, cudaStream_t s, int *launches)
 }
 
 }  // namespace tfmoe
+
+// ---------------------------------------------------------------------------
+// Allocation-free routing for callers that cannot allocate device memory
+// (tfmoe_route_noalloc in tfmoe.h). The router logits go to a fixed array
+// compiled into the library instead of a workspace: every GPU that loads the
+// library holds TFMOE_ROUTE_NOALLOC_MAX_LOGITS floats of it until exit, and all
+// calls on a device share it, so calls that overlap on the GPU race.
+namespace tfmoe {
+namespace {
+
+static __device__ __align__(256) float g_noalloc_logits[TFMOE_ROUTE_NOALLOC_MAX_LOGITS];
+
+// Device address of g_noalloc_logits per device ordinal, looked up once with
+// that device current (the host-side symbol is only a stand-in for it).
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+float *g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+cudaError_t noalloc_scratch(int device, float **out) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[device]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_logits);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[device] = static_cast<float *>(p);
+    }
+    *out = g_noalloc_ptr[device];
+    return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace tfmoe
+
+extern "C" tfmoe_status tfmoe_route_noalloc(const uint16_t *x, int32_t T, int32_t hidden,
+                                            const uint16_t *router_w, const float *router_bias,
+                                            int32_t num_experts, int32_t top_k,
+                                            int32_t *ids_out, float *weights_out, void *cuda_stream)
+{
+    using namespace tfmoe;
+    const int H = hidden, E = num_experts, k = top_k;
+    if (T < 0) return record_error(TFMOE_ERR_INVALID_ARG, "tfmoe_route_noalloc: T=%d is negative", T);
+    if (H <= 0 || H % 16)
+        return record_error(TFMOE_ERR_INVALID_ARG, "tfmoe_route_noalloc: hidden=%d must be a positive multiple of 16", H);
+    if (E <= 0 || k <= 0 || k > E)
+        return record_error(TFMOE_ERR_INVALID_ARG, "tfmoe_route_noalloc: need 1 <= top_k (%d) <= num_experts (%d)", k, E);
+    if (H % 32 || E > 256 || k > 32)
+        return record_error(TFMOE_ERR_UNSUPPORTED,
+                            "tfmoe_route_noalloc: needs hidden %% 32 == 0, num_experts <= 256, top_k <= 32");
+    if ((long long)T * E > (long long)TFMOE_ROUTE_NOALLOC_MAX_LOGITS)
+        return record_error(TFMOE_ERR_INVALID_ARG,
+                            "tfmoe_route_noalloc: T * num_experts = %lld exceeds the fixed scratch of %d logits; "
+                            "route the batch in parts of at most %d tokens",
+                            (long long)T * E, TFMOE_ROUTE_NOALLOC_MAX_LOGITS, TFMOE_ROUTE_NOALLOC_MAX_LOGITS / E);
+    if (T == 0) return record_ok();
+    if (!x || !router_w || !ids_out || !weights_out)
+        return record_error(TFMOE_ERR_INVALID_ARG, "tfmoe_route_noalloc: NULL buffer");
+    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(router_w)) & 15u)
+        return record_error(TFMOE_ERR_INVALID_ARG, "tfmoe_route_noalloc: x and router_w must be 16-byte aligned");
+    int device = 0;
+    cudaError_t e = cudaGetDevice(&device);
+    if (e == cudaSuccess && (device < 0 || device >= kNoAllocMaxDevices))
+        return record_error(TFMOE_ERR_UNSUPPORTED, "tfmoe_route_noalloc: device ordinal %d too large", device);
+    float *logits = nullptr;
+    if (e == cudaSuccess) e = noalloc_scratch(device, &logits);
+    if (e != cudaSuccess)
+        return record_error(TFMOE_ERR_CUDA, "tfmoe_route_noalloc: scratch address: %s", cudaGetErrorString(e));
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    if (T <= 2 * kSmallTokens) {
+        const int warps = E * ((T + kSmallTokens - 1) / kSmallTokens);
+        router_small_kernel<<<(warps + 3) / 4, 128, 0, s>>>(x, router_w, router_bias, logits, T, H, E, nullptr, 0);
+    } else {
+        dim3 grid((T + RT_T - 1) / RT_T, (E + RT_E - 1) / RT_E);
+        router_tiled_kernel<<<grid, 256, 0, s>>>(x, router_w, router_bias, logits, T, H, E, nullptr, 0);
+    }
+    topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(logits, ids_out, weights_out, T, E, k);
+    e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return record_error(TFMOE_ERR_CUDA, "tfmoe_route_noalloc: launch: %s", cudaGetErrorString(e));
+    return record_ok();
+}
+

@@ -27,7 +27,9 @@ BUF_LOGITS, BUF_TOPK_IDS, BUF_TOPK_WEIGHTS, BUF_EXPERT_COUNTS, BUF_EXPERT_OFFSET
 
 EXPORTED = ["tfmoe_create", "tfmoe_load_weights", "tfmoe_forward", "tfmoe_forward_host", "tfmoe_sync_status",
             "tfmoe_destroy", "tfmoe_last_error", "tfmoe_get_buffer", "tfmoe_last_launch_count",
-            "tfmoe_profile_enable", "tfmoe_profile_read"]
+            "tfmoe_profile_enable", "tfmoe_profile_read", "tfmoe_route_noalloc"]
+
+ROUTE_NOALLOC_MAX_LOGITS = 1 << 20
 
 STAGES = ["router", "topk", "permute", "gemv_gate_up", "gemv_down", "mma_gate_up", "mma_down", "combine", "gather"]
 
@@ -85,6 +87,8 @@ def load_library(path: str = LIB_PATH):
     lib.tfmoe_profile_enable.restype = ctypes.c_int
     lib.tfmoe_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(i32), i32]
     lib.tfmoe_profile_read.restype = ctypes.c_int
+    lib.tfmoe_route_noalloc.argtypes = [vp, i32, i32, vp, vp, i32, i32, vp, vp, vp]
+    lib.tfmoe_route_noalloc.restype = ctypes.c_int
     del u32
     _lib = lib
     return lib
@@ -193,6 +197,19 @@ class MoELayer:
             self.close()
         except Exception:
             pass
+
+
+def route_noalloc(x, router_w, router_bias, top_k: int, ids_out, weights_out, T: Optional[int] = None,
+                  stream=None) -> int:
+    """Routing through tfmoe_route_noalloc: no handle, no allocation inside the library.
+
+    For callers that cannot allocate device memory; the logits go to the
+    library's fixed per-device scratch. Returns the status code."""
+    if T is None:
+        T = x.shape[0]
+    E, H = router_w.shape
+    return load_library().tfmoe_route_noalloc(_ptr(x), T, H, _ptr(router_w), _ptr(router_bias), E, top_k,
+                                              _ptr(ids_out), _ptr(weights_out), _stream_handle(stream))
 
 
 class _DeviceView:
