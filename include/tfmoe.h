@@ -81,8 +81,9 @@ typedef struct {
     int32_t max_tokens;        /* the largest T tfmoe_forward will accept; sizes the workspace */
     int32_t has_router_bias;   /* 1: router_bias is read and added to the logits */
     uint32_t flags;            /* TFMOE_FLAG_* */
-    int32_t gemv_max_tokens;   /* experts routed <= this many tokens use the GEMV regime;
-                                  <= 0 selects the built-in crossover */
+    int32_t gemv_max_tokens;   /* experts routed to <= this many tokens use the CUDA-core GEMV
+                                  regime, the others the tcgen05 tensor-core regime;
+                                  <= 0 selects the built-in crossover (8) */
 } tfmoe_layer_desc;
 
 /*
@@ -199,6 +200,19 @@ typedef enum {
     TFMOE_STAGE_GATHER = 8,       /* tensor-core regime: activation row gather */
     TFMOE_STAGE_COUNT = 9
 } tfmoe_stage;
+
+/*
+ * Re-enqueue the kernels of one stage of the last tfmoe_forward on this
+ * handle, reading the workspace that forward left (routing, plan,
+ * intermediates) and rewriting that stage's outputs; a measurement aid for
+ * timing one kernel in isolation. T must equal the last forward's T and x
+ * must be its input (read by the gate/up stages); out receives the combine
+ * stage's result. Supported stages: GEMV_GATE_UP, GEMV_DOWN, MMA_GATE_UP,
+ * MMA_DOWN, GATHER, COMBINE (others return TFMOE_ERR_UNSUPPORTED); a stage
+ * whose kernels the forward did not use enqueues nothing.
+ */
+TFMOE_API tfmoe_status tfmoe_forward_stage(tfmoe_layer *layer, int32_t stage, const uint16_t *x, int32_t T,
+                                           uint16_t *out, void *cuda_stream);
 
 TFMOE_API tfmoe_status tfmoe_profile_enable(tfmoe_layer *layer, int32_t enable);
 TFMOE_API tfmoe_status tfmoe_profile_read(tfmoe_layer *layer, float *ms_total, int32_t *calls, int32_t reset);

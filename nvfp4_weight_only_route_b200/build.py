@@ -32,8 +32,8 @@ def _headers_mtime():
     return max(os.path.getmtime(h) for h in hs)
 
 
-def _compile(src, extra):
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+def _compile(src, extra, build_dir=BUILD):
+    obj = os.path.join(build_dir, os.path.basename(src) + ".o")
     cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
@@ -41,23 +41,24 @@ def _compile(src, extra):
     return obj, r.stderr
 
 
-def build(force: bool = False, extra=(), verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, extra=(), verbose: bool = False, out: str = LIB, build_dir: str = BUILD) -> str:
+    """Compile every csrc/*.cu and link `out` (default: the in-tree libtfmoe.so)."""
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sources()
     newest = max(max(os.path.getmtime(s) for s in srcs), _headers_mtime(), os.path.getmtime(__file__))
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest:
-        return LIB
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= newest:
+        return out
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        results = list(ex.map(lambda s: _compile(s, list(extra)), srcs))
+        results = list(ex.map(lambda s: _compile(s, list(extra), build_dir), srcs))
     if verbose:
         for _, log in results:
             if log.strip():
                 print(log, file=sys.stderr)
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *[o for o, _ in results], "-lcuda"]
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *[o for o, _ in results]]
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":

@@ -73,6 +73,9 @@ void carve_workspace(Layer &L, uint8_t *base, size_t *total) {
     c.take(&w.mma_list, E, base);
     c.take(&w.list_sizes, 4, base);
     c.take(&w.err_word, 1, base);
+    c.take(&w.route_counter, 1, base);
+    c.take(&w.mma_entries, 4 * max_mma_entries(P, E), base);
+    c.take(&w.x_perm, P * H, base);
     c.take(&w.act, P * I, base);
     c.take(&w.y, P * H, base);
     c.take(&w.x_stage, T * H, base);
@@ -174,8 +177,11 @@ tfmoe_status tfmoe_create(const tfmoe_layer_desc *desc, tfmoe_layer **out)
     carve_workspace(L, static_cast<uint8_t *>(L.ws_block), &L.ws_bytes);
     carve_weights(L, static_cast<uint8_t *>(L.w_block), &L.w_bytes);
     e = cudaMemset(L.ws.err_word, 0, sizeof(int32_t));
+    if (e == cudaSuccess) e = cudaMemset(L.ws.route_counter, 0, sizeof(int32_t));
     if (e == cudaSuccess) e = gemv_setup(L);
+    if (e == cudaSuccess) e = mma_setup(L);
     if (e != cudaSuccess) {
+        mma_teardown(L);
         cudaFree(L.ws_block);
         cudaFree(L.w_block);
         delete h;
@@ -242,12 +248,24 @@ tfmoe_status tfmoe_forward(tfmoe_layer *layer, const uint16_t *x, int32_t T, uin
     DeviceGuard dg(L.device);
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
     int n = 0;
+    // An expert holds at most T tokens, so with T <= the GEMV threshold no expert can be
+    // in the MMA regime and its launches are skipped (likewise under the FORCE flags).
+    const bool use_mma = !(L.desc.flags & TFMOE_FLAG_FORCE_GEMV) &&
+                         ((L.desc.flags & TFMOE_FLAG_FORCE_MMA) || T > L.gemv_max_tokens);
+    const bool use_gemv = !(L.desc.flags & TFMOE_FLAG_FORCE_MMA);
     cudaError_t e = launch_router(L, x, T, s, &n);
     if (e == cudaSuccess) e = launch_permute(L, T, s, &n);
-    if (e == cudaSuccess) e = launch_gemv(L, x, T, s, &n);
+    if (e == cudaSuccess && use_mma) e = launch_gather(L, x, T, s, &n);
+    if (e == cudaSuccess && use_mma) e = launch_mma_gate_up(L, s, &n);
+    if (e == cudaSuccess && use_gemv) e = launch_gemv_gate_up(L, x, s, &n);
+    if (e == cudaSuccess && use_mma) e = launch_mma_down(L, s, &n);
+    if (e == cudaSuccess && use_gemv) e = launch_gemv_down(L, s, &n);
     if (e == cudaSuccess) e = launch_combine(L, T, out, s, &n);
+    L.last_use_mma = use_mma;
+    L.last_use_gemv = use_gemv;
     L.last_launches = n;
     if (e != cudaSuccess) return cuda_fail(e, "tfmoe_forward: launch");
+    L.last_T = T;
     if (L.profiling) {
         e = cudaStreamSynchronize(s);
         for (int st = 0; st < TFMOE_STAGE_COUNT && e == cudaSuccess; ++st) {
@@ -314,6 +332,7 @@ void tfmoe_destroy(tfmoe_layer *layer)
                 if (ev) cudaEventDestroy(ev);
         if (L.ws_block) cudaFree(L.ws_block);
         if (L.w_block) cudaFree(L.w_block);
+        mma_teardown(L);
     }
     delete layer;
 }
@@ -341,6 +360,48 @@ tfmoe_status tfmoe_get_buffer(tfmoe_layer *layer, tfmoe_buffer which, void **dev
 }
 
 int32_t tfmoe_last_launch_count(tfmoe_layer *layer) { return layer ? layer->impl.last_launches : 0; }
+
+tfmoe_status tfmoe_forward_stage(tfmoe_layer *layer, int32_t stage, const uint16_t *x, int32_t T, uint16_t *out,
+                                 void *cuda_stream)
+{
+    if (!layer) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward_stage: layer is NULL");
+    Layer &L = layer->impl;
+    if (!L.loaded) return fail(TFMOE_ERR_NOT_LOADED, "tfmoe_forward_stage: weights not loaded");
+    if (T <= 0 || T != L.last_T)
+        return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward_stage: T=%d must equal the last forward's T=%d", T, L.last_T);
+    DeviceGuard dg(L.device);
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    int n = 0;
+    cudaError_t e = cudaSuccess;
+    switch (stage) {
+    case TFMOE_STAGE_GEMV_GATE_UP:
+        if (!x) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward_stage: x is NULL");
+        if (L.last_use_gemv) e = launch_gemv_gate_up(L, x, s, &n);
+        break;
+    case TFMOE_STAGE_GEMV_DOWN:
+        if (L.last_use_gemv) e = launch_gemv_down(L, s, &n);
+        break;
+    case TFMOE_STAGE_GATHER:
+        if (!x) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward_stage: x is NULL");
+        if (L.last_use_mma) e = launch_gather(L, x, T, s, &n);
+        break;
+    case TFMOE_STAGE_MMA_GATE_UP:
+        if (L.last_use_mma) e = launch_mma_gate_up(L, s, &n);
+        break;
+    case TFMOE_STAGE_MMA_DOWN:
+        if (L.last_use_mma) e = launch_mma_down(L, s, &n);
+        break;
+    case TFMOE_STAGE_COMBINE:
+        if (!out) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward_stage: out is NULL");
+        e = launch_combine(L, T, out, s, &n);
+        break;
+    default:
+        return fail(TFMOE_ERR_UNSUPPORTED, "tfmoe_forward_stage: stage %d cannot be replayed", stage);
+    }
+    L.last_launches = n;
+    if (e != cudaSuccess) return cuda_fail(e, "tfmoe_forward_stage: launch");
+    return ok();
+}
 
 tfmoe_status tfmoe_profile_enable(tfmoe_layer *layer, int32_t enable)
 {

@@ -10,16 +10,28 @@
 namespace tfmoe {
 
 // Tile geometry of the repacked NVFP4 weights: 128 rows x 64 reduction
-// elements per tile; a tile holds 4096 code bytes laid out as
-// [half of the 64 columns][128 rows][16 bytes], then its 512 scale bytes as
-// [128 rows][4 blocks of 16].
+// elements per tile. Codes: 4096 bytes per tile laid out as
+// [half of the 64 columns][128 rows][16 bytes], tiles ordered
+// [expert][row tile][column tile]. Scales: per (expert, row tile) a block of
+// KT * 512 bytes laid out [64-row half][column tile][64 rows][4 bytes], so the
+// scales of one 64-row half across all column tiles are contiguous.
 constexpr int kTileRows = 128;
 constexpr int kTileK = 64;
 constexpr int kTileCodeBytes = kTileRows * kTileK / 2;   // 4096
 constexpr int kTileScaleBytes = kTileRows * kTileK / 16; // 512
 
+// Byte offset of the scales of 64-row half `sub` of row tile `rt`, column tile `kt`.
+__host__ __device__ __forceinline__ size_t scale_offset(size_t row_tile_index, int KT, int sub, int kt) {
+    return row_tile_index * (size_t)KT * kTileScaleBytes + (size_t)sub * KT * (kTileScaleBytes / 2) +
+           (size_t)kt * (kTileScaleBytes / 2);
+}
+
 // Default crossover: experts routed to at most this many tokens use the GEMV regime.
-constexpr int kDefaultGemvMaxTokens = 1 << 30;
+constexpr int kDefaultGemvMaxTokens = 8;
+
+// Tokens per tensor-core tile (the MMA N dimension is at most 256).
+constexpr int kMmaTileTokens = 256;
+__host__ __device__ constexpr size_t max_mma_entries(size_t P, size_t E) { return P / kMmaTileTokens + E + 1; }
 
 struct Workspace {
     float *logits = nullptr;        // [maxT][E]
@@ -32,8 +44,11 @@ struct Workspace {
     int32_t *regime = nullptr;      // [E]
     int32_t *gemv_list = nullptr;   // [E]   experts in the GEMV regime, ascending
     int32_t *mma_list = nullptr;    // [E]   experts in the MMA regime, ascending
-    int32_t *list_sizes = nullptr;  // [4]   n_gemv, n_mma, (reserved)
+    int32_t *list_sizes = nullptr;  // [4]   n_gemv, n_mma, n_mma_entries, (reserved)
     int32_t *err_word = nullptr;    // [1]
+    int32_t *route_counter = nullptr; // [1] arrivals of the fused routing kernel (left at 0)
+    int32_t *mma_entries = nullptr; // [max_mma_entries][4] token tiles of the MMA regime
+    uint16_t *x_perm = nullptr;     // [maxP][H] bf16 activation rows in permuted order (MMA regime)
     uint16_t *act = nullptr;        // [maxP][I] bf16
     float *y = nullptr;             // [maxP][H]
     uint16_t *x_stage = nullptr;    // [maxT][H] bf16, for forward_host
@@ -65,7 +80,10 @@ struct Layer {
     Workspace ws;
     Weights w;
     int32_t last_launches = 0;
+    int32_t last_T = -1;            // T of the last successful forward (stage replays need it)
+    bool last_use_mma = false, last_use_gemv = false;
     int gemv_grid_gu = 0, gemv_grid_down = 0;
+    void *mma_maps = nullptr;       // tensor maps of the MMA regime's token operands
     // per-stage profiling (tfmoe_profile_enable)
     bool profiling = false;
     cudaEvent_t prof_ev[TFMOE_STAGE_COUNT][2] = {};
@@ -92,9 +110,16 @@ struct StageTimer {
 cudaError_t launch_router(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches);
 cudaError_t launch_permute(Layer &L, int T, cudaStream_t s, int *launches);
 cudaError_t launch_gemv(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches);
+cudaError_t launch_gemv_gate_up(Layer &L, const uint16_t *x, cudaStream_t s, int *launches);
+cudaError_t launch_gemv_down(Layer &L, cudaStream_t s, int *launches);
 cudaError_t launch_combine(Layer &L, int T, uint16_t *out, cudaStream_t s, int *launches);
 cudaError_t launch_repack(const Layer &L, const tfmoe_weights &src, cudaStream_t s);
 cudaError_t gemv_setup(Layer &L);
+cudaError_t mma_setup(Layer &L);
+void mma_teardown(Layer &L);
+cudaError_t launch_gather(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches);
+cudaError_t launch_mma_gate_up(Layer &L, cudaStream_t s, int *launches);
+cudaError_t launch_mma_down(Layer &L, cudaStream_t s, int *launches);
 
 // Sets the thread-local message returned by tfmoe_last_error() and returns st.
 tfmoe_status record_error(tfmoe_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));

@@ -3,10 +3,12 @@
 // Tile (128 rows x 64 reduction elements) of projection matrix M of expert e:
 //   codes  : 4096 bytes = [half h of the 64 columns][row r of 128][16 bytes]
 //            byte b of (h, r) holds columns 32h + 2b (low nibble) and 32h + 2b + 1
-//   scales :  512 bytes = [row r of 128][4 scale bytes of the 4 16-column blocks]
 // Tiles are stored [expert][row tile][column tile], so a row tile's columns
-// are contiguous. Gate and up share one matrix of 2I rows: row 2j is gate row
-// j and row 2j+1 is up row j.
+// are contiguous. Scales of (expert, row tile) form one block of KT * 512
+// bytes: [64-row half][column tile][64 rows][4 scale bytes of the 4 16-column
+// blocks], so one half's scales for every column tile are contiguous.
+// Gate and up share one matrix of 2I rows: row 2j is gate row j and row 2j+1
+// is up row j.
 #include "common.cuh"
 #include "internal.h"
 
@@ -45,7 +47,8 @@ __global__ void repack_kernel(const uint8_t *__restrict__ codes_a, const uint8_t
         uint8_t *ct = out_codes + tile * kTileCodeBytes + (r % kTileRows) * 16;
         *reinterpret_cast<uint4 *>(ct) = *reinterpret_cast<const uint4 *>(crow);
         *reinterpret_cast<uint4 *>(ct + 2048) = *reinterpret_cast<const uint4 *>(crow + 16);
-        *reinterpret_cast<uint32_t *>(out_scales + tile * kTileScaleBytes + (r % kTileRows) * 4) =
+        const size_t rti = (size_t)e * RT + r / kTileRows;
+        *reinterpret_cast<uint32_t *>(out_scales + scale_offset(rti, KT, (r % kTileRows) / 64, kt) + (r % 64) * 4) =
             *reinterpret_cast<const uint32_t *>(srow);
     }
 }

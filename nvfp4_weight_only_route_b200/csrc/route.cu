@@ -145,19 +145,14 @@ __global__ void __launch_bounds__(256) router_tiled_kernel(
 // One warp per token: k rounds of a warp arg-max over (logit desc, index asc),
 // then softmax over the selected logits (max-subtracted, fp32).
 constexpr int kMaxEPerLane = 8;   // E <= 256
-__global__ void __launch_bounds__(256) topk_kernel(
-    const float *__restrict__ logits, int32_t *__restrict__ ids, float *__restrict__ wts,
-    int T, int E, int k)
+__device__ __forceinline__ void topk_warp(const float *row, int E, int k, int32_t *ids_row, float *w_row)
 {
-    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
-    if (t >= T) return;
     float v[kMaxEPerLane];
-    const float *row = logits + (size_t)t * E;
 #pragma unroll
     for (int i = 0; i < kMaxEPerLane; ++i) {
         const int e = lane + 32 * i;
-        v[i] = (e < E) ? row[e] : -INFINITY;
+        v[i] = (e < E) ? __ldcg(row + e) : -INFINITY;
     }
     uint32_t taken = 0;
     float sel_first = 0.f, my_sel = 0.f;
@@ -186,44 +181,58 @@ __global__ void __launch_bounds__(256) topk_kernel(
         if (s == 0) sel_first = bv;
         if (lane == s) { my_sel = bv; my_id = bi; }
     }
-    // softmax over the k selected logits (slot order), fp32
     const float ex = (lane < k) ? expf(my_sel - sel_first) : 0.f;
     float den = ex;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
     if (lane < k) {
-        ids[(size_t)t * k + lane] = my_id;
-        wts[(size_t)t * k + lane] = ex / den;
+        ids_row[lane] = my_id;
+        w_row[lane] = ex / den;
     }
 }
 
-// Single CTA of 32 warps. Pairs p = t*k + s are split into 32 contiguous
-// segments, one per warp. Pass 1 counts per (segment, expert); a scan turns
-// the counts into per-expert offsets and per-segment bases; pass 2 places each
-// pair at base + its rank among same-expert pairs of the segment, so rows are
-// ordered by (expert, pair index) -- a stable counting sort.
-constexpr int kPermWarps = 32;
-__global__ void __launch_bounds__(1024) permute_kernel(
-    const int32_t *__restrict__ ids, int P, int E, int gemv_max_tokens, uint32_t flags,
-    int32_t *__restrict__ counts, int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
-    int32_t *__restrict__ inv, int32_t *__restrict__ regime, int32_t *__restrict__ gemv_list,
-    int32_t *__restrict__ mma_list, int32_t *__restrict__ list_sizes, int32_t *err_word, int debug)
+__global__ void __launch_bounds__(256) topk_kernel(
+    const float *__restrict__ logits, int32_t *__restrict__ ids, float *__restrict__ wts, int T, int E, int k)
 {
-    extern __shared__ int32_t sm[];
-    int32_t *cnt = sm;                       // [32][E]
-    int32_t *tot = sm + kPermWarps * E;      // [E]
-    int32_t *off = tot + E;                  // [E+1]
+    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (t >= T) return;
+    topk_warp(logits + (size_t)t * E, E, k, ids + (size_t)t * k, wts + (size_t)t * k);
+}
+
+// The expert plan, computed by one CTA of W warps. Pairs p = t*k + s are split
+// into W contiguous segments, one per warp. Pass 1 counts per (segment,
+// expert); a scan turns the counts into per-expert offsets and per-segment
+// bases; pass 2 places each pair at base + its rank among same-expert pairs of
+// the segment, so rows are ordered by (expert, pair index): a stable counting
+// sort. Then every routed expert gets its regime and joins its regime's list.
+struct PlanArgs {
+    int E, gemv_max_tokens;
+    uint32_t flags;
+    int32_t *counts, *offsets, *perm, *inv, *regime, *gemv_list, *mma_list, *list_sizes, *err_word;
+    int32_t *mma_entries;   // [max][4]: expert, first permuted row, rows (<= kMmaTileTokens), 0
+    int debug;
+};
+
+__host__ __device__ constexpr size_t plan_smem_ints(int warps, int E) { return (size_t)warps * E + 2 * E + 1; }
+
+__device__ void plan_block(const int32_t *__restrict__ ids, int P, const PlanArgs &pa, int32_t *sm)
+{
+    const int E = pa.E;
+    const int W = blockDim.x >> 5;
+    int32_t *cnt = sm;               // [W][E]
+    int32_t *tot = sm + W * E;       // [E]
+    int32_t *off = tot + E;          // [E+1]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) cnt[i] = 0;
+    for (int i = threadIdx.x; i < W * E; i += blockDim.x) cnt[i] = 0;
     __syncthreads();
-    const int seg = (P + kPermWarps - 1) / kPermWarps;
+    const int seg = (P + W - 1) / W;
     const int p_begin = min(P, warp * seg), p_end = min(P, p_begin + seg);
     int32_t *my_cnt = cnt + warp * E;
     for (int p0 = p_begin; p0 < p_end; p0 += 32) {
         const int p = p0 + lane;
-        int e = (p < p_end) ? ids[p] : -1;
+        int e = (p < p_end) ? __ldcg(ids + p) : -1;
         if (e >= E || (e < 0 && p < p_end)) {
-            if (debug) atomicOr(err_word, DEV_ERR_BAD_EXPERT);
+            if (pa.debug) atomicOr(pa.err_word, DEV_ERR_BAD_EXPERT);
             e = -1;
         }
         const uint32_t m = __match_any_sync(0xffffffffu, e);
@@ -231,10 +240,9 @@ __global__ void __launch_bounds__(1024) permute_kernel(
         __syncwarp();
     }
     __syncthreads();
-    // per-expert totals and per-segment bases (exclusive over segments)
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int run = 0;
-        for (int w = 0; w < kPermWarps; ++w) {
+        for (int w = 0; w < W; ++w) {
             const int c = cnt[w * E + e];
             cnt[w * E + e] = run;
             run += c;
@@ -266,25 +274,24 @@ __global__ void __launch_bounds__(1024) permute_kernel(
         if (lane == 31) off[E] = incl;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) cnt[i] += off[i % E];
-    for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets[e] = off[e];
+    for (int i = threadIdx.x; i < W * E; i += blockDim.x) cnt[i] += off[i % E];
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) pa.offsets[e] = off[e];
     __syncthreads();
     for (int p0 = p_begin; p0 < p_end; p0 += 32) {
         const int p = p0 + lane;
-        int e = (p < p_end) ? ids[p] : -1;
+        int e = (p < p_end) ? __ldcg(ids + p) : -1;
         if (e >= E) e = -1;
         const uint32_t m = __match_any_sync(0xffffffffu, e);
         if (e >= 0) {
             const int rank = __popc(m & ((1u << lane) - 1u));
             const int r = my_cnt[e] + rank;
-            perm[r] = p;
-            inv[p] = r;
+            pa.perm[r] = p;
+            pa.inv[p] = r;
         }
         __syncwarp();
         if (e >= 0 && lane == __ffs(m) - 1) my_cnt[e] += __popc(m);
         __syncwarp();
     }
-    // regimes and compacted expert lists (ascending expert order)
     if (warp == 0) {
         int n_gemv = 0, n_mma = 0;
         for (int e0 = 0; e0 < E; e0 += 32) {
@@ -292,41 +299,177 @@ __global__ void __launch_bounds__(1024) permute_kernel(
             const int m = (e < E) ? tot[e] : 0;
             int reg = 0;
             if (m > 0) {
-                if (flags & TFMOE_FLAG_FORCE_GEMV) reg = 1;
-                else if (flags & TFMOE_FLAG_FORCE_MMA) reg = 2;
-                else reg = (m <= gemv_max_tokens) ? 1 : 2;
+                if (pa.flags & TFMOE_FLAG_FORCE_GEMV) reg = 1;
+                else if (pa.flags & TFMOE_FLAG_FORCE_MMA) reg = 2;
+                else reg = (m <= pa.gemv_max_tokens) ? 1 : 2;
             }
-            if (e < E) { regime[e] = reg; counts[e] = m; }
+            if (e < E) { pa.regime[e] = reg; pa.counts[e] = m; }
             const uint32_t bg = __ballot_sync(0xffffffffu, reg == 1);
             const uint32_t bm = __ballot_sync(0xffffffffu, reg == 2);
             const uint32_t lt = (1u << lane) - 1u;
-            if (reg == 1) gemv_list[n_gemv + __popc(bg & lt)] = e;
-            if (reg == 2) mma_list[n_mma + __popc(bm & lt)] = e;
+            if (reg == 1) pa.gemv_list[n_gemv + __popc(bg & lt)] = e;
+            if (reg == 2) pa.mma_list[n_mma + __popc(bm & lt)] = e;
             n_gemv += __popc(bg);
             n_mma += __popc(bm);
         }
-        if (lane == 0) { list_sizes[0] = n_gemv; list_sizes[1] = n_mma; }
+        if (lane == 0) { pa.list_sizes[0] = n_gemv; pa.list_sizes[1] = n_mma; }
+        // token tiles of the MMA-regime experts: ceil(m_e / kMmaTileTokens) entries per
+        // expert, in expert order; lane l handles experts 8l .. 8l+7
+        int ntl[8], mine = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane * 8 + i;
+            int n = 0;
+            if (e < E) {
+                const int m = tot[e];
+                const bool mma = m > 0 && !(pa.flags & TFMOE_FLAG_FORCE_GEMV) &&
+                                 ((pa.flags & TFMOE_FLAG_FORCE_MMA) || m > pa.gemv_max_tokens);
+                n = mma ? (m + kMmaTileTokens - 1) / kMmaTileTokens : 0;
+            }
+            ntl[i] = n;
+            mine += n;
+        }
+        int incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int idx = incl - mine;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane * 8 + i;
+            for (int j = 0; j < ntl[i]; ++j, ++idx) {
+                int32_t *ent = pa.mma_entries + 4 * (size_t)idx;
+                ent[0] = e;
+                ent[1] = off[e] + j * kMmaTileTokens;
+                ent[2] = min(kMmaTileTokens, tot[e] - j * kMmaTileTokens);
+                ent[3] = 0;
+            }
+        }
+        if (lane == 31) pa.list_sizes[2] = incl;
     }
 }
 
+__global__ void __launch_bounds__(1024) permute_kernel(const int32_t *__restrict__ ids, int P, PlanArgs pa)
+{
+    extern __shared__ int32_t sm[];
+    plan_block(ids, P, pa, sm);
+}
+
+// Decode-sized batches (T <= 16): router, top-k and plan in one launch.
+// CTA e computes the logits of expert e for every token (its 8 warps split
+// the hidden dimension, partial sums are added in a fixed order), then the
+// last CTA to finish -- found with an atomic counter, which it resets --
+// takes the top-k of every token and builds the plan. The wide grid keeps
+// the expert dot products parallel; folding top-k into the last-arriving
+// block is the launch-saving shape proposed in TensorFold issue #627 (comment
+// on the fused tf_nemo_route_row experiment).
+constexpr int kFusedMaxT = 16;
+constexpr int kFusedThreads = 256;
+__global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(
+    const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, const float *__restrict__ bias,
+    float *__restrict__ logits, int32_t *__restrict__ ids, float *__restrict__ wts, int T, int H, int k,
+    PlanArgs pa, int32_t *counter)
+{
+    extern __shared__ int32_t sm[];
+    __shared__ double red[kFusedThreads / 32][kFusedMaxT];
+    __shared__ int is_last;
+    const int E = pa.E, e = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    double acc[kFusedMaxT];
+#pragma unroll
+    for (int t = 0; t < kFusedMaxT; ++t) acc[t] = 0.0;
+    const uint16_t *wrow = wr + (size_t)e * H;
+    for (int c = threadIdx.x * 8; c < H; c += kFusedThreads * 8) {
+        const uint4 wv = *reinterpret_cast<const uint4 *>(wrow + c);
+        const uint32_t wu[4] = {wv.x, wv.y, wv.z, wv.w};
+        double w[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            w[2 * i] = (double)bf16_bits_to_float(wu[i] & 0xFFFFu);
+            w[2 * i + 1] = (double)bf16_bits_to_float(wu[i] >> 16);
+        }
+#pragma unroll
+        for (int t = 0; t < kFusedMaxT; ++t) {
+            if (t < T) {
+                const uint4 xv = *reinterpret_cast<const uint4 *>(x + (size_t)t * H + c);
+                const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    acc[t] = fma((double)bf16_bits_to_float(xu[i] & 0xFFFFu), w[2 * i], acc[t]);
+                    acc[t] = fma((double)bf16_bits_to_float(xu[i] >> 16), w[2 * i + 1], acc[t]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < kFusedMaxT; ++t) {
+        if (t < T) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+            if (lane == 0) red[warp][t] = acc[t];
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < T) {
+        double v = 0.0;
+#pragma unroll
+        for (int w = 0; w < kFusedThreads / 32; ++w) v += red[w][threadIdx.x];
+        float l = (float)v;
+        if (bias) l = l + bias[e];
+        if (pa.debug && !isfinite(l)) atomicOr(pa.err_word, DEV_ERR_NONFINITE);
+        logits[(size_t)threadIdx.x * E + e] = l;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = (atomicAdd(counter, 1) == (int)gridDim.x - 1);
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    for (int t = warp; t < T; t += kFusedThreads / 32)
+        topk_warp(logits + (size_t)t * E, E, k, ids + (size_t)t * k, wts + (size_t)t * k);
+    __syncthreads();
+    plan_block(ids, T * k, pa, sm);
+    if (threadIdx.x == 0) *counter = 0;
+}
+
 }  // namespace
+
+static PlanArgs plan_args(const Layer &L) {
+    PlanArgs pa{};
+    pa.E = L.desc.num_experts;
+    pa.gemv_max_tokens = L.gemv_max_tokens;
+    pa.flags = L.desc.flags;
+    pa.counts = L.ws.counts; pa.offsets = L.ws.offsets; pa.perm = L.ws.perm; pa.inv = L.ws.inv;
+    pa.regime = L.ws.regime; pa.gemv_list = L.ws.gemv_list; pa.mma_list = L.ws.mma_list;
+    pa.list_sizes = L.ws.list_sizes; pa.err_word = L.ws.err_word;
+    pa.mma_entries = L.ws.mma_entries;
+    pa.debug = (L.desc.flags & TFMOE_FLAG_DEBUG_CHECKS) ? 1 : 0;
+    return pa;
+}
+
+bool route_fused_applies(const Layer &L, int T) { return T <= kFusedMaxT; }
 
 cudaError_t launch_router(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches)
 {
     const int H = L.desc.hidden, E = L.desc.num_experts, k = L.desc.top_k;
     const int debug = (L.desc.flags & TFMOE_FLAG_DEBUG_CHECKS) ? 1 : 0;
     const float *bias = L.desc.has_router_bias ? L.w.router_bias : nullptr;
+    if (route_fused_applies(L, T)) {
+        // router, top-k and plan in one launch (the permute launcher then does nothing)
+        StageTimer timer(L, TFMOE_STAGE_ROUTER, s);
+        const size_t smem = sizeof(int32_t) * plan_smem_ints(kFusedThreads / 32, E);
+        route_fused_kernel<<<E, kFusedThreads, smem, s>>>(x, L.w.router_w, bias, L.ws.logits, L.ws.ids,
+                                                          L.ws.topk_w, T, H, k, plan_args(L), L.ws.route_counter);
+        *launches += 1;
+        return cudaGetLastError();
+    }
     {
-    StageTimer timer(L, TFMOE_STAGE_ROUTER, s);
-    if (T <= 2 * kSmallTokens) {
-        const int warps = E * ((T + kSmallTokens - 1) / kSmallTokens);
-        router_small_kernel<<<(warps + 3) / 4, 128, 0, s>>>(x, L.w.router_w, bias, L.ws.logits, T, H, E,
-                                                           L.ws.err_word, debug);
-    } else {
+        StageTimer timer(L, TFMOE_STAGE_ROUTER, s);
         dim3 grid((T + RT_T - 1) / RT_T, (E + RT_E - 1) / RT_E);
         router_tiled_kernel<<<grid, 256, 0, s>>>(x, L.w.router_w, bias, L.ws.logits, T, H, E,
                                                   L.ws.err_word, debug);
-    }
     }
     {
         StageTimer timer(L, TFMOE_STAGE_TOPK, s);
@@ -338,13 +481,11 @@ cudaError_t launch_router(Layer &L, const uint16_t *x, int T, cudaStream_t s, in
 
 cudaError_t launch_permute(Layer &L, int T, cudaStream_t s, int *launches)
 {
+    if (route_fused_applies(L, T)) return cudaSuccess;
     StageTimer timer(L, TFMOE_STAGE_PERMUTE, s);
     const int E = L.desc.num_experts, P = T * L.desc.top_k;
-    const int debug = (L.desc.flags & TFMOE_FLAG_DEBUG_CHECKS) ? 1 : 0;
-    const size_t smem = sizeof(int32_t) * ((size_t)kPermWarps * E + 2 * E + 1);
-    permute_kernel<<<1, 1024, smem, s>>>(L.ws.ids, P, E, L.gemv_max_tokens, L.desc.flags, L.ws.counts,
-                                          L.ws.offsets, L.ws.perm, L.ws.inv, L.ws.regime, L.ws.gemv_list,
-                                          L.ws.mma_list, L.ws.list_sizes, L.ws.err_word, debug);
+    const size_t smem = sizeof(int32_t) * plan_smem_ints(32, E);
+    permute_kernel<<<1, 1024, smem, s>>>(L.ws.ids, P, plan_args(L));
     *launches += 1;
     return cudaGetLastError();
 }

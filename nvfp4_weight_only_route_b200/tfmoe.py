@@ -12,7 +12,7 @@ import os
 from typing import Dict, Optional
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libtfmoe.so")
+LIB_PATH = os.environ.get("TFMOE_LIB", os.path.join(PKG, "libtfmoe.so"))
 
 OK, ERR_INVALID_ARG, ERR_OOM, ERR_CUDA, ERR_NOT_LOADED, ERR_UNSUPPORTED, ERR_TIMEOUT, ERR_DEVICE = range(8)
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "OOM", 3: "CUDA", 4: "NOT_LOADED", 5: "UNSUPPORTED",
@@ -27,11 +27,12 @@ BUF_LOGITS, BUF_TOPK_IDS, BUF_TOPK_WEIGHTS, BUF_EXPERT_COUNTS, BUF_EXPERT_OFFSET
 
 EXPORTED = ["tfmoe_create", "tfmoe_load_weights", "tfmoe_forward", "tfmoe_forward_host", "tfmoe_sync_status",
             "tfmoe_destroy", "tfmoe_last_error", "tfmoe_get_buffer", "tfmoe_last_launch_count",
-            "tfmoe_profile_enable", "tfmoe_profile_read", "tfmoe_route_noalloc"]
+            "tfmoe_profile_enable", "tfmoe_profile_read", "tfmoe_route_noalloc", "tfmoe_forward_stage"]
 
 ROUTE_NOALLOC_MAX_LOGITS = 1 << 20
 
 STAGES = ["router", "topk", "permute", "gemv_gate_up", "gemv_down", "mma_gate_up", "mma_down", "combine", "gather"]
+STAGE_ID = {n: i for i, n in enumerate(STAGES)}
 
 
 class LayerDesc(ctypes.Structure):
@@ -87,6 +88,8 @@ def load_library(path: str = LIB_PATH):
     lib.tfmoe_profile_enable.restype = ctypes.c_int
     lib.tfmoe_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(i32), i32]
     lib.tfmoe_profile_read.restype = ctypes.c_int
+    lib.tfmoe_forward_stage.argtypes = [vp, i32, vp, i32, vp, vp]
+    lib.tfmoe_forward_stage.restype = ctypes.c_int
     lib.tfmoe_route_noalloc.argtypes = [vp, i32, i32, vp, vp, i32, i32, vp, vp, vp]
     lib.tfmoe_route_noalloc.restype = ctypes.c_int
     del u32
@@ -143,6 +146,10 @@ class MoELayer:
 
     def forward_raw(self, x_ptr: int, T: int, out_ptr: int, stream_handle: int) -> int:
         return self.lib.tfmoe_forward(self.handle, x_ptr, T, out_ptr, stream_handle)
+
+    def forward_stage_raw(self, stage: int, x_ptr: int, T: int, out_ptr: int, stream_handle: int) -> int:
+        """Re-enqueue one stage of the last forward (see tfmoe_forward_stage)."""
+        return self.lib.tfmoe_forward_stage(self.handle, stage, x_ptr, T, out_ptr, stream_handle)
 
     def forward_host(self, x_host, out_host, T: Optional[int] = None, stream=None):
         """Host (CPU) tensors in and out; copies happen inside the call, which returns when done."""

@@ -14,7 +14,7 @@ from gpu_harness import GpuRun, check_intermediates, check_output, check_routing
 
 pytestmark = pytest.mark.gpu
 
-REGIMES = {"gemv": 1}          # flag values: FORCE_GEMV = 1
+REGIMES = {"gemv": 1, "mma": 2, "auto": 0}     # descriptor flags: FORCE_GEMV = 1, FORCE_MMA = 2
 
 
 @pytest.fixture(scope="module", autouse=True)
