@@ -112,9 +112,10 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def kernel_source_hash():
+def kernel_source_hash(stage: str = "gemv_gate_up"):
     h = hashlib.sha256()
-    for f in ("gemv.cu", "common.cuh", "internal.h"):
+    files = ("mma.cu",) if stage.startswith("mma") else ("gemv.cu",)
+    for f in files + ("common.cuh", "internal.h"):
         h.update(open(os.path.join(ROOT, "nvfp4_weight_only_route_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
@@ -126,7 +127,7 @@ def ncu_traffic(stage: str):
         return None
     d = json.load(open(p))
     ent = d.get(stage)
-    if not ent or ent.get("kernel_source_hash") != kernel_source_hash():
+    if not ent or ent.get("kernel_source_hash") != kernel_source_hash(stage):
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -366,37 +367,53 @@ def main():
     # ---- per-kernel timing for the roofline: one forward per layer on a known batch, then
     # a CUDA graph that re-enqueues one stage of those forwards, rotating over the layers
     # (so consecutive launches read different weights), timed with events on its stream.
-    gemv_units = []
+    gemv_units, mma_pairs = [], []
     for li, L in enumerate(layers):
         with torch.cuda.stream(stream):
             tfmoe.check(L.forward_raw(xs[li][0].data_ptr(), T, out.data_ptr(), stream.cuda_stream))
         stream.synchronize()
         reg = L.buffer_tensor(tfmoe.BUF_REGIME, torch.int32, (E,)).cpu().numpy()
+        cnt = L.buffer_tensor(tfmoe.BUF_EXPERT_COUNTS, torch.int32, (E,)).cpu().numpy()
         gemv_units.append(int(np.sum(reg == 1)))
+        mma_pairs.append(int(np.sum(cnt[reg == 2])))
     kernel_us = {}
-    reps = max(1, min(50, args.steps // max(1, len(layers))))
-    for stage in ("gemv_gate_up", "gemv_down", "combine"):
+    for stage in ("gemv_gate_up", "gemv_down", "gather", "mma_gate_up", "mma_down", "combine"):
         sid = tfmoe.STAGE_ID[stage]
-        g = torch.cuda.CUDAGraph()
+        # one launch per layer, timed once, sizes the graph to ~5 ms of work
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         launched = 0
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for li, L in enumerate(layers):
+                tfmoe.check(L.forward_stage_raw(sid, xs[li][0].data_ptr(), T, out.data_ptr(), stream.cuda_stream))
+                launched += L.last_launch_count()
+            e1.record(stream)
+        stream.synchronize()
+        if launched == 0:
+            continue
+        est_us = max(1.0, e0.elapsed_time(e1) * 1e3 / len(layers))
+        reps = int(max(2, min(50, 5000.0 / est_us / len(layers))))
+        g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for r in range(reps):
                 for li, L in enumerate(layers):
                     tfmoe.check(L.forward_stage_raw(sid, xs[li][0].data_ptr(), T, out.data_ptr(), stream.cuda_stream))
-                    launched += L.last_launch_count()
-        if launched == 0:
-            continue
-        g.replay()
-        stream.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
+        for _ in range(3):      # the first replays of a new graph run slow; keep them out of the timing
             g.replay()
-            e1.record(stream)
         stream.synchronize()
-        kernel_us[stage] = e0.elapsed_time(e1) * 1e3 / (reps * len(layers))
+        samples = []
+        for _ in range(5):
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+            stream.synchronize()
+            samples.append(e0.elapsed_time(e1) * 1e3 / (reps * len(layers)))
+        kernel_us[stage] = float(np.median(samples))
         del g
     dominant = max(kernel_us, key=kernel_us.get)
+    how = (f"median of 5 replays of a graph of back-to-back launches rotating {len(layers)} layer(s), "
+           "CUDA events on the launch stream")
     if dominant in ("gemv_gate_up", "gemv_down"):
         rows = 2 * I * H if dominant == "gemv_gate_up" else H * I
         alg = float(np.mean(gemv_units)) * rows * NVFP4_BYTES_PER_WEIGHT
@@ -405,7 +422,18 @@ def main():
                     "frac": achieved / hbm_peak, "traffic": ncu_traffic(dominant),
                     "algorithmic_bytes_per_launch": alg, "avg_launch_us": kernel_us[dominant],
                     "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback",
-                    "how": f"graph of {reps * len(layers)} launches rotating {len(layers)} layers, CUDA events"}
+                    "how": how}
+    elif dominant in ("mma_gate_up", "mma_down"):
+        rows = 2 * I if dominant == "mma_gate_up" else H
+        kdim = H if dominant == "mma_gate_up" else I
+        alg = 2.0 * float(np.mean(mma_pairs)) * rows * kdim
+        achieved = alg / (kernel_us[dominant] * 1e-6) / 1e12
+        roofline = {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": bf16_peak,
+                    "unit": "TFLOP/s", "frac": achieved / bf16_peak, "traffic": ncu_traffic(dominant),
+                    "algorithmic_flops_per_launch": alg, "avg_launch_us": kernel_us[dominant],
+                    "peak_source": ("measured (MEASURED_PEAKS.json bf16_tflops, burst)" if peak_src == "measured"
+                                    else "fallback"),
+                    "how": how}
     else:
         roofline = {"bound": "hbm", "kernel": dominant, "achieved": None, "peak": hbm_peak, "unit": "GB/s",
                     "frac": None, "traffic": ncu_traffic(dominant), "avg_launch_us": kernel_us[dominant]}
@@ -464,6 +492,7 @@ def main():
                       "hbm_frac": layer_gbs / hbm_peak, "hbm_frac_of_8tbs": layer_gbs / 8000.0,
                       "flops_per_forward": flops_per_fwd, "tflops": layer_tflops,
                       "tensor_frac": layer_tflops / bf16_peak, "active_experts_mean": mean_active,
+                      "mma_pairs_mean": float(np.mean(mma_pairs)), "gemv_experts_mean": float(np.mean(gemv_units)),
                       "kernel_us_graph": kernel_us, "stage_avg_us_profiled": stage_avg_us},
             "cpu_baseline": cpu,
             "e2e": e2e,

@@ -76,6 +76,7 @@ void carve_workspace(Layer &L, uint8_t *base, size_t *total) {
     c.take(&w.route_counter, 1, base);
     c.take(&w.mma_entries, 4 * max_mma_entries(P, E), base);
     c.take(&w.x_perm, P * H, base);
+    c.take(&w.row_inv, P, base);
     c.take(&w.act, P * I, base);
     c.take(&w.y, P * H, base);
     c.take(&w.x_stage, T * H, base);

@@ -108,6 +108,8 @@ __device__ __forceinline__ uint16_t float_to_bf16_bits_rn(float f) {
     return *reinterpret_cast<uint16_t *>(&b);
 }
 
-__device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + expf(-z)); }
+// z * sigmoid(z); exp and reciprocal on the special-function unit (relative error
+// ~1e-6, far below the bf16 rounding that follows). Large -z gives rcp(inf) = 0.
+__device__ __forceinline__ float silu_f32(float z) { return z * __frcp_rn(1.0f + __expf(-z)); }
 
 }  // namespace tfmoe

@@ -29,8 +29,8 @@ __host__ __device__ __forceinline__ size_t scale_offset(size_t row_tile_index, i
 // Default crossover: experts routed to at most this many tokens use the GEMV regime.
 constexpr int kDefaultGemvMaxTokens = 8;
 
-// Tokens per tensor-core tile (the MMA N dimension is at most 256).
-constexpr int kMmaTileTokens = 256;
+// Tokens per tensor-core tile (the MMA N dimension).
+constexpr int kMmaTileTokens = 176;
 __host__ __device__ constexpr size_t max_mma_entries(size_t P, size_t E) { return P / kMmaTileTokens + E + 1; }
 
 struct Workspace {
@@ -48,7 +48,8 @@ struct Workspace {
     int32_t *err_word = nullptr;    // [1]
     int32_t *route_counter = nullptr; // [1] arrivals of the fused routing kernel (left at 0)
     int32_t *mma_entries = nullptr; // [max_mma_entries][4] token tiles of the MMA regime
-    uint16_t *x_perm = nullptr;     // [maxP][H] bf16 activation rows in permuted order (MMA regime)
+    uint16_t *x_perm = nullptr;     // [maxP][H] f16 activation rows (times 2^sh) in permuted order (MMA regime)
+    float *row_inv = nullptr;       // [maxP] 2^-sh of each x_perm row
     uint16_t *act = nullptr;        // [maxP][I] bf16
     float *y = nullptr;             // [maxP][H]
     uint16_t *x_stage = nullptr;    // [maxT][H] bf16, for forward_host

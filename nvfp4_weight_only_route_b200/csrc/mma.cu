@@ -1,29 +1,42 @@
 // mma.cu -- the prefill regime of the NVFP4 grouped expert projections:
-// dequantise into the tensor core's operand memory and run BF16 tcgen05 MMAs.
+// dequantise into the tensor core's operand memory and run tcgen05 MMAs.
 //
 // Prefill pushes all prompt tokens through the active experts as one large
 // matrix multiply, so it is limited by tensor throughput rather than memory
 // (DGX Spark GB10 bandwidth-budget page, section "Mechanism: decode is
 // bandwidth-bound, prefill is compute-bound"). The weights stay W4A16: they are
-// decoded to BF16 and multiplied against BF16 activations (TensorFold 1.0.12
-// GLM-5.3-Flash post, section "NVFP4 is neither uniform 4-bit nor all-FP4
-// compute"); the decode is exact (an E2M1 value times an E4M3 scale has at most
-// 6 significant bits) and the per-tensor fp32 scale multiplies the fp32
-// accumulator in the epilogue.
+// decoded to 16-bit floats and multiplied against the 16-bit activations
+// (TensorFold 1.0.12 GLM-5.3-Flash post, section "NVFP4 is neither uniform
+// 4-bit nor all-FP4 compute"). The decode is exact: an E2M1 value times an E4M3
+// scale has at most 6 significant bits and lies in [2^-10, 2688], so it is an
+// f16 and a bf16 value; the per-tensor fp32 scale multiplies the accumulator.
 //
-// Tile: 128 weight rows (MMA M) x N <= 256 token rows of one expert (MMA N), the
-// reduction in stages of 64. One CTA per SM, persistent over tiles; roles:
-//   warp 0     producer: per stage, the token tile (TMA, 128-byte swizzle, box
-//              64 x N) and the 4 KB code tile + 2 x 256 B scales (bulk copies)
-//   warp 1     allocates tensor memory; lane 0 issues tcgen05.mma (A from tensor
-//              memory, B from shared memory, D fp32 in tensor memory) and commits
-//   warps 4-7  thread q owns weight row q = tensor-memory lane q: decodes its 64
-//              codes per stage to BF16 and stores them into the A stage; after
-//              the last stage reads its row of D and runs the epilogue (SwiGLU for
-//              interleaved gate/up rows, fp32 store for down).
-// Tensor memory: D at columns [0, 256), A stages of 32 columns from 256 on.
-// Every wait is bounded; on a timeout the CTA records the error, stops issuing
-// work, and still frees its tensor memory.
+//   gate/up: f16 x f16 -> fp32. The activation rows are stored as f16 times an
+//            exact per-row power of two (every bf16 element within 2^28 of the
+//            row's largest is then an exact f16), undone in the epilogue.
+//            E2M1 -> f16 is one conversion, the scale one f16x2 multiply.
+//   down   : bf16 x bf16 -> fp32; the SwiGLU output a is a bf16 tensor already.
+//
+// Tile: 128 weight rows (MMA M) x N <= 176 token rows of one expert (MMA N), the
+// reduction in stages of 64. One persistent CTA per SM, 20 warps:
+//   warp 0       producer of the token tiles (TMA, 128-byte swizzle, box 64 x N)
+//                into a 5-stage ring that the MMA commit frees
+//   warp 2       producer of the 4 KB code tiles + 2 x 256 B scales (bulk copies)
+//                into a 12-stage ring that the decoders free once they have read it
+//   warp 1       allocates tensor memory; lane 0 issues the MMAs and commits. Each
+//                tcgen05.mma costs the issuing thread ~100 cycles whatever N is, so
+//                tiles are as wide as a double-buffered accumulator allows (N = 176,
+//                ~90 cycles of tensor work per MMA) and the thread does one wait and
+//                one commit per stage.
+//   warps 4-7    decode the even stages, warps 8-11 the odd ones (all 64 columns):
+//                thread q of a warpgroup owns weight row q = tensor-memory lane q
+//   warps 12-19  epilogue, two warpgroups taking alternate 16-column steps of the
+//                accumulator one tile behind the MMAs: SwiGLU for interleaved
+//                gate/up rows (row 2j gate j, 2j+1 up j) staged through shared
+//                memory into 16-byte row pieces, fp32 store for down.
+// Tensor memory: accumulators at columns [0,176) and [176,352), five A stages of
+// 32 columns from 352. Every wait is bounded; on a timeout the CTA records
+// the error, stops issuing work, lets issued copies land, frees tensor memory.
 #include <cuda.h>
 
 #include <new>
@@ -35,22 +48,28 @@ namespace tfmoe {
 namespace {
 
 constexpr int kM = 128;
-constexpr int kMaxN = kMmaTileTokens;      // 256
-constexpr int kStages = 4;
-constexpr int kThreads = 256;
-constexpr int kDequantWarp0 = 4;
+constexpr int kMaxN = kMmaTileTokens;      // 176
+constexpr int kStages = 5;                 // token-tile ring and tensor-memory A ring
+constexpr int kCStages = 16;               // code/scale ring
+constexpr int kThreads = 640;
+constexpr int kDqWarp0 = 4;                // two dequant warpgroups: warps 4..11
+constexpr int kEpiWarp0 = 12;              // two epilogue warpgroups: warps 12..19
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccCol = 0;
-constexpr uint32_t kACol = 256;
-constexpr int kBStageBytes = kMaxN * 128;  // N rows x 64 bf16
-constexpr int kNumBoxes = 5;               // token-tile heights 16, 32, 64, 128, 256
+constexpr uint32_t kACol = 2 * kMaxN;      // accumulators at [0,176), [176,352); A stages from 352
+constexpr int kBStageBytes = kMaxN * 128;  // N rows x 64 16-bit elements (22 KB, a multiple of 1 KB)
+constexpr int kNumBoxes = 5;               // token-tile heights 16, 32, 64, 128, 176
+constexpr int kEpiCols = 16;               // accumulator columns per epilogue step
+static_assert(kACol + kStages * 32 <= kTmemCols, "tensor memory budget");
+static_assert(kBStageBytes % 1024 == 0, "token stages must stay 1 KB aligned");
 
 struct MmaSmem {
-    uint8_t b[kStages][kBStageBytes];      // 1024-byte aligned (each stage is 32 KB)
-    uint8_t codes[kStages][kTileCodeBytes];
-    uint8_t scales[kStages][kTileScaleBytes];
+    uint8_t b[kStages][kBStageBytes];      // 1024-byte aligned
+    uint8_t codes[kCStages][kTileCodeBytes];
+    uint8_t scales[kCStages][kTileScaleBytes];
+    uint16_t stage_out[8][kEpiCols][16];   // per epilogue warp: 16 tokens x 16 outputs (gate/up)
     uint64_t full[kStages], empty[kStages], aready[kStages];
-    uint64_t dfull, dempty;
+    uint64_t cfull[kCStages], cempty[kCStages];
+    uint64_t dfull[2], dempty[2];
     uint32_t tmem_base;
     int32_t abort_flag;
 };
@@ -69,9 +88,25 @@ struct MmaArgs {
     const int32_t *list_sizes;             // [2] = number of entries
     uint16_t *act_out;                     // gate/up output [P][I]
     float *y_out;                          // down output [P][H]
+    const float *row_inv_scale;            // gate/up: 2^-sh of each f16 activation row [P]
     int I;
     int32_t *err_word;
 };
+
+#ifdef TFMOE_MMA_STATS
+// Instrumented build only: cycles each role spends in barrier waits, per CTA.
+constexpr int kStatSlots = 12;
+__device__ unsigned long long g_mma_stats[160][kStatSlots];
+#define STAT_WAIT(slot, expr)                                                              \
+    ([&]() {                                                                               \
+        const long long _t0 = clock64();                                                   \
+        const bool _r = (expr);                                                            \
+        atomicAdd(&g_mma_stats[blockIdx.x % 160][slot], (unsigned long long)(clock64() - _t0)); \
+        return _r;                                                                         \
+    }())
+#else
+#define STAT_WAIT(slot, expr) (expr)
+#endif
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, MmaSmem &sm, int32_t *err) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -95,12 +130,12 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
            ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
 }
 
-// kind::f16, A = B = BF16 (K-major), D = F32, M = 128, N given.
-__device__ __forceinline__ uint32_t instr_desc_bf16(int n) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kM >> 4) << 24);
+// kind::f16, A and B K-major of one 16-bit type (0 = f16, 1 = bf16), D = F32, M = 128, N given.
+__device__ __forceinline__ uint32_t instr_desc_16bit(int n, uint32_t type) {
+    return (1u << 4) | (type << 7) | (type << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kM >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+__device__ __forceinline__ void mma_16bit_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                             uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
@@ -119,24 +154,18 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         ::"r"(smem_u32(dst)), "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
         ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
-        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
-        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]));
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]));
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
 }
 
@@ -144,6 +173,13 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Two E2M1 codes (one byte) times the block scale (f16 pair, both halves equal) -> f16x2.
+__device__ __forceinline__ uint32_t dequant_pair_f16(uint32_t byte, __half2 scale2) {
+    const uint32_t h = e2m1x2_to_f16x2(byte);
+    const __half2 v = __hmul2(*reinterpret_cast<const __half2 *>(&h), scale2);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
 
 // Two E2M1 codes (one byte) times the block scale (f16 pair, both halves equal) -> bf16x2.
 // Products are exact in f16 (<= 6 significant bits, magnitudes 2^-10 .. 2688) and in bf16.
@@ -155,9 +191,11 @@ __device__ __forceinline__ uint32_t dequant_pair_bf16(uint32_t byte, __half2 sca
     return *reinterpret_cast<const uint32_t *>(&b);
 }
 
+// Token-tile heights: 16, 32, 64, 128, then kMaxN.
+__device__ __forceinline__ int box_rows(int i) { return i < kNumBoxes - 1 ? (16 << i) : kMaxN; }
 __device__ __forceinline__ int box_index(int rows) {
     int i = 0;
-    while ((16 << i) < rows && i < kNumBoxes - 1) ++i;
+    while (box_rows(i) < rows && i < kNumBoxes - 1) ++i;
     return i;
 }
 
@@ -171,6 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
     const int KT = a.K / kTileK, RT = a.R / kM;
     const int n_tiles = __ldg(a.list_sizes + 2) * RT;
     if ((int)blockIdx.x >= n_tiles) return;
+    constexpr uint32_t kType = (P == Proj::GateUp) ? 0u : 1u;   // f16 : bf16
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -178,8 +217,14 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
             mbar_init(&sm.empty[s], 1);
             mbar_init(&sm.aready[s], 128);
         }
-        mbar_init(&sm.dfull, 1);
-        mbar_init(&sm.dempty, 128);
+        for (int c = 0; c < kCStages; ++c) {
+            mbar_init(&sm.cfull[c], 1);
+            mbar_init(&sm.cempty[c], 128);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.dfull[b], 1);
+            mbar_init(&sm.dempty[b], 256);
+        }
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -192,131 +237,214 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+#ifdef TFMOE_MMA_STATS
+    const long long t_kernel0 = clock64();
+#endif
 
-    if (warp == 0) {
+    if (warp == 0 || warp == 2) {
+        // warp 0: token tiles into the 8-stage ring (freed by the MMA commit);
+        // warp 2: code/scale tiles into the 16-stage ring (freed once decoded)
         if (lane == 0) {
-            uint32_t g = 0;
-            uint32_t issued = 0;
+            const bool tokens = (warp == 0);
+            const int nst = tokens ? kStages : kCStages;
+            uint32_t g = 0, issued = 0;
             for (int t = blockIdx.x; t < n_tiles && !sm.abort_flag; t += gridDim.x) {
                 const int32_t *ent = a.entries + 4 * (t / RT);
                 const int e = __ldg(ent), row0 = __ldg(ent + 1), rows = __ldg(ent + 2);
                 const int rt = t % RT, bi = box_index(rows);
-                const uint32_t b_bytes = (uint32_t)(16 << bi) * 128u;
+                const uint32_t b_bytes = (uint32_t)box_rows(bi) * 128u;
                 const size_t rti = (size_t)e * RT + rt;
                 for (int kt = 0; kt < KT; ++kt, ++g) {
-                    const int s = g % kStages;
-                    const uint32_t ph = (g / kStages) & 1u;
-                    if (!wait_or_abort(&sm.empty[s], ph ^ 1u, sm, a.err_word)) break;
-                    mbar_arrive_expect_tx(&sm.full[s], b_bytes + kTileCodeBytes + kTileScaleBytes);
-                    tma_load_2d(sm.b[s], &maps.box[bi], kt * kTileK, row0, &sm.full[s]);
-                    bulk_g2s(sm.codes[s], a.codes + (rti * KT + kt) * kTileCodeBytes, kTileCodeBytes, &sm.full[s]);
-                    bulk_g2s(sm.scales[s], a.scales + scale_offset(rti, KT, 0, kt), kTileScaleBytes / 2, &sm.full[s]);
-                    bulk_g2s(sm.scales[s] + kTileScaleBytes / 2, a.scales + scale_offset(rti, KT, 1, kt),
-                             kTileScaleBytes / 2, &sm.full[s]);
+                    const int s = g % nst;
+                    const uint32_t ph = (g / nst) & 1u;
+                    if (tokens) {
+                        if (!STAT_WAIT(0, wait_or_abort(&sm.empty[s], ph ^ 1u, sm, a.err_word))) break;
+                        mbar_arrive_expect_tx(&sm.full[s], b_bytes);
+                        tma_load_2d(sm.b[s], &maps.box[bi], kt * kTileK, row0, &sm.full[s]);
+                    } else {
+                        if (!STAT_WAIT(1, wait_or_abort(&sm.cempty[s], ph ^ 1u, sm, a.err_word))) break;
+                        mbar_arrive_expect_tx(&sm.cfull[s], kTileCodeBytes + kTileScaleBytes);
+                        bulk_g2s(sm.codes[s], a.codes + (rti * KT + kt) * kTileCodeBytes, kTileCodeBytes, &sm.cfull[s]);
+                        bulk_g2s(sm.scales[s], a.scales + scale_offset(rti, KT, 0, kt), kTileScaleBytes / 2,
+                                 &sm.cfull[s]);
+                        bulk_g2s(sm.scales[s] + kTileScaleBytes / 2, a.scales + scale_offset(rti, KT, 1, kt),
+                                 kTileScaleBytes / 2, &sm.cfull[s]);
+                    }
                     issued = g + 1;
                 }
             }
             if (sm.abort_flag) {
                 // aborted: let the copies already issued land before the CTA exits (bounded)
-                for (uint32_t j = (issued > kStages ? issued - kStages : 0); j < issued; ++j) {
+                for (uint32_t j = (issued > (uint32_t)nst ? issued - nst : 0); j < issued; ++j) {
+                    uint64_t *bar = tokens ? &sm.full[j % nst] : &sm.cfull[j % nst];
                     const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(&sm.full[j % kStages], (j / kStages) & 1u) &&
-                           global_timer_ns() - t0 < kWaitLimitNs / 4) {
+                    while (!mbar_try_wait(bar, (j / nst) & 1u) && global_timer_ns() - t0 < kWaitLimitNs / 4) {
                     }
                 }
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
+            // one wait per stage (the decoders also wait for the token tile), descriptors
+            // advanced by adds, one commit per stage: the issuing thread does little else
+            const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sm.b[0]));
             uint32_t g = 0, tile_i = 0;
             for (int t = blockIdx.x; t < n_tiles && !sm.abort_flag; t += gridDim.x, ++tile_i) {
                 const int rows = __ldg(a.entries + 4 * (t / RT) + 2);
-                const int n = 16 << box_index(rows);
-                const uint32_t idesc = instr_desc_bf16(n);
-                if (!wait_or_abort(&sm.dempty, (tile_i & 1u) ^ 1u, sm, a.err_word)) break;
+                const uint32_t idesc = instr_desc_16bit(box_rows(box_index(rows)), kType);
+                const int buf = tile_i & 1;
+                if (!STAT_WAIT(2, wait_or_abort(&sm.dempty[buf], ((tile_i >> 1) & 1u) ^ 1u, sm, a.err_word))) break;
                 tc_fence_after();
+                const uint32_t dt = tmem + (uint32_t)buf * kMaxN;
                 bool ok = true;
                 for (int kt = 0; kt < KT; ++kt, ++g) {
                     const int s = g % kStages;
                     const uint32_t ph = (g / kStages) & 1u;
-                    if (!wait_or_abort(&sm.full[s], ph, sm, a.err_word) ||
-                        !wait_or_abort(&sm.aready[s], ph, sm, a.err_word)) { ok = false; break; }
+                    if (!STAT_WAIT(4, wait_or_abort(&sm.aready[s], ph, sm, a.err_word))) { ok = false; break; }
+#ifdef TFMOE_MMA_STATS
+                    const long long tm0 = clock64();
+#endif
                     tc_fence_after();
-                    const uint32_t b0 = smem_u32(sm.b[s]);
-#pragma unroll
-                    for (int k4 = 0; k4 < kTileK / 16; ++k4)
-                        mma_bf16_ts(tmem + kAccCol, tmem + kACol + (uint32_t)s * 32u + (uint32_t)k4 * 8u,
-                                    smem_desc_sw128(b0 + (uint32_t)k4 * 32u), idesc, (kt | k4) != 0);
+                    const uint64_t bd = bdesc0 + (uint64_t)(s * (kBStageBytes >> 4));
+                    const uint32_t ad = tmem + kACol + (uint32_t)s * 32u;
+                    mma_16bit_ts(dt, ad, bd, idesc, kt != 0);
+                    mma_16bit_ts(dt, ad + 8u, bd + 2u, idesc, 1u);
+                    mma_16bit_ts(dt, ad + 16u, bd + 4u, idesc, 1u);
+                    mma_16bit_ts(dt, ad + 24u, bd + 6u, idesc, 1u);
+#ifdef TFMOE_MMA_STATS
+                    const long long tm1 = clock64();
+#endif
                     mma_commit(&sm.empty[s]);
+#ifdef TFMOE_MMA_STATS
+                    const long long tm2 = clock64();
+                    g_mma_stats[blockIdx.x % 160][10] += (unsigned long long)(tm1 - tm0);
+                    g_mma_stats[blockIdx.x % 160][11] += (unsigned long long)(tm2 - tm1);
+#endif
                 }
                 if (!ok) break;
-                mma_commit(&sm.dfull);
+                mma_commit(&sm.dfull[buf]);
             }
         }
-    } else if (warp >= kDequantWarp0) {
-        const int q = threadIdx.x - kDequantWarp0 * 32;          // weight row of the tile = TMEM lane
-        const uint32_t lane_base = (uint32_t)((warp - kDequantWarp0) * 32) << 16;
-        uint32_t g = 0, tile_i = 0;
-        for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tile_i) {
-            const int32_t *ent = a.entries + 4 * (t / RT);
-            const int e = __ldg(ent), row0 = __ldg(ent + 1), rows = __ldg(ent + 2);
-            const int rt = t % RT;
-            const int n = 16 << box_index(rows);
-            bool ok = !sm.abort_flag;
-            for (int kt = 0; kt < KT && ok; ++kt, ++g) {
-                const int s = g % kStages;
-                const uint32_t ph = (g / kStages) & 1u;
-                ok = wait_or_abort(&sm.full[s], ph, sm, a.err_word);
-                if (ok) ok = wait_or_abort(&sm.empty[s], ph ^ 1u, sm, a.err_word);   // A stage free
+    } else if (warp >= kDqWarp0 && warp < kEpiWarp0) {
+        // decode: warpgroup gq takes the stages g with g % 2 == gq (all 64 columns), so two
+        // stages are decoded concurrently; thread q owns weight row q = TMEM lane q
+        const int gq = (warp - kDqWarp0) >> 2;
+        const int q = (warp & 3) * 32 + lane;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        uint32_t g = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+            for (int kt = 0; kt < KT; ++kt, ++g) {
+                if ((int)(g & 1u) != gq) continue;
+                const int s = g % kStages, cs = g % kCStages;
+                const uint32_t ph = (g / kStages) & 1u, pc = (g / kCStages) & 1u;
+                ok = (lane == 0) ? STAT_WAIT(5, wait_or_abort(&sm.cfull[cs], pc, sm, a.err_word))
+                                 : wait_or_abort(&sm.cfull[cs], pc, sm, a.err_word);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-                const uint4 c0 = *reinterpret_cast<const uint4 *>(sm.codes[s] + q * 16);
-                const uint4 c1 = *reinterpret_cast<const uint4 *>(sm.codes[s] + 2048 + q * 16);
-                const uint32_t sc4 = *reinterpret_cast<const uint32_t *>(sm.scales[s] + q * 4);
+                const uint4 c0 = *reinterpret_cast<const uint4 *>(sm.codes[cs] + q * 16);
+                const uint4 c1 = *reinterpret_cast<const uint4 *>(sm.codes[cs] + 2048 + q * 16);
+                const uint32_t sc4 = *reinterpret_cast<const uint32_t *>(sm.scales[cs] + q * 4);
+                mbar_arrive(&sm.cempty[cs]);                              // code stage consumed
+                ok = (lane == 0) ? STAT_WAIT(6, wait_or_abort(&sm.empty[s], ph ^ 1u, sm, a.err_word))
+                                 : wait_or_abort(&sm.empty[s], ph ^ 1u, sm, a.err_word);  // A stage free
+                if (ok) ok = wait_or_abort(&sm.full[s], ph, sm, a.err_word);             // token tile landed
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 const uint32_t s01 = e4m3x2_to_f16x2(sc4 & 0xFFFFu), s23 = e4m3x2_to_f16x2(sc4 >> 16);
                 const __half2 h01 = *reinterpret_cast<const __half2 *>(&s01);
                 const __half2 h23 = *reinterpret_cast<const __half2 *>(&s23);
                 const __half2 sb[4] = {__low2half2(h01), __high2half2(h01), __low2half2(h23), __high2half2(h23)};
                 const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                uint32_t r[32];
 #pragma unroll
-                for (int w8 = 0; w8 < 8; ++w8)       // word w8 holds elements 8*w8 .. 8*w8 + 7
+                for (int hh = 0; hh < 2; ++hh) {      // columns 0..31, then 32..63
+                    uint32_t r[16];
 #pragma unroll
-                    for (int b = 0; b < 4; ++b)
-                        r[4 * w8 + b] = dequant_pair_bf16((words[w8] >> (8 * b)) & 0xFFu, sb[w8 >> 1]);
-                tmem_st32(tmem + lane_base + kACol + (uint32_t)s * 32u, r);
+                    for (int w4 = 0; w4 < 4; ++w4)    // word holds elements 8*w4 .. 8*w4 + 7 of the half
+#pragma unroll
+                        for (int b = 0; b < 4; ++b) {
+                            const uint32_t byte = (words[4 * hh + w4] >> (8 * b)) & 0xFFu;
+                            const __half2 sc = sb[2 * hh + (w4 >> 1)];
+                            r[4 * w4 + b] = (kType == 0u) ? dequant_pair_f16(byte, sc) : dequant_pair_bf16(byte, sc);
+                        }
+                    tmem_st16(tmem + lane_base + kACol + (uint32_t)s * 32u + (uint32_t)hh * 16u, r);
+                }
                 tc_wait_st();
                 tc_fence_before();
                 mbar_arrive(&sm.aready[s]);
+#ifdef TFMOE_MMA_STATS
+                if (lane == 0) atomicAdd(&g_mma_stats[blockIdx.x % 160][9], 1ull);
+#endif
             }
-            if (!ok) break;
-            // epilogue: this thread's row of D, N token columns
-            if (!wait_or_abort(&sm.dfull, tile_i & 1u, sm, a.err_word)) break;
+        }
+    } else if (warp >= kEpiWarp0) {
+        // two warpgroups split the accumulator columns in steps of 16; one buffer behind the MMAs
+        const int eg = (warp - kEpiWarp0) >> 2;
+        const int ew = warp - kEpiWarp0;                           // 0..7: staging slot
+        const int q = (warp & 3) * 32 + lane;                      // weight row = TMEM lane
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        uint32_t tile_i = 0;
+        for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tile_i) {
+            const int32_t *ent = a.entries + 4 * (t / RT);
+            const int e = __ldg(ent), row0 = __ldg(ent + 1), rows = __ldg(ent + 2);
+            const int rt = t % RT;
+            const int n = box_rows(box_index(rows));
+            const int buf = tile_i & 1;
+            if (!((lane == 0) ? STAT_WAIT(7, wait_or_abort(&sm.dfull[buf], (tile_i >> 1) & 1u, sm, a.err_word))
+                              : wait_or_abort(&sm.dfull[buf], (tile_i >> 1) & 1u, sm, a.err_word)))
+                break;
             tc_fence_after();
             const int grow = rt * kM + q;
             const float gs = (P == Proj::GateUp) ? ((grow & 1) ? __ldg(a.glob1 + e) : __ldg(a.glob0 + e))
                                                  : __ldg(a.glob0 + e);
-            for (int c = 0; c < n; c += 32) {
-                uint32_t d[32];
-                tmem_ld32(tmem + lane_base + kAccCol + (uint32_t)c, d);
+            // this group's steps: eg 0 takes steps 0, 2, 4, ..., eg 1 takes 1, 3, 5, ...
+            const int steps = n / kEpiCols;
+            bool handed_back = false;
+            for (int st = eg; st < steps; st += 2) {
+                const int c = st * kEpiCols;
+                uint32_t d[16];
+                tmem_ld16(tmem + lane_base + (uint32_t)buf * kMaxN + (uint32_t)c, d);
                 tc_wait_ld();
+                if (st + 2 >= steps) {           // last read of this group: hand the buffer back
+                    tc_fence_before();
+                    mbar_arrive(&sm.dempty[buf]);
+                    handed_back = true;
+                }
+                if (P == Proj::GateUp) {
+                    // even lane 2i holds gate j = (grow >> 1), lane 2i+1 the up row of the same j;
+                    // stage a[16 tokens][16 j] in shared memory, then write 16-byte row pieces
+                    const float xi = (lane < kEpiCols && c + lane < rows) ? __ldg(a.row_inv_scale + row0 + c + lane) : 0.f;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float v = __uint_as_float(d[i]) * gs;
-                    const int tok = c + i;
-                    if (P == Proj::GateUp) {
+                    for (int i = 0; i < kEpiCols; ++i) {
+                        const float v = __uint_as_float(d[i]) * gs * __shfl_sync(0xffffffffu, xi, i);
                         const float other = __shfl_xor_sync(0xffffffffu, v, 1);
-                        if (!(grow & 1) && tok < rows)
-                            a.act_out[(size_t)(row0 + tok) * a.I + (grow >> 1)] = float_to_bf16_bits_rn(silu_f32(v) * other);
-                    } else {
-                        if (tok < rows) a.y_out[(size_t)(row0 + tok) * a.R + grow] = v;
+                        if (!(lane & 1)) sm.stage_out[ew][i][lane >> 1] = float_to_bf16_bits_rn(silu_f32(v) * other);
+                    }
+                    __syncwarp();
+                    // 16 tokens x 32 bytes: lane l writes token l/2, bytes 16*(l&1) .. +16
+                    const int tok = c + (lane >> 1);
+                    if (tok < rows) {
+                        const uint4 v4 = *reinterpret_cast<const uint4 *>(&sm.stage_out[ew][lane >> 1][8 * (lane & 1)]);
+                        const int j0 = (rt * kM + (warp & 3) * 32) / 2 + 8 * (lane & 1);
+                        *reinterpret_cast<uint4 *>(a.act_out + (size_t)(row0 + tok) * a.I + j0) = v4;
+                    }
+                    __syncwarp();
+                } else {
+#pragma unroll
+                    for (int i = 0; i < kEpiCols; ++i) {
+                        const int tok = c + i;
+                        if (tok < rows) a.y_out[(size_t)(row0 + tok) * a.R + grow] = __uint_as_float(d[i]) * gs;
                     }
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&sm.dempty);
+            if (!handed_back) {                  // no step for this group in this tile
+                tc_fence_before();
+                mbar_arrive(&sm.dempty[buf]);
+            }
         }
     }
     __syncthreads();
+#ifdef TFMOE_MMA_STATS
+    if (threadIdx.x == 0) atomicAdd(&g_mma_stats[blockIdx.x % 160][8], (unsigned long long)(clock64() - t_kernel0));
+#endif
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
@@ -324,22 +452,54 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
     }
 }
 
-// x_perm[r] = x[token of pair perm[r]] for the rows of every MMA token tile.
+// x_perm[r] = f16(x[token of pair perm[r]] * 2^sh_r) for the rows of every MMA token
+// tile, sh_r the power of two that puts the row's largest magnitude just below
+// 2^15 (exact for every element within 2^28 of the largest); row_inv[r] = 2^-sh_r.
 __global__ void __launch_bounds__(256) gather_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ perm,
                                                      const int32_t *__restrict__ entries,
                                                      const int32_t *__restrict__ list_sizes, int H, int k,
-                                                     uint16_t *__restrict__ x_perm)
+                                                     uint16_t *__restrict__ x_perm, float *__restrict__ row_inv)
 {
+    __shared__ uint32_t wmax[8];
     const int ent = blockIdx.x;
     if (ent >= __ldg(list_sizes + 2)) return;
     const int row0 = __ldg(entries + 4 * ent + 1), rows = __ldg(entries + 4 * ent + 2);
     const int chunks = H / 8;
     for (int rr = blockIdx.y; rr < rows; rr += gridDim.y) {
         const int r = row0 + rr;
-        const uint16_t *src = x + (size_t)(__ldg(perm + r) / k) * H;
-        uint16_t *dst = x_perm + (size_t)r * H;
-        for (int c = threadIdx.x; c < chunks; c += blockDim.x)
-            reinterpret_cast<uint4 *>(dst)[c] = __ldg(reinterpret_cast<const uint4 *>(src) + c);
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)(__ldg(perm + r) / k) * H);
+        uint4 *dst = reinterpret_cast<uint4 *>(x_perm + (size_t)r * H);
+        uint32_t emax = 0;
+        for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+            const uint4 v = __ldg(src + c);
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) emax = max(emax, max((u[j] >> 7) & 0xFFu, (u[j] >> 23) & 0xFFu));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
+        if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = emax;
+        __syncthreads();
+        emax = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) emax = max(emax, wmax[w]);
+        __syncthreads();
+        int sh = 14 - ((int)emax - 127);
+        sh = max(-120, min(120, sh));
+        const float up = __int_as_float((127 + sh) << 23);
+        if (threadIdx.x == 0) row_inv[r] = __int_as_float((127 - sh) << 23);
+        for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+            const uint4 v = __ldg(src + c);
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const __half lo = __float2half_rn(bf16_bits_to_float(u[j] & 0xFFFFu) * up);
+                const __half hi = __float2half_rn(bf16_bits_to_float(u[j] >> 16) * up);
+                o[j] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+            }
+            dst[c] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
     }
 }
 
@@ -363,15 +523,15 @@ EncodeTiledFn encode_tiled_fn() {
     return fn;
 }
 
-CUresult make_token_maps(TokenMaps &m, void *base, int cols, int rows) {
+CUresult make_token_maps(TokenMaps &m, void *base, int cols, int rows, CUtensorMapDataType type) {
     EncodeTiledFn encode = encode_tiled_fn();
     if (!encode) return CUDA_ERROR_NOT_FOUND;
     for (int i = 0; i < kNumBoxes; ++i) {
         const cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
         const cuuint64_t gstride[1] = {(cuuint64_t)cols * 2};
-        const cuuint32_t box[2] = {(cuuint32_t)kTileK, (cuuint32_t)(16 << i)};
+        const cuuint32_t box[2] = {(cuuint32_t)kTileK, (cuuint32_t)(i < kNumBoxes - 1 ? (16 << i) : kMaxN)};
         const cuuint32_t estride[2] = {1, 1};
-        CUresult r = encode(&m.box[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, gdim, gstride, box,
+        CUresult r = encode(&m.box[i], type, 2, base, gdim, gstride, box,
                                             estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return r;
@@ -390,8 +550,8 @@ cudaError_t mma_setup(Layer &L)
     const int maxP = L.desc.max_tokens * L.desc.top_k;
     MmaMaps *mm = new (std::nothrow) MmaMaps();
     if (!mm) return cudaErrorMemoryAllocation;
-    if (make_token_maps(mm->x_perm, L.ws.x_perm, L.desc.hidden, maxP) != CUDA_SUCCESS ||
-        make_token_maps(mm->act, L.ws.act, L.desc.intermediate, maxP) != CUDA_SUCCESS) {
+    if (make_token_maps(mm->x_perm, L.ws.x_perm, L.desc.hidden, maxP, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) != CUDA_SUCCESS ||
+        make_token_maps(mm->act, L.ws.act, L.desc.intermediate, maxP, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) != CUDA_SUCCESS) {
         delete mm;
         return cudaErrorInvalidValue;
     }
@@ -416,7 +576,7 @@ cudaError_t launch_gather(Layer &L, const uint16_t *x, int T, cudaStream_t s, in
     const int P = T * L.desc.top_k;
     dim3 grid((unsigned)max_mma_entries(P, L.desc.num_experts), 16);
     gather_kernel<<<grid, 256, 0, s>>>(x, L.ws.perm, L.ws.mma_entries, L.ws.list_sizes, L.desc.hidden,
-                                       L.desc.top_k, L.ws.x_perm);
+                                       L.desc.top_k, L.ws.x_perm, L.ws.row_inv);
     *launches += 1;
     return cudaGetLastError();
 }
@@ -438,6 +598,7 @@ cudaError_t launch_mma_gate_up(Layer &L, cudaStream_t s, int *launches)
     a.glob0 = L.w.gate_global; a.glob1 = L.w.up_global;
     a.R = 2 * L.desc.intermediate; a.K = L.desc.hidden;
     a.act_out = L.ws.act;
+    a.row_inv_scale = L.ws.row_inv;
     const MmaMaps *mm = static_cast<const MmaMaps *>(L.mma_maps);
     mma_kernel<Proj::GateUp><<<L.num_sms, kThreads, mma_smem_bytes(), s>>>(mm->x_perm, a);
     *launches += 1;
@@ -459,3 +620,15 @@ cudaError_t launch_mma_down(Layer &L, cudaStream_t s, int *launches)
 }
 
 }  // namespace tfmoe
+
+#ifdef TFMOE_MMA_STATS
+extern "C" __attribute__((visibility("default"))) int tfmoe_debug_mma_stats(unsigned long long *out, int clear)
+{
+    if (cudaMemcpyFromSymbol(out, tfmoe::g_mma_stats, sizeof(tfmoe::g_mma_stats)) != cudaSuccess) return 1;
+    if (clear) {
+        static unsigned long long zeros[160][tfmoe::kStatSlots];
+        if (cudaMemcpyToSymbol(tfmoe::g_mma_stats, zeros, sizeof(zeros)) != cudaSuccess) return 1;
+    }
+    return 0;
+}
+#endif
