@@ -225,6 +225,8 @@ def main():
     ap.add_argument("--impl", choices=["tfmoe", "reference"], default="tfmoe")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
     ap.add_argument("--flags", type=int, default=0, help="descriptor flags (1 = force GEMV, 2 = force MMA)")
+    ap.add_argument("--gemv-max-tokens", type=int, default=0,
+                    help="per-expert token count up to which the GEMV regime is used (0 = library default)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", type=int, default=100, help="forwards per CUDA graph (0 = no graphs)")
@@ -248,7 +250,8 @@ def main():
     for s in seeds:
         lnp = synth.make_layer(shape, s + 1000 * rank) if rank else synth.make_layer(shape, s)
         layers_np.append(lnp)
-        L = tfmoe.MoELayer(H, I, E, k, T, has_router_bias=lnp["router_bias"] is not None, flags=args.flags)
+        L = tfmoe.MoELayer(H, I, E, k, T, has_router_bias=lnp["router_bias"] is not None, flags=args.flags,
+                           gemv_max_tokens=args.gemv_max_tokens)
         L.load_weights(tfmoe.layer_to_device(lnp, dev))
         layers.append(L)
         xs.append([torch.from_numpy(synth.make_x(shape, s, T, stream=r + 100 * rank).view(np.int16)).to(dev)
@@ -486,7 +489,8 @@ def main():
                                    f"seeds {list(seeds)} rotated", "global_batch": T * world,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2: rotating seeded layers / full weight sets exceed 126 MB",
-                       "flags": args.flags, "graph_forwards": G},
+                       "flags": args.flags, "gemv_max_tokens": args.gemv_max_tokens or "default",
+                       "graph_forwards": G},
             "roofline": roofline,
             "layer": {"algorithmic_bytes_per_forward": bytes_per_fwd, "hbm_gbs": layer_gbs,
                       "hbm_frac": layer_gbs / hbm_peak, "hbm_frac_of_8tbs": layer_gbs / 8000.0,

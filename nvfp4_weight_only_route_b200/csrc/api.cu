@@ -78,6 +78,10 @@ void carve_workspace(Layer &L, uint8_t *base, size_t *total) {
     c.take(&w.x_perm, P * H, base);
     c.take(&w.row_inv, P, base);
     c.take(&w.act, P * I, base);
+    c.take(&w.xq, T * H, base);
+    c.take(&w.xq_inv, T * H / 16, base);
+    c.take(&w.aq, P * I, base);
+    c.take(&w.aq_inv, P * I / 16, base);
     c.take(&w.y, P * H, base);
     c.take(&w.x_stage, T * H, base);
     c.take(&w.out_stage, T * H, base);
@@ -147,10 +151,15 @@ tfmoe_status tfmoe_create(const tfmoe_layer_desc *desc, tfmoe_layer **out)
     if (d.hidden % 128 || d.intermediate % 64)
         return fail(TFMOE_ERR_UNSUPPORTED, "this build needs hidden %% 128 == 0 and intermediate %% 64 == 0 (got %d, %d)",
                     d.hidden, d.intermediate);
+    if (d.hidden > kMaxReduction || d.intermediate > kMaxReduction)
+        return fail(TFMOE_ERR_UNSUPPORTED, "this build supports hidden and intermediate up to %d (got %d, %d)",
+                    kMaxReduction, d.hidden, d.intermediate);
     if (d.num_experts > 256 || d.top_k > 32)
         return fail(TFMOE_ERR_UNSUPPORTED, "this build supports num_experts <= 256 and top_k <= 32");
     if ((long long)d.max_tokens * d.top_k > (1LL << 30))
         return fail(TFMOE_ERR_UNSUPPORTED, "max_tokens * top_k too large");
+    if ((long long)d.max_tokens * d.top_k * (d.hidden > d.intermediate ? d.hidden : d.intermediate) >= (1LL << 32))
+        return fail(TFMOE_ERR_UNSUPPORTED, "max_tokens * top_k * max(hidden, intermediate) must stay below 2^32");
 
     const char *fail_env = getenv("TFMOE_FAIL_ALLOC");
     if (fail_env && atoi(fail_env) != 0)
@@ -183,6 +192,7 @@ tfmoe_status tfmoe_create(const tfmoe_layer_desc *desc, tfmoe_layer **out)
     if (e == cudaSuccess) e = mma_setup(L);
     if (e != cudaSuccess) {
         mma_teardown(L);
+        gemv_teardown(L);
         cudaFree(L.ws_block);
         cudaFree(L.w_block);
         delete h;
@@ -334,6 +344,7 @@ void tfmoe_destroy(tfmoe_layer *layer)
         if (L.ws_block) cudaFree(L.ws_block);
         if (L.w_block) cudaFree(L.w_block);
         mma_teardown(L);
+        gemv_teardown(L);
     }
     delete layer;
 }

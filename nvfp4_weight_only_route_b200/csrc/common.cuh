@@ -1,6 +1,7 @@
 // common.cuh -- small device helpers shared by the libtfmoe kernels (sm_100a).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -60,13 +61,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
         : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
     return ok != 0;
 }
+// As mbar_try_wait, but a thread whose phase is not complete is suspended (up to
+// kSuspendHintNs) instead of returning at once, so waiting warps do not take issue
+// slots from the warps doing the work.
+constexpr uint32_t kSuspendHintNs = 20000;
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs) : "memory");
+    return ok != 0;
+}
 // Bounded wait: returns false (and sets the error word) when the limit passes.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, int32_t *err_word) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
-        for (int i = 0; i < 256; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+        for (int i = 0; i < 4; ++i)
+            if (mbar_try_wait_sleep(bar, parity)) return true;
         if (global_timer_ns() - t0 > kWaitLimitNs) {
             if (err_word) atomicOr(err_word, DEV_ERR_WAIT_TIMEOUT);
             return false;
@@ -82,12 +96,29 @@ __device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gmem_src, u
         ::"r"(smem_u32(smem_dst)), "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
 
+// 2-D tensor copy global -> shared (box given by the tensor map), completing on an
+// mbarrier. The innermost coordinate times the element size must be a multiple of 16.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar)) : "memory");
+}
+
 // ---------------------------------------------------------------- formats
 // Two E2M1 codes (one byte: element 2i low nibble, 2i+1 high nibble) -> f16x2.
 __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
     uint32_t out;
     asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(out) : "r"(byte));
     return out;
+}
+// Eight E2M1 codes (one 32-bit word; byte i holds elements 2i (low nibble) and 2i+1)
+// -> four f16x2. Unpacking the word into byte registers lets each conversion read its
+// byte directly (about one instruction per pair instead of shift, mask and convert).
+__device__ __forceinline__ void e2m1x8_to_f16x2x4(uint32_t w, uint32_t (&o)[4]) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3]) : "r"(w));
 }
 // Two E4M3 bytes (low byte first) -> f16x2 (exact: every E4M3 value is an f16 value).
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
@@ -106,6 +137,32 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {
 __device__ __forceinline__ uint16_t float_to_bf16_bits_rn(float f) {
     __nv_bfloat16 b = __float2bfloat16_rn(f);
     return *reinterpret_cast<uint16_t *>(&b);
+}
+
+// Sixteen bf16 values -> f16 values times 2^sh, sh chosen from the block's largest
+// exponent so that the largest magnitude lands in [2^14, 2^15). Every bf16 element
+// within 2^28 of the block's largest is then an exact f16 (its 8-bit significand stays
+// above the f16 normal range); returns 2^-sh. src and dst 16-byte aligned.
+__device__ __forceinline__ float block16_bf16_to_f16(const uint16_t *src, uint16_t *dst) {
+    const uint4 v0 = *reinterpret_cast<const uint4 *>(src);
+    const uint4 v1 = *reinterpret_cast<const uint4 *>(src + 8);
+    const uint32_t u[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    uint32_t emax = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) emax = max(emax, max((u[j] >> 7) & 0xFFu, (u[j] >> 23) & 0xFFu));
+    int sh = 14 - ((int)emax - 127);
+    sh = max(-120, min(120, sh));
+    const float up = __int_as_float((127 + sh) << 23);
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const __half lo = __float2half_rn(bf16_bits_to_float(u[j] & 0xFFFFu) * up);
+        const __half hi = __float2half_rn(bf16_bits_to_float(u[j] >> 16) * up);
+        o[j] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+    }
+    *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4 *>(dst + 8) = make_uint4(o[4], o[5], o[6], o[7]);
+    return __int_as_float((127 - sh) << 23);
 }
 
 // z * sigmoid(z); exp and reciprocal on the special-function unit (relative error

@@ -6,90 +6,129 @@
 // page, section "Mechanism: decode is bandwidth-bound, prefill is
 // compute-bound"); the expert up/down kernels are the largest share of decode
 // GPU time in TensorFold issue #627 (comment with the RTX 4090 per-launch
-// table). The kernel streams the packed codes with 128-bit coalesced loads
-// (16 in flight per lane), stages the E4M3 block scales into shared memory
-// with bulk (TMA) copies one task ahead, keeps the routed activation rows in
-// shared memory, and combines the two half-rows with a warp shuffle.
+// table). So the kernel is built around the memory stream: the packed codes
+// arrive with 128-bit coalesced loads, double-buffered in registers across
+// column chunks and prefetched across tasks; each task's E4M3 block scales
+// arrive in shared memory with one 2-D tensor copy (TMA) issued a task ahead;
+// the inner loop spends about one instruction per weight and token.
 //
-// Work item: (expert in the GEMV list, block of 64 weight rows). A CTA of 4
-// warps covers the 64 rows; lane l of warp w owns row 16w + (l % 16) and half
-// (l / 16) of every 64-column tile (16 code bytes = 32 weights, 2 scale bytes)
-// and accumulates across all tiles of the row.
+// Task = (expert of the GEMV list, 16*RG consecutive weight rows). The 8 warps
+// of a CTA split it as RG row groups x KS column slices (RG * KS = 8): lane l
+// of a warp owns row (l % 16) of its group and half (l / 16) of every 64-column
+// tile of its slice (16 code bytes = 32 weights, 2 scale bytes). Partial sums
+// leave the warp through a shuffle (the two halves) and shared memory (the
+// slices), added in a fixed order; then the epilogue threads (one per row and
+// token) apply the per-tensor scale and either SwiGLU (gate/up) or the fp32
+// store (down). Tasks are small so that the few waves of a decode step stay
+// balanced across the CTAs.
 //
-// Inner products (per 16-element block b of a lane's 32 weights):
-//   partial_b = sum of w*x in fp32, acc += scale_b * partial_b, and the
-//   per-tensor scale multiplies the finished sum.
-// Two forms, chosen at compile time:
-//   kMathF32  : E2M1 -> f16 (exact) -> fp32, x in fp32, packed fp32x2 FMAs.
-//   kMathF16  : E2M1 -> f16 (exact), x as f16 times a power of two per
-//               32-element block (exact for every bf16 value within 2^28 of the
-//               block's largest), single-rounding f16*f16+f32 FMAs; the block's
-//               power of two is folded into the scale.
-// Gate/up rows are interleaved (row 2j = gate j, 2j+1 = up j), so lanes l and
-// l^1 hold G and U of the same j and the SwiGLU epilogue
-// a = bf16(silu(G) * U) runs in registers.
+// Arithmetic: the activation operand is an f16 tensor with one power of two
+// per 16 elements (exact for every bf16 element within 2^28 of its block's
+// largest; the routing kernels write it for x, the gate/up epilogue for the
+// SwiGLU output a). E2M1 -> f16 is exact and each product w*x is exact inside
+// one mixed-precision fma.rn.f32.f16, so a 16-element partial sum is an fp32
+// sum of exact products; it is scaled by (E4M3 block scale * inverse power of
+// two of the activation block, an exact product) into the fp32 row accumulator.
+#include <new>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace tfmoe {
 namespace {
 
-constexpr int kRowsPerTask = 64;
-constexpr int kWarps = 4;
-constexpr int kThreads = kWarps * 32;
-constexpr int kTokGroup = 4;      // activation rows staged per pass
-constexpr int kBatch = 8;         // 64-column tiles per load batch (two batches in flight per lane)
-constexpr int kMathF32 = 0, kMathF16 = 1;
-#ifndef TFMOE_GEMV_MATH
-#define TFMOE_GEMV_MATH 1
+constexpr int kWarps = 8;                       // compute warps (column slices x row groups)
+constexpr int kComputeWarps = kWarps;
+constexpr int kThreads = (kComputeWarps + 1) * 32;   // + the control warp
+#ifndef TFMOE_GEMV_CTAS_PER_SM
+#define TFMOE_GEMV_CTAS_PER_SM 2
 #endif
-constexpr int kMath = TFMOE_GEMV_MATH;
+#ifndef TFMOE_GEMV_TOKENS_PER_PASS
+#define TFMOE_GEMV_TOKENS_PER_PASS 2
+#endif
+constexpr int kCtasPerSm = TFMOE_GEMV_CTAS_PER_SM;
+#ifndef TFMOE_GEMV_RING
+#define TFMOE_GEMV_RING 6
+#endif
+constexpr int kChunk = 2;          // column tiles per ring slot of a compute warp
+constexpr int kRing = TFMOE_GEMV_RING;   // ring slots per compute warp (kRing - 1 chunks in flight)
+static_assert(kRing >= 3, "ring depth");
+constexpr int kMaxNT = TFMOE_GEMV_TOKENS_PER_PASS;   // tokens per pass (2 or 4)
+static_assert(kMaxNT == 2 || kMaxNT == 4, "tokens per pass");
 
 enum class Proj { GateUp, Down };
 
 struct GemvArgs {
     const uint8_t *codes;       // tiled codes of all experts
-    const uint8_t *scales;      // tiled scales of all experts
     const float *glob0;         // gate (GateUp) or down (Down) per-tensor scale [E]
     const float *glob1;         // up (GateUp)
     int R, K;                   // rows (2I or H) and reduction length (H or I)
+    int KS, RG;                 // column slices and 16-row groups of a task
     const int32_t *expert_list; // GEMV-regime experts
     const int32_t *list_size;   // [0] = number of GEMV experts
     const int32_t *offsets;     // [E+1]
     const int32_t *perm;        // [P] pair index of permuted row
     int top_k;
-    const uint16_t *src;        // GateUp: x [T][H]; Down: act [P][I]
-    uint16_t *act_out;          // GateUp output [P][I]
+    const uint16_t *src;        // GateUp: xq [T][H] (token rows); Down: aq [P][I] (permuted rows)
+    const float *src_inv;       // [rows][K/16] inverse powers of two of src
+    uint16_t *act_out;          // GateUp: act [P][I] bf16
+    uint16_t *aq_out;           // GateUp: aq [P][I]
+    float *aq_inv_out;          // GateUp: [P][I/16]
     float *y_out;               // Down output [P][H]
     int I;
     int32_t *err_word;
 };
 
-__device__ __forceinline__ uint32_t byte_of(uint32_t w, int b) { return (w >> (8 * b)) & 0xFFu; }
+struct Geometry {
+    int KS, RG;
+};
 
-// fp32 x and weights widened to fp32; two interleaved fp32x2 accumulators per block.
-__device__ __forceinline__ void dot_f32(const uint4 c, const float *xrow, float &p0, float &p1) {
-    const uint32_t words[4] = {c.x, c.y, c.z, c.w};
-    float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
-    const float4 *xp = reinterpret_cast<const float4 *>(xrow);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const float4 xa = xp[2 * q], xb = xp[2 * q + 1];
-        const float2 w01 = f16x2_to_float2(e2m1x2_to_f16x2(byte_of(words[q], 0)));
-        const float2 w23 = f16x2_to_float2(e2m1x2_to_f16x2(byte_of(words[q], 1)));
-        const float2 w45 = f16x2_to_float2(e2m1x2_to_f16x2(byte_of(words[q], 2)));
-        const float2 w67 = f16x2_to_float2(e2m1x2_to_f16x2(byte_of(words[q], 3)));
-        float2 &acc = (q < 2) ? a0 : a1;
-        acc = __ffma2_rn(w01, make_float2(xa.x, xa.y), acc);
-        acc = __ffma2_rn(w23, make_float2(xa.z, xa.w), acc);
-        acc = __ffma2_rn(w45, make_float2(xb.x, xb.y), acc);
-        acc = __ffma2_rn(w67, make_float2(xb.z, xb.w), acc);
-    }
-    p0 = a0.x + a0.y;
-    p1 = a1.x + a1.y;
+// Gate/up tasks hold at least two 16-row groups (32 interleaved rows = 16 SwiGLU
+// outputs = one 16-element block of a). KT = K / 64 is even there (H % 128 == 0).
+Geometry geometry(bool gate_up, int K) {
+    const int KT = K / kTileK;
+    int KS = gate_up ? 4 : 8;
+    while (KT % KS) KS >>= 1;
+    return {KS, kWarps / KS};
 }
 
-__device__ __forceinline__ float fma_f16_f32(uint32_t w2, uint32_t x2, float acc) {
+// Shared memory of a CTA, in bytes from a 128-byte aligned base: two buffers each of
+// the task's scales [KT][16*RG] u32, the partial sums [KS][16*RG][kMaxNT] f32, the
+// pass's activation rows [kMaxNT][K] f16 and their inverse scales [kMaxNT][K/16] f32;
+// the GEMV list table [3][<= 256] i32; per compute warp a ring of kRing code chunks
+// (kChunk tiles x 32 lanes x 16 bytes); 8 mbarriers and an abort flag.
+constexpr int kMaxList = 256;
+struct SmemLayout {
+    size_t sc_sz, red_sz, x_sz, xi_sz;
+    size_t sc, red, x, xi, tab, ring, bar, total;
+    __host__ __device__ __forceinline__ SmemLayout(int K, int KS, int RG) {
+        sc_sz = ((size_t)(K / kTileK) * 16 * RG * 4 + 127) & ~static_cast<size_t>(127);
+        red_sz = (size_t)KS * 16 * RG * kMaxNT * 4;
+        x_sz = (size_t)kMaxNT * K * 2;
+        xi_sz = ((size_t)kMaxNT * (K / 16) * 4 + 127) & ~static_cast<size_t>(127);
+        sc = 0;
+        red = sc + 2 * sc_sz;
+        x = red + 2 * red_sz;
+        xi = x + 2 * x_sz;
+        tab = xi + 2 * xi_sz;
+        ring = tab + 3 * kMaxList * 4;
+        bar = ring + (size_t)kComputeWarps * kRing * kChunk * 32 * 16;
+        total = bar + 9 * sizeof(uint64_t);
+    }
+};
+size_t gemv_smem_bytes(int K, Geometry g) { return 128 + SmemLayout(K, g.KS, g.RG).total; }
+
+// 16-byte asynchronous copy global -> shared (cp.async, bypassing L1): the code stream
+// stays 128-bit coalesced loads while the data waits in shared memory, not registers.
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// acc += w * x over two f16 pairs, each product exact, one fp32 rounding per step.
+__device__ __forceinline__ float fma2_f16_f32(uint32_t w2, uint32_t x2, float acc) {
     asm("{\n\t.reg .f16 wl, wh, xl, xh;\n\t"
         "mov.b32 {wl, wh}, %1;\n\tmov.b32 {xl, xh}, %2;\n\t"
         "fma.rn.f32.f16 %0, wl, xl, %0;\n\tfma.rn.f32.f16 %0, wh, xh, %0;\n\t}"
@@ -97,283 +136,418 @@ __device__ __forceinline__ float fma_f16_f32(uint32_t w2, uint32_t x2, float acc
     return acc;
 }
 
-// f16 x (block-scaled), weights as f16, mixed-precision FMAs.
-__device__ __forceinline__ void dot_f16(const uint4 c, const uint16_t *xrow, float &p0, float &p1) {
-    const uint32_t words[4] = {c.x, c.y, c.z, c.w};
-    const uint4 *xp = reinterpret_cast<const uint4 *>(xrow);
-    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const uint4 xv = xp[q];     // 8 f16 x values for this word's 8 weights
-        const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
-        float &u = (q < 2) ? ((q & 1) ? b0 : a0) : ((q & 1) ? b1 : a1);
-#pragma unroll
-        for (int b = 0; b < 4; ++b) u = fma_f16_f32(e2m1x2_to_f16x2(byte_of(words[q], b)), xs[b], u);
-    }
-    p0 = a0 + b0;
-    p1 = a1 + b1;
-}
-
-template <Proj P>
-__device__ __forceinline__ const uint16_t *src_row(const GemvArgs &a, int r) {
-    return (P == Proj::GateUp) ? a.src + (size_t)(__ldg(a.perm + r) / a.top_k) * a.K : a.src + (size_t)r * a.K;
-}
-
-// Stage activation rows [r0, r0 + nt) into shared memory in the kernel's math form.
-template <Proj P>
-__device__ __forceinline__ void stage_x(const GemvArgs &a, int r0, int nt, float *xs32, uint16_t *xs16, float *xinv) {
-    const int K = a.K;
-    if (kMath == kMathF32) {
-        for (int i = threadIdx.x; i < nt * (K / 8); i += kThreads) {
-            const int tt = i / (K / 8), c8 = (i % (K / 8)) * 8;
-            const uint4 v = *reinterpret_cast<const uint4 *>(src_row<P>(a, r0 + tt) + c8);
-            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-            float4 lo, hi;
-            lo.x = bf16_bits_to_float(u[0] & 0xFFFFu); lo.y = bf16_bits_to_float(u[0] >> 16);
-            lo.z = bf16_bits_to_float(u[1] & 0xFFFFu); lo.w = bf16_bits_to_float(u[1] >> 16);
-            hi.x = bf16_bits_to_float(u[2] & 0xFFFFu); hi.y = bf16_bits_to_float(u[2] >> 16);
-            hi.z = bf16_bits_to_float(u[3] & 0xFFFFu); hi.w = bf16_bits_to_float(u[3] >> 16);
-            *reinterpret_cast<float4 *>(xs32 + tt * K + c8) = lo;
-            *reinterpret_cast<float4 *>(xs32 + tt * K + c8 + 4) = hi;
-        }
-    } else {
-        // one thread per (token, 32-element block): the power of two 2^sh that puts the
-        // block's largest magnitude just below 2^15 makes every element an exact f16
-        for (int i = threadIdx.x; i < nt * (K / 32); i += kThreads) {
-            const int tt = i / (K / 32), b = i % (K / 32);
-            const uint16_t *srow = src_row<P>(a, r0 + tt) + b * 32;
-            uint4 v[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) v[q] = *reinterpret_cast<const uint4 *>(srow + 8 * q);
-            uint32_t emax = 0;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint32_t u[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) emax = max(emax, max((u[j] >> 7) & 0xFFu, (u[j] >> 23) & 0xFFu));
-            }
-            int sh = 14 - ((int)emax - 127);
-            sh = max(-120, min(120, sh));
-            const float up = __int_as_float((127 + sh) << 23);       // exact powers of two
-            xinv[tt * (K / 32) + b] = __int_as_float((127 - sh) << 23);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint32_t u[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
-                uint32_t ow[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const __half lo = __float2half_rn(bf16_bits_to_float(u[j] & 0xFFFFu) * up);
-                    const __half hi = __float2half_rn(bf16_bits_to_float(u[j] >> 16) * up);
-                    ow[j] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
-                }
-                *reinterpret_cast<uint4 *>(xs16 + tt * K + b * 32 + 8 * q) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-            }
-        }
-    }
-}
-
-template <Proj P>
-__global__ void __launch_bounds__(kThreads, 4) gemv_kernel(const GemvArgs a)
+// One lane's share of n <= kChunk column tiles for NT tokens. cs points at the lane's
+// 16 code bytes of the chunk's first tile in its ring slot (tiles 32 x 16 bytes apart);
+// tile0 indexes that tile inside the warp's slice; xs / xis point (in shared memory) at
+// token 0's activation values / inverse scales at the slice's first tile and the lane's
+// half; token t's row starts K values (K/16 inverse scales) further on.
+template <int NT>
+__device__ __forceinline__ void chunk_compute(const uint4 *cs, int n, int tile0, const uint32_t *sc, int rows_task,
+                                              int h, const uint16_t *xs, const float *xis, int K,
+                                              float (&acc)[kMaxNT])
 {
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    const int K = a.K, KT = K / kTileK;
-    // layout: x rows | x block scales (f16 form) | scales [2][KT][64][4] | mbarriers[2]
-    uint8_t *p = smem_raw;
-    float *xs32 = reinterpret_cast<float *>(p);
-    uint16_t *xs16 = reinterpret_cast<uint16_t *>(p);
-    p += (kMath == kMathF32) ? sizeof(float) * kTokGroup * K : sizeof(uint16_t) * kTokGroup * K;
-    float *xinv = reinterpret_cast<float *>(p);
-    if (kMath == kMathF16) p += sizeof(float) * kTokGroup * (K / 32);
-    uint8_t *sc = p;
-    const int sc_bytes = KT * kRowsPerTask * 4;
-    p += 2 * (size_t)sc_bytes;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(p);
+#pragma unroll
+    for (int j = 0; j < kChunk; ++j) {
+        if (j >= n) break;
+        const int tw = tile0 + j;
+        const uint32_t s4 = sc[tw * rows_task];
+        const float2 s = f16x2_to_float2(e4m3x2_to_f16x2(h ? (s4 >> 16) : (s4 & 0xFFFFu)));
+        const uint4 cw = cs[j * 32];
+        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+        float p[NT][2];
+#pragma unroll
+        for (int t = 0; t < NT; ++t) p[t][0] = p[t][1] = 0.f;
+        // word q holds columns 8q .. 8q+7 of the lane's 32 (16-column block q / 2)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t wp[4];
+            e2m1x8_to_f16x2x4(words[q], wp);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                const uint4 xv = *(reinterpret_cast<const uint4 *>(xs + t * K + tw * kTileK) + q);
+                float &pp = p[t][q >> 1];
+                pp = fma2_f16_f32(wp[0], xv.x, pp);
+                pp = fma2_f16_f32(wp[1], xv.y, pp);
+                pp = fma2_f16_f32(wp[2], xv.z, pp);
+                pp = fma2_f16_f32(wp[3], xv.w, pp);
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            const float2 inv = *reinterpret_cast<const float2 *>(xis + t * (K / 16) + tw * (kTileK / 16));
+            acc[t] = fmaf(p[t][0], s.x * inv.x, acc[t]);
+            acc[t] = fmaf(p[t][1], s.y * inv.y, acc[t]);
+        }
+    }
+}
+
+// All column chunks of one pass: wait for the lane's oldest copies, compute, and let
+// `refill` put the next chunk of the stream into the slot freed by the previous one.
+template <int NT, class Refill>
+__device__ __forceinline__ void pass_run(const uint4 *ring, int &slot_use, int KTW, const uint32_t *sc, int rows_task,
+                                         int h, const uint16_t *xs, const float *xis, int K, float (&acc)[kMaxNT],
+                                         Refill &refill)
+{
+    const int nch = (KTW + kChunk - 1) / kChunk;
+    for (int ch = 0; ch < nch; ++ch) {
+        cp_async_wait<kRing - 2>();
+        chunk_compute<NT>(ring + (size_t)slot_use * kChunk * 32, min(kChunk, KTW - ch * kChunk), ch * kChunk, sc,
+                          rows_task, h, xs, xis, K, acc);
+        refill();
+        slot_use = (slot_use + 1 == kRing) ? 0 : slot_use + 1;
+    }
+}
+
+// Bounded mbarrier wait shared by every role of the CTA: gives up (returning false)
+// once another thread has flagged an abort or after kWaitLimitNs, flagging it itself.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int32_t *abort_flag,
+                                              int32_t *err_word) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        for (int i = 0; i < 4; ++i)
+            if (mbar_try_wait_sleep(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(err_word, DEV_ERR_WAIT_TIMEOUT);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+// CTA = 8 compute warps + 1 control warp. The compute warps only stream codes and
+// do arithmetic: they never wait for one another. The control warp runs one pass
+// ahead issuing the tensor/bulk copies of scales and activation rows, and one pass
+// behind adding the compute warps' partial sums (in slice order) and storing the
+// outputs, so no warp holds a CTA-wide barrier per pass.
+//
+// Barriers (parity = use count / 2 mod 2, every barrier alternating between 2 buffers):
+//   sfull[b]  scales of task #i landed (b = i & 1; expect-tx by the control warp)
+//   xfull[b]  activation rows of pass #p landed (b = p & 1)
+//   full[b]   the 8 compute warps wrote their partial sums of pass #p (count 8)
+//   rfree[b]  the control warp consumed the partial sums of pass #p (count 1)
+// A buffer of scales / activations is refilled only after the control warp saw
+// full[] of the last pass that read it, which the compute warps signal after reading.
+template <Proj P>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid_constant__ CUtensorMap smap,
+                                                                    const GemvArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    const int K = a.K, KT = K / kTileK, KS = a.KS, RG = a.RG;
+    const int rows_task = 16 * RG, KTW = KT / KS;
+    const int RT = a.R / kTileRows, tpe = a.R / rows_task;
+    const int n_list = __ldg(a.list_size);
+    const int n_tasks = n_list * tpe;
+    if ((int)blockIdx.x >= n_tasks) return;
+
+    const SmemLayout lay(K, KS, RG);
+    auto sbuf = [&](int b) { return reinterpret_cast<uint32_t *>(base + lay.sc + b * lay.sc_sz); };
+    auto red = [&](int b) { return reinterpret_cast<float *>(base + lay.red + b * lay.red_sz); };
+    auto xbuf = [&](int b) { return reinterpret_cast<uint16_t *>(base + lay.x + b * lay.x_sz); };
+    auto xibuf = [&](int b) { return reinterpret_cast<float *>(base + lay.xi + b * lay.xi_sz); };
+    int32_t *tab = reinterpret_cast<int32_t *>(base + lay.tab);     // [3][n_list]: expert, first row, rows
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + lay.bar);
+    uint64_t *sfull = bars, *xfull = bars + 2, *full = bars + 4, *rfree = bars + 6;
+    volatile int32_t *abort_flag = reinterpret_cast<volatile int32_t *>(bars + 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int half = lane >> 4, lrow = lane & 15;
-    const int blocks_per_expert = a.R / kRowsPerTask;
-    const int n_tasks = __ldg(a.list_size) * blocks_per_expert;
-    if ((int)blockIdx.x >= n_tasks) return;
-    const int RT = a.R / kTileRows;
-
-    if (threadIdx.x == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); fence_mbar_init(); }
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sfull[i], 1);
+            mbar_init(&xfull[i], 1);
+            mbar_init(&full[i], kComputeWarps);
+            mbar_init(&rfree[i], 1);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    // the GEMV list with each expert's rows, read once (one dependent load per thread)
+    for (int i = threadIdx.x; i < n_list; i += kThreads) {
+        const int e = __ldg(a.expert_list + i);
+        const int rb = __ldg(a.offsets + e);
+        tab[i] = e;
+        tab[n_list + i] = rb;
+        tab[2 * n_list + i] = __ldg(a.offsets + e + 1) - rb;
+    }
     __syncthreads();
 
-    // the scales of a task (64 rows x all column tiles) are one contiguous span: one bulk copy
-    auto issue_scales = [&](int task, int buf) {
-        const int e = __ldg(a.expert_list + task / blocks_per_expert);
-        const int blk = task % blocks_per_expert;
-        const uint8_t *st = a.scales + scale_offset((size_t)e * RT + (blk >> 1), KT, blk & 1, 0);
-        mbar_arrive_expect_tx(&bar[buf], (uint32_t)sc_bytes);
-        bulk_g2s(sc + (size_t)buf * sc_bytes, st, (uint32_t)sc_bytes, &bar[buf]);
+    auto task_expert = [&](int task) { return tab[task / tpe]; };
+    auto task_rows = [&](int task, int &r_begin) {
+        r_begin = tab[n_list + task / tpe];
+        return tab[2 * n_list + task / tpe];
     };
-    if (threadIdx.x == 0) issue_scales(blockIdx.x, 0);
-    uint32_t phase0 = 0u, phase1 = 0u;
-    int staged_e = -1, staged_g0 = -1;
+    // the pass after (task, t0) in this CTA's sequence; tasks without rows have no pass
+    auto next_pass = [&](int task, int t0, int m, int &ntask, int &nt0) {
+        if (t0 + kMaxNT < m) { ntask = task; nt0 = t0 + kMaxNT; return true; }
+        for (int tk = task + (int)gridDim.x; tk < n_tasks; tk += gridDim.x) {
+            int rb;
+            if (task_rows(tk, rb) > 0) { ntask = tk; nt0 = 0; return true; }
+        }
+        return false;
+    };
+    auto first_pass = [&](int &ftask) {
+        int rb, t0;
+        if (task_rows(blockIdx.x, rb) > 0) { ftask = blockIdx.x; return true; }
+        return next_pass(blockIdx.x, 0, 0, ftask, t0);
+    };
 
-    int it = 0;
-    for (int task = blockIdx.x; task < n_tasks; task += gridDim.x, ++it) {
-        const int buf = it & 1;
-        const int e = __ldg(a.expert_list + task / blocks_per_expert);
-        const int blk = task % blocks_per_expert;
-        const int rt = blk >> 1, sub = blk & 1;
-        const int row_in_tile = sub * kRowsPerTask + warp * 16 + lrow;
-        const uint8_t *codes0 = a.codes + ((size_t)e * RT + rt) * KT * kTileCodeBytes + half * 2048 + row_in_tile * 16;
-        const uint8_t *scl = sc + (size_t)buf * sc_bytes + (warp * 16 + lrow) * 4 + half * 2;
-        const int r_begin = __ldg(a.offsets + e), m = __ldg(a.offsets + e + 1) - r_begin;
-
-        __syncthreads();   // the previous task is done with x and with the other scale buffer
-        if (threadIdx.x == 0 && task + (int)gridDim.x < n_tasks) issue_scales(task + gridDim.x, buf ^ 1);
-        bool scales_ready = false;
-
-        for (int g0 = 0; g0 < m; g0 += kTokGroup) {
-            const int nt = min(kTokGroup, m - g0);
-            // code loads of the first two batches go out before the activation staging
-            uint4 cA[kBatch], cB[kBatch];
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-                if (u < KT) cA[u] = ldg_stream_v4(codes0 + (size_t)u * kTileCodeBytes);
-                if (kBatch + u < KT) cB[u] = ldg_stream_v4(codes0 + (size_t)(kBatch + u) * kTileCodeBytes);
+    if (warp == kComputeWarps) {
+        // ------------------------------------------------------------ control warp
+        const uint32_t scale_tx = (uint32_t)(KT * rows_task * 4);
+        int last_s = -1, last_x = -1;                 // barriers of the latest copies issued
+        uint32_t last_s_par = 0, last_x_par = 0;
+        auto issue = [&](int task, int t0, int tn, int p) {
+            int r_begin;
+            const int m = task_rows(task, r_begin);
+            const int nt = min(kMaxNT, m - t0);
+            int row = 0;
+            if (lane < nt) {
+                const int r = r_begin + t0 + lane;
+                row = (P == Proj::GateUp) ? __ldg(a.perm + r) / a.top_k : r;
             }
-            if (e != staged_e || g0 != staged_g0) {
-                if (g0 > 0) __syncthreads();
-                stage_x<P>(a, r_begin + g0, nt, xs32, xs16, xinv);
-                staged_e = e;
-                staged_g0 = g0;
-                __syncthreads();
+            const int xb = p & 1;
+            if (lane == 0) {
+                if (t0 == 0) {
+                    const int sb = tn & 1, row0 = (task % tpe) * rows_task;
+                    mbar_arrive_expect_tx(&sfull[sb], scale_tx);
+                    tma_load_2d(sbuf(sb), &smap, row0 % kTileRows, (task_expert(task) * RT + row0 / kTileRows) * KT,
+                                &sfull[sb]);
+                    last_s = sb;
+                    last_s_par = (tn >> 1) & 1;
+                }
+                mbar_arrive_expect_tx(&xfull[xb], (uint32_t)nt * (uint32_t)(K * 2 + K / 4));
+                last_x = xb;
+                last_x_par = (p >> 1) & 1;
             }
-            if (!scales_ready) {
-                mbar_wait_bounded(&bar[buf], buf ? phase1 : phase0, a.err_word);
-                if (buf) phase1 ^= 1u; else phase0 ^= 1u;
-                scales_ready = true;
+            for (int t = 0; t < nt; ++t) {
+                const int rr = __shfl_sync(0xffffffffu, row, t);
+                if (lane == 0) {
+                    bulk_g2s(xbuf(xb) + (size_t)t * K, a.src + (size_t)rr * K, (uint32_t)K * 2, &xfull[xb]);
+                    bulk_g2s(xibuf(xb) + (size_t)t * (K / 16), a.src_inv + (size_t)rr * (K / 16), (uint32_t)K / 4,
+                             &xfull[xb]);
+                }
             }
-
-            float acc[kTokGroup];
-#pragma unroll
-            for (int t = 0; t < kTokGroup; ++t) acc[t] = 0.f;
-
-            auto compute = [&](const uint4 (&cv)[kBatch], int kt0) {
-#pragma unroll
-                for (int u = 0; u < kBatch; ++u) {
-                    const int kt = kt0 + u;
-                    if (kt >= KT) break;
-                    const uint32_t sbytes = *reinterpret_cast<const uint16_t *>(scl + kt * kRowsPerTask * 4);
-                    const float2 s = f16x2_to_float2(e4m3x2_to_f16x2(sbytes));
-                    const int col = kt * kTileK + half * 32;
-#pragma unroll
-                    for (int t = 0; t < kTokGroup; ++t) {
-                        if (t < nt) {
-                            float p0, p1;
-                            if (kMath == kMathF32) {
-                                dot_f32(cv[u], xs32 + t * K + col, p0, p1);
-                                acc[t] = fmaf(s.x, p0, acc[t]);
-                                acc[t] = fmaf(s.y, p1, acc[t]);
-                            } else {
-                                dot_f16(cv[u], xs16 + t * K + col, p0, p1);
-                                const float xi = xinv[t * (K / 32) + (col >> 5)];
-                                acc[t] = fmaf(s.x * xi, p0, acc[t]);
-                                acc[t] = fmaf(s.y * xi, p1, acc[t]);
+        };
+        int ftask;
+        if (first_pass(ftask)) {
+            issue(ftask, 0, 0, 0);
+            int p = 0, tn = 0;
+            for (int task = ftask; task < n_tasks; task += gridDim.x) {
+                int r_begin;
+                const int m = task_rows(task, r_begin);
+                if (m <= 0) continue;
+                const int e = task_expert(task), row0 = (task % tpe) * rows_task;
+                for (int t0 = 0; t0 < m; t0 += kMaxNT, ++p) {
+                    const int nt = min(kMaxNT, m - t0);
+                    int ntask, nt0;
+                    // the buffers of pass p+1 were last read in pass p-1, whose sums were consumed below
+                    if (next_pass(task, t0, m, ntask, nt0)) issue(ntask, nt0, ntask == task ? tn : tn + 1, p + 1);
+                    wait_or_abort(&full[p & 1], (p >> 1) & 1, abort_flag, a.err_word);
+                    const float *rb = red(p & 1);
+                    if (P == Proj::GateUp) {
+                        // rows_task is a multiple of 32: a round covers 32 rows (16 gate/up pairs) of one token
+                        const float g0 = __ldg(a.glob0 + e), g1 = __ldg(a.glob1 + e);
+                        for (int i0 = 0; i0 < rows_task * nt; i0 += 32) {
+                            const int i = i0 + lane, t = i / rows_task, rl = i % rows_task;
+                            float v = 0.f;
+                            for (int s = 0; s < KS; ++s) v += rb[((size_t)s * rows_task + rl) * kMaxNT + t];
+                            const int grow = row0 + rl;
+                            const bool up = (grow & 1) != 0;
+                            v *= up ? g1 : g0;
+                            const float other = __shfl_xor_sync(0xffffffffu, v, 1);
+                            const size_t r = (size_t)(r_begin + t0 + t);
+                            const int j = grow >> 1;
+                            uint32_t ab = 0;
+                            if (!up) {
+                                ab = float_to_bf16_bits_rn(silu_f32(v) * other);
+                                a.act_out[r * a.I + j] = (uint16_t)ab;
                             }
+                            // the round's 16 outputs form one block of aq and share its power of two
+                            const uint32_t emax = __reduce_max_sync(0xffffffffu, up ? 0u : ((ab >> 7) & 0xFFu));
+                            int sh = 14 - ((int)emax - 127);
+                            sh = max(-120, min(120, sh));
+                            if (!up)
+                                a.aq_out[r * a.I + j] = __half_as_ushort(
+                                    __float2half_rn(bf16_bits_to_float(ab) * __int_as_float((127 + sh) << 23)));
+                            if (lane == 0) a.aq_inv_out[r * (a.I / 16) + (j >> 4)] = __int_as_float((127 - sh) << 23);
+                        }
+                    } else {
+                        const float gs = __ldg(a.glob0 + e);
+                        for (int i = lane; i < rows_task * nt; i += 32) {
+                            const int t = i / rows_task, rl = i % rows_task;
+                            float v = 0.f;
+                            for (int s = 0; s < KS; ++s) v += rb[((size_t)s * rows_task + rl) * kMaxNT + t];
+                            a.y_out[(size_t)(r_begin + t0 + t) * a.R + row0 + rl] = v * gs;
                         }
                     }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&rfree[p & 1]);
                 }
-            };
-            for (int kt0 = 0; kt0 < KT; kt0 += 2 * kBatch) {
-                compute(cA, kt0);
-                if (kt0 + 2 * kBatch < KT) {
-#pragma unroll
-                    for (int u = 0; u < kBatch; ++u)
-                        if (kt0 + 2 * kBatch + u < KT)
-                            cA[u] = ldg_stream_v4(codes0 + (size_t)(kt0 + 2 * kBatch + u) * kTileCodeBytes);
-                }
-                if (kt0 + kBatch < KT) compute(cB, kt0 + kBatch);
-                if (kt0 + 3 * kBatch < KT) {
-#pragma unroll
-                    for (int u = 0; u < kBatch; ++u)
-                        if (kt0 + 3 * kBatch + u < KT)
-                            cB[u] = ldg_stream_v4(codes0 + (size_t)(kt0 + 3 * kBatch + u) * kTileCodeBytes);
-                }
-            }
-#pragma unroll
-            for (int t = 0; t < kTokGroup; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 16);
-            const int grow = rt * kTileRows + row_in_tile;   // row of the projection
-            if (P == Proj::GateUp) {
-                const bool is_up = (grow & 1) != 0;
-                const float gs = is_up ? __ldg(a.glob1 + e) : __ldg(a.glob0 + e);
-#pragma unroll
-                for (int t = 0; t < kTokGroup; ++t) {
-                    const float v = acc[t] * gs;
-                    const float other = __shfl_xor_sync(0xffffffffu, v, 1);
-                    if (t < nt && !is_up && half == 0) {
-                        const int r = r_begin + g0 + t;
-                        a.act_out[(size_t)r * a.I + (grow >> 1)] = float_to_bf16_bits_rn(silu_f32(v) * other);
-                    }
-                }
-            } else {
-                const float gs = __ldg(a.glob0 + e);
-#pragma unroll
-                for (int t = 0; t < kTokGroup; ++t) {
-                    if (t < nt && half == 0) {
-                        const int r = r_begin + g0 + t;
-                        a.y_out[(size_t)r * a.R + grow] = acc[t] * gs;
-                    }
-                }
+                ++tn;
             }
         }
-        if (!scales_ready) {   // no tokens (cannot happen for a listed expert): keep the barrier phase in step
-            mbar_wait_bounded(&bar[buf], buf ? phase1 : phase0, a.err_word);
-            if (buf) phase1 ^= 1u; else phase0 ^= 1u;
+        // after an abort, let the latest copies land before the CTA exits (bounded)
+        if (lane == 0 && *abort_flag) {
+            if (last_s >= 0) mbar_wait_bounded(&sfull[last_s], last_s_par, a.err_word);
+            if (last_x >= 0) mbar_wait_bounded(&xfull[last_x], last_x_par, a.err_word);
         }
+        return;
     }
-}
 
-size_t gemv_smem_bytes(int K) {
-    size_t b = (kMath == kMathF32) ? sizeof(float) * kTokGroup * (size_t)K : sizeof(uint16_t) * kTokGroup * (size_t)K;
-    if (kMath == kMathF16) b += sizeof(float) * kTokGroup * (size_t)(K / 32);
-    b += 2 * (size_t)(K / kTileK) * kRowsPerTask * 4;   // double-buffered scales
-    return b + 2 * sizeof(uint64_t);
+    // ---------------------------------------------------------------- compute warps
+    const int ks = warp % KS, rgl = warp / KS;
+    const int h = lane >> 4;
+    const int lrow = rgl * 16 + (lane & 15);              // row of the lane inside the task
+    const int col0 = ks * KTW * kTileK + h * 32;          // first column of the lane's slice and half
+    auto lane_codes = [&](int task) -> const uint8_t * {
+        const int row0 = (task % tpe) * rows_task;
+        return a.codes + ((size_t)(task_expert(task) * RT + row0 / kTileRows) * KT + (size_t)ks * KTW) *
+                   kTileCodeBytes + h * 2048 + (row0 % kTileRows + lrow) * 16;
+    };
+    // The warp's code stream: the (task, pass, chunk) sequence it consumes, kRing - 1
+    // chunks ahead. Each lane copies and later reads only its own 16-byte pieces, so a
+    // lane's cp.async.wait_group is all the synchronisation the ring needs.
+    const uint4 *ring = reinterpret_cast<const uint4 *>(base + lay.ring) + (size_t)warp * kRing * kChunk * 32 + lane;
+    const int nch = (KTW + kChunk - 1) / kChunk;
+    int ptask = -1, pt0 = 0, pch = 0, slot_fill = 0;
+    {
+        int ft;
+        if (first_pass(ft)) ptask = ft;
+    }
+    auto refill = [&]() {
+        if (ptask >= 0) {
+            const uint8_t *g = lane_codes(ptask) + (size_t)pch * kChunk * kTileCodeBytes;
+            const int n = min(kChunk, KTW - pch * kChunk);
+            uint4 *d = const_cast<uint4 *>(ring) + (size_t)slot_fill * kChunk * 32;
+#pragma unroll
+            for (int j = 0; j < kChunk; ++j)
+                if (j < n) cp_async16(d + j * 32, g + (size_t)j * kTileCodeBytes);
+            if (++pch == nch) {
+                pch = 0;
+                int rb, ntask, nt0;
+                const int m = task_rows(ptask, rb);
+                if (next_pass(ptask, pt0, m, ntask, nt0)) { ptask = ntask; pt0 = nt0; }
+                else ptask = -1;
+            }
+        }
+        cp_async_commit();
+        slot_fill = (slot_fill + 1 == kRing) ? 0 : slot_fill + 1;
+    };
+    for (int i = 0; i < kRing - 1; ++i) refill();
+
+    int slot_use = 0;
+    int p = 0, tn = 0;
+    for (int task = blockIdx.x; task < n_tasks; task += gridDim.x) {
+        int r_begin;
+        const int m = task_rows(task, r_begin);
+        if (m <= 0) continue;
+        const int sb = tn & 1;
+        const uint32_t *sc = sbuf(sb) + (size_t)(ks * KTW) * rows_task + lrow;
+        wait_or_abort(&sfull[sb], (tn >> 1) & 1, abort_flag, a.err_word);
+        for (int t0 = 0; t0 < m; t0 += kMaxNT, ++p) {
+            const int nt = min(kMaxNT, m - t0);
+            const int xb = p & 1;
+            wait_or_abort(&xfull[xb], (p >> 1) & 1, abort_flag, a.err_word);
+            const uint16_t *xs = xbuf(xb) + col0;
+            const float *xis = xibuf(xb) + col0 / 16;
+            float acc[kMaxNT] = {};
+            switch (nt) {
+            case 1: pass_run<1>(ring, slot_use, KTW, sc, rows_task, h, xs, xis, K, acc, refill); break;
+            case 2: pass_run<2>(ring, slot_use, KTW, sc, rows_task, h, xs, xis, K, acc, refill); break;
+            case 3: pass_run<(kMaxNT > 2 ? 3 : 2)>(ring, slot_use, KTW, sc, rows_task, h, xs, xis, K, acc, refill); break;
+            default: pass_run<kMaxNT>(ring, slot_use, KTW, sc, rows_task, h, xs, xis, K, acc, refill); break;
+            }
+#pragma unroll
+            for (int t = 0; t < kMaxNT; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 16);
+            // the control warp has consumed what pass p-2 left in this buffer
+            if (p >= 2) wait_or_abort(&rfree[xb], ((p - 2) >> 1) & 1, abort_flag, a.err_word);
+            float *rb = red(xb);
+            if (h == 0) {
+#pragma unroll
+                for (int t = 0; t < kMaxNT; ++t) rb[((size_t)ks * rows_task + lrow) * kMaxNT + t] = acc[t];
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full[xb]);
+        }
+        ++tn;
+    }
+    cp_async_wait<0>();   // copies of the empty tail groups: nothing may be in flight at exit
 }
 
 template <Proj P>
-int gemv_grid(int K, int num_sms) {
+int gemv_grid(int K, Geometry g, int num_sms) {
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_kernel<P>, kThreads, gemv_smem_bytes(K)) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gemv_kernel<P>, kThreads, gemv_smem_bytes(K, g)) !=
             cudaSuccess || per_sm < 1)
         per_sm = 1;
     return per_sm * num_sms;
 }
 
+struct GemvMaps {
+    CUtensorMap gu, down;
+    Geometry g_gu, g_down;
+};
+
 }  // namespace
 
 cudaError_t gemv_setup(Layer &L)
 {
-    const int H = L.desc.hidden, I = L.desc.intermediate;
+    const int H = L.desc.hidden, I = L.desc.intermediate, E = L.desc.num_experts;
+    GemvMaps *gm = new (std::nothrow) GemvMaps();
+    if (!gm) return cudaErrorMemoryAllocation;
+    gm->g_gu = geometry(true, H);
+    gm->g_down = geometry(false, I);
+    // scale slabs viewed as [E * RT * KT][128 rows] of u32; a task's box is 16*RG rows x all KT slabs
+    const uint64_t slabs_gu = (uint64_t)E * (2 * I / kTileRows) * (H / kTileK);
+    const uint64_t slabs_d = (uint64_t)E * (H / kTileRows) * (I / kTileK);
+    if (encode_tensor_map_2d(&gm->gu, CU_TENSOR_MAP_DATA_TYPE_UINT32, L.w.gu_scales, kTileRows, slabs_gu,
+                             kTileScaleBytes, 16 * gm->g_gu.RG, H / kTileK, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
+        encode_tensor_map_2d(&gm->down, CU_TENSOR_MAP_DATA_TYPE_UINT32, L.w.d_scales, kTileRows, slabs_d,
+                             kTileScaleBytes, 16 * gm->g_down.RG, I / kTileK, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS) {
+        delete gm;
+        return cudaErrorInvalidValue;
+    }
+    L.gemv_maps = gm;
     cudaError_t e = cudaFuncSetAttribute(gemv_kernel<Proj::GateUp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)gemv_smem_bytes(H));
+                                         (int)gemv_smem_bytes(H, gm->g_gu));
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(gemv_kernel<Proj::Down>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)gemv_smem_bytes(I));
+                                 (int)gemv_smem_bytes(I, gm->g_down));
     if (e != cudaSuccess) return e;
-    L.gemv_grid_gu = gemv_grid<Proj::GateUp>(H, L.num_sms);
-    L.gemv_grid_down = gemv_grid<Proj::Down>(I, L.num_sms);
+    L.gemv_grid_gu = gemv_grid<Proj::GateUp>(H, gm->g_gu, L.num_sms);
+    L.gemv_grid_down = gemv_grid<Proj::Down>(I, gm->g_down, L.num_sms);
     return cudaSuccess;
 }
 
-static GemvArgs gate_up_args(const Layer &L, const uint16_t *x) {
+void gemv_teardown(Layer &L)
+{
+    delete static_cast<GemvMaps *>(L.gemv_maps);
+    L.gemv_maps = nullptr;
+}
+
+static GemvArgs common_args(const Layer &L) {
     GemvArgs g{};
-    g.codes = L.w.gu_codes; g.scales = L.w.gu_scales;
-    g.glob0 = L.w.gate_global; g.glob1 = L.w.up_global;
-    g.R = 2 * L.desc.intermediate; g.K = L.desc.hidden;
     g.expert_list = L.ws.gemv_list; g.list_size = L.ws.list_sizes;
     g.offsets = L.ws.offsets; g.perm = L.ws.perm; g.top_k = L.desc.top_k;
-    g.src = x; g.act_out = L.ws.act; g.y_out = nullptr; g.I = L.desc.intermediate; g.err_word = L.ws.err_word;
+    g.I = L.desc.intermediate; g.err_word = L.ws.err_word;
     return g;
 }
 
 cudaError_t launch_gemv_gate_up(Layer &L, const uint16_t *x, cudaStream_t s, int *launches)
 {
+    (void)x;   // the routing kernels left x in block-scaled f16 form in ws.xq
     StageTimer timer(L, TFMOE_STAGE_GEMV_GATE_UP, s);
-    gemv_kernel<Proj::GateUp><<<L.gemv_grid_gu, kThreads, gemv_smem_bytes(L.desc.hidden), s>>>(gate_up_args(L, x));
+    const GemvMaps *gm = static_cast<const GemvMaps *>(L.gemv_maps);
+    GemvArgs g = common_args(L);
+    g.codes = L.w.gu_codes;
+    g.glob0 = L.w.gate_global; g.glob1 = L.w.up_global;
+    g.R = 2 * L.desc.intermediate; g.K = L.desc.hidden;
+    g.KS = gm->g_gu.KS; g.RG = gm->g_gu.RG;
+    g.src = L.ws.xq; g.src_inv = L.ws.xq_inv;
+    g.act_out = L.ws.act; g.aq_out = L.ws.aq; g.aq_inv_out = L.ws.aq_inv;
+    gemv_kernel<Proj::GateUp><<<L.gemv_grid_gu, kThreads, gemv_smem_bytes(g.K, gm->g_gu), s>>>(gm->gu, g);
     *launches += 1;
     return cudaGetLastError();
 }
@@ -381,12 +555,15 @@ cudaError_t launch_gemv_gate_up(Layer &L, const uint16_t *x, cudaStream_t s, int
 cudaError_t launch_gemv_down(Layer &L, cudaStream_t s, int *launches)
 {
     StageTimer timer(L, TFMOE_STAGE_GEMV_DOWN, s);
-    GemvArgs d = gate_up_args(L, nullptr);
-    d.codes = L.w.d_codes; d.scales = L.w.d_scales;
+    const GemvMaps *gm = static_cast<const GemvMaps *>(L.gemv_maps);
+    GemvArgs d = common_args(L);
+    d.codes = L.w.d_codes;
     d.glob0 = L.w.down_global; d.glob1 = nullptr;
     d.R = L.desc.hidden; d.K = L.desc.intermediate;
-    d.src = L.ws.act; d.act_out = nullptr; d.y_out = L.ws.y;
-    gemv_kernel<Proj::Down><<<L.gemv_grid_down, kThreads, gemv_smem_bytes(L.desc.intermediate), s>>>(d);
+    d.KS = gm->g_down.KS; d.RG = gm->g_down.RG;
+    d.src = L.ws.aq; d.src_inv = L.ws.aq_inv;
+    d.y_out = L.ws.y;
+    gemv_kernel<Proj::Down><<<L.gemv_grid_down, kThreads, gemv_smem_bytes(d.K, gm->g_down), s>>>(gm->down, d);
     *launches += 1;
     return cudaGetLastError();
 }

@@ -1,6 +1,7 @@
 // internal.h -- layer handle, workspace carving and kernel launchers of libtfmoe.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stddef.h>
@@ -12,19 +13,23 @@ namespace tfmoe {
 // Tile geometry of the repacked NVFP4 weights: 128 rows x 64 reduction
 // elements per tile. Codes: 4096 bytes per tile laid out as
 // [half of the 64 columns][128 rows][16 bytes], tiles ordered
-// [expert][row tile][column tile]. Scales: per (expert, row tile) a block of
-// KT * 512 bytes laid out [64-row half][column tile][64 rows][4 bytes], so the
-// scales of one 64-row half across all column tiles are contiguous.
+// [expert][row tile][column tile]. Scales: one 512-byte slab per tile, ordered
+// like the tiles, holding [128 rows][4 bytes] (the E4M3 scales of the row's
+// four 16-column blocks of the tile).
 constexpr int kTileRows = 128;
 constexpr int kTileK = 64;
 constexpr int kTileCodeBytes = kTileRows * kTileK / 2;   // 4096
 constexpr int kTileScaleBytes = kTileRows * kTileK / 16; // 512
 
-// Byte offset of the scales of 64-row half `sub` of row tile `rt`, column tile `kt`.
-__host__ __device__ __forceinline__ size_t scale_offset(size_t row_tile_index, int KT, int sub, int kt) {
-    return row_tile_index * (size_t)KT * kTileScaleBytes + (size_t)sub * KT * (kTileScaleBytes / 2) +
-           (size_t)kt * (kTileScaleBytes / 2);
+// Byte offset of the scale slab of row tile `row_tile_index` (= expert * RT + rt), column tile `kt`.
+__host__ __device__ __forceinline__ size_t scale_offset(size_t row_tile_index, int KT, int kt) {
+    return (row_tile_index * (size_t)KT + (size_t)kt) * kTileScaleBytes;
 }
+
+// Largest reduction length (hidden or intermediate) of this build: a GEMV task
+// stages the scales of all its column tiles with one tensor copy, whose box
+// extent is limited to 256 tiles.
+constexpr int kMaxReduction = 256 * kTileK;
 
 // Default crossover: experts routed to at most this many tokens use the GEMV regime.
 constexpr int kDefaultGemvMaxTokens = 8;
@@ -51,6 +56,10 @@ struct Workspace {
     uint16_t *x_perm = nullptr;     // [maxP][H] f16 activation rows (times 2^sh) in permuted order (MMA regime)
     float *row_inv = nullptr;       // [maxP] 2^-sh of each x_perm row
     uint16_t *act = nullptr;        // [maxP][I] bf16
+    uint16_t *xq = nullptr;         // [maxT][H] f16: x times a power of two per 16 elements (GEMV regime)
+    float *xq_inv = nullptr;        // [maxT][H/16] the inverse powers of two
+    uint16_t *aq = nullptr;         // [maxP][I] f16: act times a power of two per 16 elements (GEMV regime)
+    float *aq_inv = nullptr;        // [maxP][I/16]
     float *y = nullptr;             // [maxP][H]
     uint16_t *x_stage = nullptr;    // [maxT][H] bf16, for forward_host
     uint16_t *out_stage = nullptr;  // [maxT][H] bf16, for forward_host
@@ -84,6 +93,7 @@ struct Layer {
     int32_t last_T = -1;            // T of the last successful forward (stage replays need it)
     bool last_use_mma = false, last_use_gemv = false;
     int gemv_grid_gu = 0, gemv_grid_down = 0;
+    void *gemv_maps = nullptr;      // tensor maps of the GEMV regime's scale slabs
     void *mma_maps = nullptr;       // tensor maps of the MMA regime's token operands
     // per-stage profiling (tfmoe_profile_enable)
     bool profiling = false;
@@ -116,11 +126,18 @@ cudaError_t launch_gemv_down(Layer &L, cudaStream_t s, int *launches);
 cudaError_t launch_combine(Layer &L, int T, uint16_t *out, cudaStream_t s, int *launches);
 cudaError_t launch_repack(const Layer &L, const tfmoe_weights &src, cudaStream_t s);
 cudaError_t gemv_setup(Layer &L);
+void gemv_teardown(Layer &L);
 cudaError_t mma_setup(Layer &L);
 void mma_teardown(Layer &L);
 cudaError_t launch_gather(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches);
 cudaError_t launch_mma_gate_up(Layer &L, cudaStream_t s, int *launches);
 cudaError_t launch_mma_down(Layer &L, cudaStream_t s, int *launches);
+
+// cuTensorMapEncodeTiled for a 2-D tensor (dim0 contiguous), resolved through the
+// runtime's driver entry point so the library does not link the driver library.
+CUresult encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType type, void *base, uint64_t dim0,
+                              uint64_t dim1, uint64_t row_stride_bytes, uint32_t box0, uint32_t box1,
+                              CUtensorMapSwizzle swizzle);
 
 // Sets the thread-local message returned by tfmoe_last_error() and returns st.
 tfmoe_status record_error(tfmoe_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));

@@ -22,7 +22,7 @@
 //   warp 0       producer of the token tiles (TMA, 128-byte swizzle, box 64 x N)
 //                into a 5-stage ring that the MMA commit frees
 //   warp 2       producer of the 4 KB code tiles + 2 x 256 B scales (bulk copies)
-//                into a 12-stage ring that the decoders free once they have read it
+//                into a 16-stage ring that the decoders free once they have read it
 //   warp 1       allocates tensor memory; lane 0 issues the MMAs and commits. Each
 //                tcgen05.mma costs the issuing thread ~100 cycles whatever N is, so
 //                tiles are as wide as a double-buffered accumulator allows (N = 176,
@@ -112,8 +112,8 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, Mm
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
-        for (int i = 0; i < 128; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+        for (int i = 0; i < 4; ++i)
+            if (mbar_try_wait_sleep(bar, parity)) return true;
         if (*reinterpret_cast<volatile int32_t *>(&sm.abort_flag)) return false;
         if (global_timer_ns() - t0 > kWaitLimitNs) {
             atomicOr(err, DEV_ERR_WAIT_TIMEOUT);
@@ -148,12 +148,6 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
                  ::"r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-        ::"r"(smem_u32(dst)), "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar)) : "memory");
-}
-
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
@@ -174,17 +168,15 @@ __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// Two E2M1 codes (one byte) times the block scale (f16 pair, both halves equal) -> f16x2.
-__device__ __forceinline__ uint32_t dequant_pair_f16(uint32_t byte, __half2 scale2) {
-    const uint32_t h = e2m1x2_to_f16x2(byte);
+// Two decoded E2M1 values (f16x2) times the block scale (f16 pair, both halves equal) -> f16x2.
+__device__ __forceinline__ uint32_t scale_pair_f16(uint32_t h, __half2 scale2) {
     const __half2 v = __hmul2(*reinterpret_cast<const __half2 *>(&h), scale2);
     return *reinterpret_cast<const uint32_t *>(&v);
 }
 
-// Two E2M1 codes (one byte) times the block scale (f16 pair, both halves equal) -> bf16x2.
-// Products are exact in f16 (<= 6 significant bits, magnitudes 2^-10 .. 2688) and in bf16.
-__device__ __forceinline__ uint32_t dequant_pair_bf16(uint32_t byte, __half2 scale2) {
-    const uint32_t h = e2m1x2_to_f16x2(byte);
+// Two decoded E2M1 values (f16x2) times the block scale -> bf16x2. Products are exact
+// in f16 (<= 6 significant bits, magnitudes 2^-10 .. 2688) and in bf16.
+__device__ __forceinline__ uint32_t scale_pair_bf16(uint32_t h, __half2 scale2) {
     const __half2 v = __hmul2(*reinterpret_cast<const __half2 *>(&h), scale2);
     const float2 f = __half22float2(v);
     const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
@@ -265,10 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
                         if (!STAT_WAIT(1, wait_or_abort(&sm.cempty[s], ph ^ 1u, sm, a.err_word))) break;
                         mbar_arrive_expect_tx(&sm.cfull[s], kTileCodeBytes + kTileScaleBytes);
                         bulk_g2s(sm.codes[s], a.codes + (rti * KT + kt) * kTileCodeBytes, kTileCodeBytes, &sm.cfull[s]);
-                        bulk_g2s(sm.scales[s], a.scales + scale_offset(rti, KT, 0, kt), kTileScaleBytes / 2,
-                                 &sm.cfull[s]);
-                        bulk_g2s(sm.scales[s] + kTileScaleBytes / 2, a.scales + scale_offset(rti, KT, 1, kt),
-                                 kTileScaleBytes / 2, &sm.cfull[s]);
+                        bulk_g2s(sm.scales[s], a.scales + scale_offset(rti, KT, kt), kTileScaleBytes, &sm.cfull[s]);
                     }
                     issued = g + 1;
                 }
@@ -278,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
                 for (uint32_t j = (issued > (uint32_t)nst ? issued - nst : 0); j < issued; ++j) {
                     uint64_t *bar = tokens ? &sm.full[j % nst] : &sm.cfull[j % nst];
                     const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(bar, (j / nst) & 1u) && global_timer_ns() - t0 < kWaitLimitNs / 4) {
+                    while (!mbar_try_wait_sleep(bar, (j / nst) & 1u) && global_timer_ns() - t0 < kWaitLimitNs / 4) {
                     }
                 }
             }
@@ -358,13 +347,14 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
                 for (int hh = 0; hh < 2; ++hh) {      // columns 0..31, then 32..63
                     uint32_t r[16];
 #pragma unroll
-                    for (int w4 = 0; w4 < 4; ++w4)    // word holds elements 8*w4 .. 8*w4 + 7 of the half
+                    for (int w4 = 0; w4 < 4; ++w4) {  // word holds elements 8*w4 .. 8*w4 + 7 of the half
+                        uint32_t h4[4];
+                        e2m1x8_to_f16x2x4(words[4 * hh + w4], h4);
+                        const __half2 sc = sb[2 * hh + (w4 >> 1)];
 #pragma unroll
-                        for (int b = 0; b < 4; ++b) {
-                            const uint32_t byte = (words[4 * hh + w4] >> (8 * b)) & 0xFFu;
-                            const __half2 sc = sb[2 * hh + (w4 >> 1)];
-                            r[4 * w4 + b] = (kType == 0u) ? dequant_pair_f16(byte, sc) : dequant_pair_bf16(byte, sc);
-                        }
+                        for (int b = 0; b < 4; ++b)
+                            r[4 * w4 + b] = (kType == 0u) ? scale_pair_f16(h4[b], sc) : scale_pair_bf16(h4[b], sc);
+                    }
                     tmem_st16(tmem + lane_base + kACol + (uint32_t)s * 32u + (uint32_t)hh * 16u, r);
                 }
                 tc_wait_st();
@@ -505,35 +495,11 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint16_t *__restrict_
 
 size_t mma_smem_bytes() { return sizeof(MmaSmem) + 1024; }
 
-// cuTensorMapEncodeTiled, looked up through the runtime so the library does not
-// link the driver library directly (it loads on machines without a GPU driver).
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_tiled_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
 CUresult make_token_maps(TokenMaps &m, void *base, int cols, int rows, CUtensorMapDataType type) {
-    EncodeTiledFn encode = encode_tiled_fn();
-    if (!encode) return CUDA_ERROR_NOT_FOUND;
     for (int i = 0; i < kNumBoxes; ++i) {
-        const cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-        const cuuint64_t gstride[1] = {(cuuint64_t)cols * 2};
-        const cuuint32_t box[2] = {(cuuint32_t)kTileK, (cuuint32_t)(i < kNumBoxes - 1 ? (16 << i) : kMaxN)};
-        const cuuint32_t estride[2] = {1, 1};
-        CUresult r = encode(&m.box[i], type, 2, base, gdim, gstride, box,
-                                            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        const uint32_t box_rows = (uint32_t)(i < kNumBoxes - 1 ? (16 << i) : kMaxN);
+        CUresult r = encode_tensor_map_2d(&m.box[i], type, base, (uint64_t)cols, (uint64_t)rows, (uint64_t)cols * 2,
+                                          (uint32_t)kTileK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
         if (r != CUDA_SUCCESS) return r;
     }
     return CUDA_SUCCESS;

@@ -4,9 +4,8 @@
 //   codes  : 4096 bytes = [half h of the 64 columns][row r of 128][16 bytes]
 //            byte b of (h, r) holds columns 32h + 2b (low nibble) and 32h + 2b + 1
 // Tiles are stored [expert][row tile][column tile], so a row tile's columns
-// are contiguous. Scales of (expert, row tile) form one block of KT * 512
-// bytes: [64-row half][column tile][64 rows][4 scale bytes of the 4 16-column
-// blocks], so one half's scales for every column tile are contiguous.
+// are contiguous. The scales of a tile form one 512-byte slab stored in the
+// same order: [128 rows][4 scale bytes of the row's 4 16-column blocks].
 // Gate and up share one matrix of 2I rows: row 2j is gate row j and row 2j+1
 // is up row j.
 #include "common.cuh"
@@ -48,7 +47,7 @@ __global__ void repack_kernel(const uint8_t *__restrict__ codes_a, const uint8_t
         *reinterpret_cast<uint4 *>(ct) = *reinterpret_cast<const uint4 *>(crow);
         *reinterpret_cast<uint4 *>(ct + 2048) = *reinterpret_cast<const uint4 *>(crow + 16);
         const size_t rti = (size_t)e * RT + r / kTileRows;
-        *reinterpret_cast<uint32_t *>(out_scales + scale_offset(rti, KT, (r % kTileRows) / 64, kt) + (r % 64) * 4) =
+        *reinterpret_cast<uint32_t *>(out_scales + scale_offset(rti, KT, kt) + (r % kTileRows) * 4) =
             *reinterpret_cast<const uint32_t *>(srow);
     }
 }

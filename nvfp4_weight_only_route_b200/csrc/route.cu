@@ -191,9 +191,23 @@ __device__ __forceinline__ void topk_warp(const float *row, int E, int k, int32_
     }
 }
 
+// x [T][H] -> xq (f16 times a power of two per 16 elements) and xq_inv, for the
+// GEMV regime; blocks spread over all threads of the grid.
+__device__ __forceinline__ void convert_x_blocks(const uint16_t *__restrict__ x, int T, int H, uint16_t *xq,
+                                                 float *xq_inv) {
+    const int per_row = H / 16, n = T * per_row;
+    for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < n; b += gridDim.x * blockDim.x) {
+        const size_t off = (size_t)(b / per_row) * H + (size_t)(b % per_row) * 16;
+        xq_inv[b] = block16_bf16_to_f16(x + off, xq + off);
+    }
+}
+
+// One warp per token; with xq given, the grid also writes the GEMV regime's x operand.
 __global__ void __launch_bounds__(256) topk_kernel(
-    const float *__restrict__ logits, int32_t *__restrict__ ids, float *__restrict__ wts, int T, int E, int k)
+    const float *__restrict__ logits, int32_t *__restrict__ ids, float *__restrict__ wts, int T, int E, int k,
+    const uint16_t *__restrict__ x, int H, uint16_t *xq, float *xq_inv)
 {
+    if (xq) convert_x_blocks(x, T, H, xq, xq_inv);
     const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (t >= T) return;
     topk_warp(logits + (size_t)t * E, E, k, ids + (size_t)t * k, wts + (size_t)t * k);
@@ -370,7 +384,7 @@ constexpr int kFusedThreads = 256;
 __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(
     const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, const float *__restrict__ bias,
     float *__restrict__ logits, int32_t *__restrict__ ids, float *__restrict__ wts, int T, int H, int k,
-    PlanArgs pa, int32_t *counter)
+    PlanArgs pa, int32_t *counter, uint16_t *xq, float *xq_inv)
 {
     extern __shared__ int32_t sm[];
     __shared__ double red[kFusedThreads / 32][kFusedMaxT];
@@ -421,6 +435,7 @@ __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(
         if (pa.debug && !isfinite(l)) atomicOr(pa.err_word, DEV_ERR_NONFINITE);
         logits[(size_t)threadIdx.x * E + e] = l;
     }
+    if (xq) convert_x_blocks(x, T, H, xq, xq_inv);
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) is_last = (atomicAdd(counter, 1) == (int)gridDim.x - 1);
@@ -456,12 +471,14 @@ cudaError_t launch_router(Layer &L, const uint16_t *x, int T, cudaStream_t s, in
     const int H = L.desc.hidden, E = L.desc.num_experts, k = L.desc.top_k;
     const int debug = (L.desc.flags & TFMOE_FLAG_DEBUG_CHECKS) ? 1 : 0;
     const float *bias = L.desc.has_router_bias ? L.w.router_bias : nullptr;
+    const bool gemv = !(L.desc.flags & TFMOE_FLAG_FORCE_MMA);   // the GEMV regime may run: write its x operand
     if (route_fused_applies(L, T)) {
         // router, top-k and plan in one launch (the permute launcher then does nothing)
         StageTimer timer(L, TFMOE_STAGE_ROUTER, s);
         const size_t smem = sizeof(int32_t) * plan_smem_ints(kFusedThreads / 32, E);
         route_fused_kernel<<<E, kFusedThreads, smem, s>>>(x, L.w.router_w, bias, L.ws.logits, L.ws.ids,
-                                                          L.ws.topk_w, T, H, k, plan_args(L), L.ws.route_counter);
+                                                          L.ws.topk_w, T, H, k, plan_args(L), L.ws.route_counter,
+                                                          gemv ? L.ws.xq : nullptr, L.ws.xq_inv);
         *launches += 1;
         return cudaGetLastError();
     }
@@ -473,7 +490,8 @@ cudaError_t launch_router(Layer &L, const uint16_t *x, int T, cudaStream_t s, in
     }
     {
         StageTimer timer(L, TFMOE_STAGE_TOPK, s);
-        topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(L.ws.logits, L.ws.ids, L.ws.topk_w, T, E, k);
+        topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(L.ws.logits, L.ws.ids, L.ws.topk_w, T, E, k, x, H,
+                                                  gemv ? L.ws.xq : nullptr, L.ws.xq_inv);
     }
     *launches += 2;
     return cudaGetLastError();
@@ -565,7 +583,7 @@ extern "C" tfmoe_status tfmoe_route_noalloc(const uint16_t *x, int32_t T, int32_
         dim3 grid((T + RT_T - 1) / RT_T, (E + RT_E - 1) / RT_E);
         router_tiled_kernel<<<grid, 256, 0, s>>>(x, router_w, router_bias, logits, T, H, E, nullptr, 0);
     }
-    topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(logits, ids_out, weights_out, T, E, k);
+    topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(logits, ids_out, weights_out, T, E, k, x, H, nullptr, nullptr);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return record_error(TFMOE_ERR_CUDA, "tfmoe_route_noalloc: launch: %s", cudaGetErrorString(e));
