@@ -83,7 +83,8 @@ typedef struct {
     uint32_t flags;            /* TFMOE_FLAG_* */
     int32_t gemv_max_tokens;   /* experts routed to <= this many tokens use the CUDA-core GEMV
                                   regime, the others the tcgen05 tensor-core regime;
-                                  <= 0 selects the built-in crossover (8) */
+                                  <= 0 selects the built-in crossover: every expert in the
+                                  GEMV regime while T <= 16, else 2 tokens */
 } tfmoe_layer_desc;
 
 /*

@@ -1,6 +1,7 @@
 // api.cu -- the C ABI of libtfmoe (declared in include/tfmoe.h): argument
 // validation, device memory ownership, and the stream-ordered launch chain
 // router -> top-k -> permute -> expert projections -> combine.
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -62,6 +63,8 @@ void carve_workspace(Layer &L, uint8_t *base, size_t *total) {
     Workspace &w = L.ws;
     Carver c;
     c.take(&w.logits, T * E, base);
+    L.router_partial_cap = std::min(kRouterPartialMax, (size_t)kRouterMaxSlices * T * E);
+    c.take(&w.router_partial, L.router_partial_cap, base);
     c.take(&w.ids, P, base);
     c.take(&w.topk_w, P, base);
     c.take(&w.counts, E, base);
@@ -169,7 +172,7 @@ tfmoe_status tfmoe_create(const tfmoe_layer_desc *desc, tfmoe_layer **out)
     if (!h) return fail(TFMOE_ERR_OOM, "tfmoe_create: host allocation failed");
     Layer &L = h->impl;
     L.desc = d;
-    L.gemv_max_tokens = d.gemv_max_tokens > 0 ? d.gemv_max_tokens : kDefaultGemvMaxTokens;
+    L.gemv_max_tokens = d.gemv_max_tokens;
     cudaError_t e = cudaGetDevice(&L.device);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&L.num_sms, cudaDevAttrMultiProcessorCount, L.device);
     if (e != cudaSuccess) { delete h; return cuda_fail(e, "tfmoe_create: device query"); }
@@ -262,7 +265,7 @@ tfmoe_status tfmoe_forward(tfmoe_layer *layer, const uint16_t *x, int32_t T, uin
     // An expert holds at most T tokens, so with T <= the GEMV threshold no expert can be
     // in the MMA regime and its launches are skipped (likewise under the FORCE flags).
     const bool use_mma = !(L.desc.flags & TFMOE_FLAG_FORCE_GEMV) &&
-                         ((L.desc.flags & TFMOE_FLAG_FORCE_MMA) || T > L.gemv_max_tokens);
+                         ((L.desc.flags & TFMOE_FLAG_FORCE_MMA) || T > gemv_threshold(L, T));
     const bool use_gemv = !(L.desc.flags & TFMOE_FLAG_FORCE_MMA);
     cudaError_t e = launch_router(L, x, T, s, &n);
     if (e == cudaSuccess) e = launch_permute(L, T, s, &n);

@@ -31,8 +31,17 @@ __host__ __device__ __forceinline__ size_t scale_offset(size_t row_tile_index, i
 // extent is limited to 256 tiles.
 constexpr int kMaxReduction = 256 * kTileK;
 
-// Default crossover: experts routed to at most this many tokens use the GEMV regime.
-constexpr int kDefaultGemvMaxTokens = 8;
+// Built-in crossover between the regimes (measured on B200): for batches of at most
+// kSmallBatchTokens tokens every expert stays in the GEMV regime (the tensor-core
+// regime's extra launches cost more than they save); above that, experts routed to at
+// most kDefaultGemvMaxTokens tokens use the GEMV regime.
+constexpr int kSmallBatchTokens = 16;
+constexpr int kDefaultGemvMaxTokens = 2;
+
+// Router for T > 16: at most this many hidden-dimension slices, and at most
+// kRouterPartialMax fp64 partial logits held at once.
+constexpr int kRouterMaxSlices = 16;
+constexpr size_t kRouterPartialMax = size_t(1) << 22;
 
 // Tokens per tensor-core tile (the MMA N dimension).
 constexpr int kMmaTileTokens = 176;
@@ -40,6 +49,7 @@ __host__ __device__ constexpr size_t max_mma_entries(size_t P, size_t E) { retur
 
 struct Workspace {
     float *logits = nullptr;        // [maxT][E]
+    double *router_partial = nullptr; // [router_partial_cap] fp64 partial logits of hidden-dimension slices
     int32_t *ids = nullptr;         // [maxT][k]
     float *topk_w = nullptr;        // [maxT][k]
     int32_t *counts = nullptr;      // [E]
@@ -81,7 +91,7 @@ struct Layer {
     tfmoe_layer_desc desc{};
     int device = 0;
     int num_sms = 0;
-    int gemv_max_tokens = kDefaultGemvMaxTokens;
+    int gemv_max_tokens = 0;        // the descriptor's value; <= 0 = the built-in crossover
     bool loaded = false;
     void *ws_block = nullptr;
     size_t ws_bytes = 0;
@@ -93,6 +103,7 @@ struct Layer {
     int32_t last_T = -1;            // T of the last successful forward (stage replays need it)
     bool last_use_mma = false, last_use_gemv = false;
     int gemv_grid_gu = 0, gemv_grid_down = 0;
+    size_t router_partial_cap = 0;  // doubles in ws.router_partial
     void *gemv_maps = nullptr;      // tensor maps of the GEMV regime's scale slabs
     void *mma_maps = nullptr;       // tensor maps of the MMA regime's token operands
     // per-stage profiling (tfmoe_profile_enable)
@@ -115,6 +126,12 @@ struct StageTimer {
         if (L.profiling) { cudaEventRecord(L.prof_ev[stage][1], s); L.prof_used[stage] = true; }
     }
 };
+
+// Per-expert token count up to which the GEMV regime is used, for a batch of T tokens.
+inline int gemv_threshold(const Layer &L, int T) {
+    if (L.gemv_max_tokens > 0) return L.gemv_max_tokens;
+    return T <= kSmallBatchTokens ? T : kDefaultGemvMaxTokens;
+}
 
 // Launchers. Each returns cudaGetLastError() after its launches and adds
 // the number of kernels it enqueued to *launches.

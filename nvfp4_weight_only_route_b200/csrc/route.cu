@@ -12,6 +12,7 @@
 // then plus the fp32 bias: this makes the top-k ids bit-reproducible against
 // a float64 reference (issue #627, "Description": error stated against a
 // 64-bit reference).
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -142,6 +143,79 @@ __global__ void __launch_bounds__(256) router_tiled_kernel(
     }
 }
 
+// Layer path for T > 16: (16M tokens x 16M experts) tiles, M = 2 or 4, over a z-range of
+// the hidden dimension each. With one z-slice the CTA rounds its fp64 sums to fp32 and
+// adds the bias; with several it writes fp64 partial sums [z][T][E] that the top-k
+// kernel adds in z order. Small batches get small tiles and many slices, so the grid
+// still covers the GPU.
+template <int M>
+__global__ void __launch_bounds__(256) router_split_kernel(
+    const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, const float *__restrict__ bias,
+    float *__restrict__ logits, double *__restrict__ partial, int T, int H, int E, int k_len, int32_t *err_word,
+    int debug)
+{
+    constexpr int TT = 16 * M, TE = 16 * M, KC = 32;
+    __shared__ double xs[KC][TT + 1];
+    __shared__ double ws[KC][TE + 1];
+    const int t_base = blockIdx.x * TT, e_base = blockIdx.y * TE, k_begin = blockIdx.z * k_len;
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    double acc[M][M];
+#pragma unroll
+    for (int i = 0; i < M; ++i)
+#pragma unroll
+        for (int j = 0; j < M; ++j) acc[i][j] = 0.0;
+    for (int k0 = k_begin; k0 < k_begin + k_len; k0 += KC) {
+        // TT rows x 32 columns of x and of wr: 8 elements per item
+        for (int i = threadIdx.x; i < TT * KC / 8; i += 256) {
+            const int row = i / (KC / 8), col = (i % (KC / 8)) * 8;
+            const int t = t_base + row, e = e_base + row;
+            uint4 xv = make_uint4(0, 0, 0, 0), wv = make_uint4(0, 0, 0, 0);
+            if (t < T) xv = *reinterpret_cast<const uint4 *>(x + (size_t)t * H + k0 + col);
+            if (e < E) wv = *reinterpret_cast<const uint4 *>(wr + (size_t)e * H + k0 + col);
+            const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w}, wu[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                xs[col + 2 * j][row] = (double)bf16_bits_to_float(xu[j] & 0xFFFFu);
+                xs[col + 2 * j + 1][row] = (double)bf16_bits_to_float(xu[j] >> 16);
+                ws[col + 2 * j][row] = (double)bf16_bits_to_float(wu[j] & 0xFFFFu);
+                ws[col + 2 * j + 1][row] = (double)bf16_bits_to_float(wu[j] >> 16);
+            }
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int kk = 0; kk < KC; ++kk) {
+            double xv[M], wv[M];
+#pragma unroll
+            for (int i = 0; i < M; ++i) xv[i] = xs[kk][ty + 16 * i];
+#pragma unroll
+            for (int j = 0; j < M; ++j) wv[j] = ws[kk][tx + 16 * j];
+#pragma unroll
+            for (int i = 0; i < M; ++i)
+#pragma unroll
+                for (int j = 0; j < M; ++j) acc[i][j] = fma(xv[i], wv[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < M; ++i) {
+        const int t = t_base + ty + 16 * i;
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < M; ++j) {
+            const int e = e_base + tx + 16 * j;
+            if (e >= E) continue;
+            if (partial) {
+                partial[((size_t)blockIdx.z * T + t) * E + e] = acc[i][j];
+            } else {
+                float l = (float)acc[i][j];
+                if (bias) l = l + bias[e];
+                if (debug && !isfinite(l)) atomicOr(err_word, DEV_ERR_NONFINITE);
+                logits[(size_t)t * E + e] = l;
+            }
+        }
+    }
+}
+
 // One warp per token: k rounds of a warp arg-max over (logit desc, index asc),
 // then softmax over the selected logits (max-subtracted, fp32).
 constexpr int kMaxEPerLane = 8;   // E <= 256
@@ -203,13 +277,27 @@ __device__ __forceinline__ void convert_x_blocks(const uint16_t *__restrict__ x,
 }
 
 // One warp per token; with xq given, the grid also writes the GEMV regime's x operand.
+// With S > 1 fp64 partial sums [S][T][E], the warp first adds them in slice order,
+// rounds once to fp32, adds the bias and stores the token's logits.
 __global__ void __launch_bounds__(256) topk_kernel(
-    const float *__restrict__ logits, int32_t *__restrict__ ids, float *__restrict__ wts, int T, int E, int k,
-    const uint16_t *__restrict__ x, int H, uint16_t *xq, float *xq_inv)
+    float *__restrict__ logits, int32_t *__restrict__ ids, float *__restrict__ wts, int T, int E, int k,
+    const uint16_t *__restrict__ x, int H, uint16_t *xq, float *xq_inv, const double *__restrict__ partial, int S,
+    const float *__restrict__ bias, int32_t *err_word, int debug)
 {
     if (xq) convert_x_blocks(x, T, H, xq, xq_inv);
     const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (t >= T) return;
+    if (partial) {
+        for (int e = threadIdx.x & 31; e < E; e += 32) {
+            double v = 0.0;
+            for (int z = 0; z < S; ++z) v += partial[((size_t)z * T + t) * E + e];
+            float l = (float)v;
+            if (bias) l = l + bias[e];
+            if (debug && !isfinite(l)) atomicOr(err_word, DEV_ERR_NONFINITE);
+            logits[(size_t)t * E + e] = l;
+        }
+        __syncwarp();
+    }
     topk_warp(logits + (size_t)t * E, E, k, ids + (size_t)t * k, wts + (size_t)t * k);
 }
 
@@ -451,10 +539,10 @@ __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(
 
 }  // namespace
 
-static PlanArgs plan_args(const Layer &L) {
+static PlanArgs plan_args(const Layer &L, int T) {
     PlanArgs pa{};
     pa.E = L.desc.num_experts;
-    pa.gemv_max_tokens = L.gemv_max_tokens;
+    pa.gemv_max_tokens = gemv_threshold(L, T);
     pa.flags = L.desc.flags;
     pa.counts = L.ws.counts; pa.offsets = L.ws.offsets; pa.perm = L.ws.perm; pa.inv = L.ws.inv;
     pa.regime = L.ws.regime; pa.gemv_list = L.ws.gemv_list; pa.mma_list = L.ws.mma_list;
@@ -477,21 +565,35 @@ cudaError_t launch_router(Layer &L, const uint16_t *x, int T, cudaStream_t s, in
         StageTimer timer(L, TFMOE_STAGE_ROUTER, s);
         const size_t smem = sizeof(int32_t) * plan_smem_ints(kFusedThreads / 32, E);
         route_fused_kernel<<<E, kFusedThreads, smem, s>>>(x, L.w.router_w, bias, L.ws.logits, L.ws.ids,
-                                                          L.ws.topk_w, T, H, k, plan_args(L), L.ws.route_counter,
+                                                          L.ws.topk_w, T, H, k, plan_args(L, T), L.ws.route_counter,
                                                           gemv ? L.ws.xq : nullptr, L.ws.xq_inv);
         *launches += 1;
         return cudaGetLastError();
     }
+    // tile size and hidden-dimension slices: enough CTAs for two per SM where possible
+    const int M = (T >= 2048) ? 4 : 2, tile = 16 * M;
+    const int tiles = ((T + tile - 1) / tile) * ((E + tile - 1) / tile);
+    int S = 1;
+    if (tiles < 2 * L.num_sms) {
+        S = std::min(kRouterMaxSlices, (2 * L.num_sms + tiles - 1) / tiles);
+        while (S > 1 && ((H / 32) % S || (size_t)S * T * E > L.router_partial_cap)) --S;
+    }
+    double *partial = (S > 1) ? L.ws.router_partial : nullptr;
     {
         StageTimer timer(L, TFMOE_STAGE_ROUTER, s);
-        dim3 grid((T + RT_T - 1) / RT_T, (E + RT_E - 1) / RT_E);
-        router_tiled_kernel<<<grid, 256, 0, s>>>(x, L.w.router_w, bias, L.ws.logits, T, H, E,
-                                                  L.ws.err_word, debug);
+        dim3 grid((T + tile - 1) / tile, (E + tile - 1) / tile, S);
+        if (M == 4)
+            router_split_kernel<4><<<grid, 256, 0, s>>>(x, L.w.router_w, bias, L.ws.logits, partial, T, H, E, H / S,
+                                                        L.ws.err_word, debug);
+        else
+            router_split_kernel<2><<<grid, 256, 0, s>>>(x, L.w.router_w, bias, L.ws.logits, partial, T, H, E, H / S,
+                                                        L.ws.err_word, debug);
     }
     {
         StageTimer timer(L, TFMOE_STAGE_TOPK, s);
         topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(L.ws.logits, L.ws.ids, L.ws.topk_w, T, E, k, x, H,
-                                                  gemv ? L.ws.xq : nullptr, L.ws.xq_inv);
+                                                  gemv ? L.ws.xq : nullptr, L.ws.xq_inv, partial, S, bias,
+                                                  L.ws.err_word, debug);
     }
     *launches += 2;
     return cudaGetLastError();
@@ -503,7 +605,7 @@ cudaError_t launch_permute(Layer &L, int T, cudaStream_t s, int *launches)
     StageTimer timer(L, TFMOE_STAGE_PERMUTE, s);
     const int E = L.desc.num_experts, P = T * L.desc.top_k;
     const size_t smem = sizeof(int32_t) * plan_smem_ints(32, E);
-    permute_kernel<<<1, 1024, smem, s>>>(L.ws.ids, P, plan_args(L));
+    permute_kernel<<<1, 1024, smem, s>>>(L.ws.ids, P, plan_args(L, T));
     *launches += 1;
     return cudaGetLastError();
 }
@@ -583,7 +685,8 @@ extern "C" tfmoe_status tfmoe_route_noalloc(const uint16_t *x, int32_t T, int32_
         dim3 grid((T + RT_T - 1) / RT_T, (E + RT_E - 1) / RT_E);
         router_tiled_kernel<<<grid, 256, 0, s>>>(x, router_w, router_bias, logits, T, H, E, nullptr, 0);
     }
-    topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(logits, ids_out, weights_out, T, E, k, x, H, nullptr, nullptr);
+    topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(logits, ids_out, weights_out, T, E, k, x, H, nullptr, nullptr, nullptr,
+                                            1, nullptr, nullptr, 0);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return record_error(TFMOE_ERR_CUDA, "tfmoe_route_noalloc: launch: %s", cudaGetErrorString(e));
