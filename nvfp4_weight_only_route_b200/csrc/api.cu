@@ -267,6 +267,7 @@ tfmoe_status tfmoe_forward(tfmoe_layer *layer, const uint16_t *x, int32_t T, uin
     const bool use_mma = !(L.desc.flags & TFMOE_FLAG_FORCE_GEMV) &&
                          ((L.desc.flags & TFMOE_FLAG_FORCE_MMA) || T > gemv_threshold(L, T));
     const bool use_gemv = !(L.desc.flags & TFMOE_FLAG_FORCE_MMA);
+    L.mma_small = mma_use_small_tiles(L, T);
     cudaError_t e = launch_router(L, x, T, s, &n);
     if (e == cudaSuccess) e = launch_permute(L, T, s, &n);
     if (e == cudaSuccess && use_mma) e = launch_gather(L, x, T, s, &n);

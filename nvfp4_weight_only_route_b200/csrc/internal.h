@@ -43,9 +43,13 @@ constexpr int kDefaultGemvMaxTokens = 2;
 constexpr int kRouterMaxSlices = 16;
 constexpr size_t kRouterPartialMax = size_t(1) << 22;
 
-// Tokens per tensor-core tile (the MMA N dimension).
+// Tokens per tensor-core tile (the MMA N dimension): up to kMmaTileTokens with one CTA
+// per SM, or up to kMmaSmallTileTokens with two CTAs per SM when a batch averages at most
+// kMmaSmallMaxAvgTokens tokens per expert.
 constexpr int kMmaTileTokens = 176;
-__host__ __device__ constexpr size_t max_mma_entries(size_t P, size_t E) { return P / kMmaTileTokens + E + 1; }
+constexpr int kMmaSmallTileTokens = 64;
+constexpr int kMmaSmallMaxAvgTokens = 64;
+__host__ __device__ constexpr size_t max_mma_entries(size_t P, size_t E) { return P / kMmaSmallTileTokens + E + 1; }
 
 struct Workspace {
     float *logits = nullptr;        // [maxT][E]
@@ -102,6 +106,7 @@ struct Layer {
     int32_t last_launches = 0;
     int32_t last_T = -1;            // T of the last successful forward (stage replays need it)
     bool last_use_mma = false, last_use_gemv = false;
+    bool mma_small = false;         // the tensor-core regime of the current forward uses small tiles
     int gemv_grid_gu = 0, gemv_grid_down = 0;
     size_t router_partial_cap = 0;  // doubles in ws.router_partial
     void *gemv_maps = nullptr;      // tensor maps of the GEMV regime's scale slabs
@@ -145,6 +150,7 @@ cudaError_t launch_repack(const Layer &L, const tfmoe_weights &src, cudaStream_t
 cudaError_t gemv_setup(Layer &L);
 void gemv_teardown(Layer &L);
 cudaError_t mma_setup(Layer &L);
+bool mma_use_small_tiles(const Layer &L, int T);
 void mma_teardown(Layer &L);
 cudaError_t launch_gather(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches);
 cudaError_t launch_mma_gate_up(Layer &L, cudaStream_t s, int *launches);

@@ -48,34 +48,47 @@ namespace tfmoe {
 namespace {
 
 constexpr int kM = 128;
-constexpr int kMaxN = kMmaTileTokens;      // 176
-constexpr int kStages = 5;                 // token-tile ring and tensor-memory A ring
-constexpr int kCStages = 16;               // code/scale ring
-constexpr int kThreads = 640;
-constexpr int kDqWarp0 = 4;                // two dequant warpgroups: warps 4..11
-constexpr int kEpiWarp0 = 12;              // two epilogue warpgroups: warps 12..19
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kACol = 2 * kMaxN;      // accumulators at [0,176), [176,352); A stages from 352
-constexpr int kBStageBytes = kMaxN * 128;  // N rows x 64 16-bit elements (22 KB, a multiple of 1 KB)
-constexpr int kNumBoxes = 5;               // token-tile heights 16, 32, 64, 128, 176
 constexpr int kEpiCols = 16;               // accumulator columns per epilogue step
-static_assert(kACol + kStages * 32 <= kTmemCols, "tensor memory budget");
-static_assert(kBStageBytes % 1024 == 0, "token stages must stay 1 KB aligned");
 
+// Kernel shapes. Big: one CTA per SM, token tiles of up to 176 rows (prefill). Small:
+// two CTAs per SM, token tiles of up to 64 rows (batched decode, tens of tokens per
+// expert). A single thread issues one tcgen05.mma per ~120 cycles whatever N is, and
+// MMAs issued from different CTAs of an SM overlap on the tensor core, so at small N
+// two issuing CTAs per SM nearly double the weight rate.
+//   warps 0, 2: token-tile and code producers; warp 1: TMEM owner and MMA issuer;
+//   warps kDqWarp0..: DqGroups dequant warpgroups; then EpiGroups epilogue warpgroups.
+template <int MaxN, int NumBoxes, int Stages, int CStages, int DqGroups, int EpiGroups, int CtasPerSm>
+struct MmaCfg {
+    static constexpr int kMaxN = MaxN, kNumBoxes = NumBoxes, kStages = Stages, kCStages = CStages;
+    static constexpr int kDqGroups = DqGroups, kEpiGroups = EpiGroups, kCtasPerSm = CtasPerSm;
+    static constexpr int kDqWarp0 = 4, kEpiWarp0 = 4 + 4 * DqGroups;
+    static constexpr int kThreads = 32 * (kEpiWarp0 + 4 * EpiGroups);
+    static constexpr uint32_t kACol = 2 * MaxN;      // accumulators at [0,N), [N,2N); A stages from 2N
+    static constexpr uint32_t kTmemCols =
+        (kACol + Stages * 32 <= 128) ? 128u : (kACol + Stages * 32 <= 256) ? 256u : 512u;
+    static constexpr int kBStageBytes = MaxN * 128;  // N rows x 64 16-bit elements
+    static_assert(kACol + Stages * 32 <= kTmemCols && kTmemCols * CtasPerSm <= 512, "tensor memory budget");
+    static_assert(kBStageBytes % 1024 == 0, "token stages must stay 1 KB aligned");
+};
+using BigCfg = MmaCfg<kMmaTileTokens, 5, 5, 16, 2, 2, 1>;       // 640 threads, 512 TMEM columns
+using SmallCfg = MmaCfg<kMmaSmallTileTokens, 3, 4, 12, 1, 1, 2>; // 384 threads, 256 TMEM columns
+
+template <class C>
 struct MmaSmem {
-    uint8_t b[kStages][kBStageBytes];      // 1024-byte aligned
-    uint8_t codes[kCStages][kTileCodeBytes];
-    uint8_t scales[kCStages][kTileScaleBytes];
-    uint16_t stage_out[8][kEpiCols][16];   // per epilogue warp: 16 tokens x 16 outputs (gate/up)
-    uint64_t full[kStages], empty[kStages], aready[kStages];
-    uint64_t cfull[kCStages], cempty[kCStages];
+    uint8_t b[C::kStages][C::kBStageBytes];   // 1024-byte aligned
+    uint8_t codes[C::kCStages][kTileCodeBytes];
+    uint8_t scales[C::kCStages][kTileScaleBytes];
+    uint16_t stage_out[4 * C::kEpiGroups][kEpiCols][16];   // per epilogue warp: 16 tokens x 16 outputs
+    uint64_t full[C::kStages], empty[C::kStages], aready[C::kStages];
+    uint64_t cfull[C::kCStages], cempty[C::kCStages];
     uint64_t dfull[2], dempty[2];
     uint32_t tmem_base;
     int32_t abort_flag;
 };
 
+template <class C>
 struct TokenMaps {
-    CUtensorMap box[kNumBoxes];            // same tensor, box heights 16 << i
+    CUtensorMap box[C::kNumBoxes];         // same tensor, box heights 16 << i, the last kMaxN
 };
 
 enum class Proj { GateUp, Down };
@@ -108,16 +121,16 @@ __device__ unsigned long long g_mma_stats[160][kStatSlots];
 #define STAT_WAIT(slot, expr) (expr)
 #endif
 
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, MmaSmem &sm, int32_t *err) {
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, int32_t *abort_flag, int32_t *err) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
         for (int i = 0; i < 4; ++i)
             if (mbar_try_wait_sleep(bar, parity)) return true;
-        if (*reinterpret_cast<volatile int32_t *>(&sm.abort_flag)) return false;
+        if (*reinterpret_cast<volatile int32_t *>(abort_flag)) return false;
         if (global_timer_ns() - t0 > kWaitLimitNs) {
             atomicOr(err, DEV_ERR_WAIT_TIMEOUT);
-            *reinterpret_cast<volatile int32_t *>(&sm.abort_flag) = 1;
+            *reinterpret_cast<volatile int32_t *>(abort_flag) = 1;
             return false;
         }
     }
@@ -183,19 +196,25 @@ __device__ __forceinline__ uint32_t scale_pair_bf16(uint32_t h, __half2 scale2) 
     return *reinterpret_cast<const uint32_t *>(&b);
 }
 
-// Token-tile heights: 16, 32, 64, 128, then kMaxN.
-__device__ __forceinline__ int box_rows(int i) { return i < kNumBoxes - 1 ? (16 << i) : kMaxN; }
+// Token-tile heights: 16, 32, 64, 128, ..., then kMaxN.
+template <class C>
+__host__ __device__ __forceinline__ int box_rows(int i) { return i < C::kNumBoxes - 1 ? (16 << i) : C::kMaxN; }
+template <class C>
 __device__ __forceinline__ int box_index(int rows) {
     int i = 0;
-    while (box_rows(i) < rows && i < kNumBoxes - 1) ++i;
+    while (box_rows<C>(i) < rows && i < C::kNumBoxes - 1) ++i;
     return i;
 }
 
-template <Proj P>
-__global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant__ TokenMaps maps, const MmaArgs a)
+template <class C, Proj P>
+__global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const __grid_constant__ TokenMaps<C> maps,
+                                                                         const MmaArgs a)
 {
+    constexpr int kMaxN = C::kMaxN, kStages = C::kStages, kCStages = C::kCStages;
+    constexpr int kDqWarp0 = C::kDqWarp0, kEpiWarp0 = C::kEpiWarp0, kBStageBytes = C::kBStageBytes;
+    constexpr uint32_t kTmemCols = C::kTmemCols, kACol = C::kACol;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    MmaSmem &sm = *reinterpret_cast<MmaSmem *>(
+    MmaSmem<C> &sm = *reinterpret_cast<MmaSmem<C> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KT = a.K / kTileK, RT = a.R / kM;
@@ -215,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.dfull[b], 1);
-            mbar_init(&sm.dempty[b], 256);
+            mbar_init(&sm.dempty[b], 128 * C::kEpiGroups);
         }
         sm.abort_flag = 0;
         fence_mbar_init();
@@ -243,18 +262,18 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
             for (int t = blockIdx.x; t < n_tiles && !sm.abort_flag; t += gridDim.x) {
                 const int32_t *ent = a.entries + 4 * (t / RT);
                 const int e = __ldg(ent), row0 = __ldg(ent + 1), rows = __ldg(ent + 2);
-                const int rt = t % RT, bi = box_index(rows);
-                const uint32_t b_bytes = (uint32_t)box_rows(bi) * 128u;
+                const int rt = t % RT, bi = box_index<C>(rows);
+                const uint32_t b_bytes = (uint32_t)box_rows<C>(bi) * 128u;
                 const size_t rti = (size_t)e * RT + rt;
                 for (int kt = 0; kt < KT; ++kt, ++g) {
                     const int s = g % nst;
                     const uint32_t ph = (g / nst) & 1u;
                     if (tokens) {
-                        if (!STAT_WAIT(0, wait_or_abort(&sm.empty[s], ph ^ 1u, sm, a.err_word))) break;
+                        if (!STAT_WAIT(0, wait_or_abort(&sm.empty[s], ph ^ 1u, &sm.abort_flag, a.err_word))) break;
                         mbar_arrive_expect_tx(&sm.full[s], b_bytes);
                         tma_load_2d(sm.b[s], &maps.box[bi], kt * kTileK, row0, &sm.full[s]);
                     } else {
-                        if (!STAT_WAIT(1, wait_or_abort(&sm.cempty[s], ph ^ 1u, sm, a.err_word))) break;
+                        if (!STAT_WAIT(1, wait_or_abort(&sm.cempty[s], ph ^ 1u, &sm.abort_flag, a.err_word))) break;
                         mbar_arrive_expect_tx(&sm.cfull[s], kTileCodeBytes + kTileScaleBytes);
                         bulk_g2s(sm.codes[s], a.codes + (rti * KT + kt) * kTileCodeBytes, kTileCodeBytes, &sm.cfull[s]);
                         bulk_g2s(sm.scales[s], a.scales + scale_offset(rti, KT, kt), kTileScaleBytes, &sm.cfull[s]);
@@ -280,16 +299,16 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
             uint32_t g = 0, tile_i = 0;
             for (int t = blockIdx.x; t < n_tiles && !sm.abort_flag; t += gridDim.x, ++tile_i) {
                 const int rows = __ldg(a.entries + 4 * (t / RT) + 2);
-                const uint32_t idesc = instr_desc_16bit(box_rows(box_index(rows)), kType);
+                const uint32_t idesc = instr_desc_16bit(box_rows<C>(box_index<C>(rows)), kType);
                 const int buf = tile_i & 1;
-                if (!STAT_WAIT(2, wait_or_abort(&sm.dempty[buf], ((tile_i >> 1) & 1u) ^ 1u, sm, a.err_word))) break;
+                if (!STAT_WAIT(2, wait_or_abort(&sm.dempty[buf], ((tile_i >> 1) & 1u) ^ 1u, &sm.abort_flag, a.err_word))) break;
                 tc_fence_after();
                 const uint32_t dt = tmem + (uint32_t)buf * kMaxN;
                 bool ok = true;
                 for (int kt = 0; kt < KT; ++kt, ++g) {
                     const int s = g % kStages;
                     const uint32_t ph = (g / kStages) & 1u;
-                    if (!STAT_WAIT(4, wait_or_abort(&sm.aready[s], ph, sm, a.err_word))) { ok = false; break; }
+                    if (!STAT_WAIT(4, wait_or_abort(&sm.aready[s], ph, &sm.abort_flag, a.err_word))) { ok = false; break; }
 #ifdef TFMOE_MMA_STATS
                     const long long tm0 = clock64();
 #endif
@@ -315,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
             }
         }
     } else if (warp >= kDqWarp0 && warp < kEpiWarp0) {
-        // decode: warpgroup gq takes the stages g with g % 2 == gq (all 64 columns), so two
+        // decode: warpgroup gq takes the stages g with g % kDqGroups == gq (all 64 columns), so
         // stages are decoded concurrently; thread q owns weight row q = TMEM lane q
         const int gq = (warp - kDqWarp0) >> 2;
         const int q = (warp & 3) * 32 + lane;
@@ -324,19 +343,19 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
         bool ok = true;
         for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
             for (int kt = 0; kt < KT; ++kt, ++g) {
-                if ((int)(g & 1u) != gq) continue;
+                if ((int)(g % C::kDqGroups) != gq) continue;
                 const int s = g % kStages, cs = g % kCStages;
                 const uint32_t ph = (g / kStages) & 1u, pc = (g / kCStages) & 1u;
-                ok = (lane == 0) ? STAT_WAIT(5, wait_or_abort(&sm.cfull[cs], pc, sm, a.err_word))
-                                 : wait_or_abort(&sm.cfull[cs], pc, sm, a.err_word);
+                ok = (lane == 0) ? STAT_WAIT(5, wait_or_abort(&sm.cfull[cs], pc, &sm.abort_flag, a.err_word))
+                                 : wait_or_abort(&sm.cfull[cs], pc, &sm.abort_flag, a.err_word);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 const uint4 c0 = *reinterpret_cast<const uint4 *>(sm.codes[cs] + q * 16);
                 const uint4 c1 = *reinterpret_cast<const uint4 *>(sm.codes[cs] + 2048 + q * 16);
                 const uint32_t sc4 = *reinterpret_cast<const uint32_t *>(sm.scales[cs] + q * 4);
                 mbar_arrive(&sm.cempty[cs]);                              // code stage consumed
-                ok = (lane == 0) ? STAT_WAIT(6, wait_or_abort(&sm.empty[s], ph ^ 1u, sm, a.err_word))
-                                 : wait_or_abort(&sm.empty[s], ph ^ 1u, sm, a.err_word);  // A stage free
-                if (ok) ok = wait_or_abort(&sm.full[s], ph, sm, a.err_word);             // token tile landed
+                ok = (lane == 0) ? STAT_WAIT(6, wait_or_abort(&sm.empty[s], ph ^ 1u, &sm.abort_flag, a.err_word))
+                                 : wait_or_abort(&sm.empty[s], ph ^ 1u, &sm.abort_flag, a.err_word);  // A stage free
+                if (ok) ok = wait_or_abort(&sm.full[s], ph, &sm.abort_flag, a.err_word);             // token tile landed
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 const uint32_t s01 = e4m3x2_to_f16x2(sc4 & 0xFFFFu), s23 = e4m3x2_to_f16x2(sc4 >> 16);
                 const __half2 h01 = *reinterpret_cast<const __half2 *>(&s01);
@@ -368,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
     } else if (warp >= kEpiWarp0) {
         // two warpgroups split the accumulator columns in steps of 16; one buffer behind the MMAs
         const int eg = (warp - kEpiWarp0) >> 2;
-        const int ew = warp - kEpiWarp0;                           // 0..7: staging slot
+        const int ew = warp - kEpiWarp0;                           // staging slot
         const int q = (warp & 3) * 32 + lane;                      // weight row = TMEM lane
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         uint32_t tile_i = 0;
@@ -376,24 +395,24 @@ __global__ void __launch_bounds__(kThreads, 1) mma_kernel(const __grid_constant_
             const int32_t *ent = a.entries + 4 * (t / RT);
             const int e = __ldg(ent), row0 = __ldg(ent + 1), rows = __ldg(ent + 2);
             const int rt = t % RT;
-            const int n = box_rows(box_index(rows));
+            const int n = box_rows<C>(box_index<C>(rows));
             const int buf = tile_i & 1;
-            if (!((lane == 0) ? STAT_WAIT(7, wait_or_abort(&sm.dfull[buf], (tile_i >> 1) & 1u, sm, a.err_word))
-                              : wait_or_abort(&sm.dfull[buf], (tile_i >> 1) & 1u, sm, a.err_word)))
+            if (!((lane == 0) ? STAT_WAIT(7, wait_or_abort(&sm.dfull[buf], (tile_i >> 1) & 1u, &sm.abort_flag, a.err_word))
+                              : wait_or_abort(&sm.dfull[buf], (tile_i >> 1) & 1u, &sm.abort_flag, a.err_word)))
                 break;
             tc_fence_after();
             const int grow = rt * kM + q;
             const float gs = (P == Proj::GateUp) ? ((grow & 1) ? __ldg(a.glob1 + e) : __ldg(a.glob0 + e))
                                                  : __ldg(a.glob0 + e);
-            // this group's steps: eg 0 takes steps 0, 2, 4, ..., eg 1 takes 1, 3, 5, ...
+            // this group's steps: group eg takes steps eg, eg + kEpiGroups, ...
             const int steps = n / kEpiCols;
             bool handed_back = false;
-            for (int st = eg; st < steps; st += 2) {
+            for (int st = eg; st < steps; st += C::kEpiGroups) {
                 const int c = st * kEpiCols;
                 uint32_t d[16];
                 tmem_ld16(tmem + lane_base + (uint32_t)buf * kMaxN + (uint32_t)c, d);
                 tc_wait_ld();
-                if (st + 2 >= steps) {           // last read of this group: hand the buffer back
+                if (st + C::kEpiGroups >= steps) {   // last read of this group: hand the buffer back
                     tc_fence_before();
                     mbar_arrive(&sm.dempty[buf]);
                     handed_back = true;
@@ -493,40 +512,56 @@ __global__ void __launch_bounds__(256) gather_kernel(const uint16_t *__restrict_
     }
 }
 
-size_t mma_smem_bytes() { return sizeof(MmaSmem) + 1024; }
+template <class C>
+size_t mma_smem_bytes() { return sizeof(MmaSmem<C>) + 1024; }
 
-CUresult make_token_maps(TokenMaps &m, void *base, int cols, int rows, CUtensorMapDataType type) {
-    for (int i = 0; i < kNumBoxes; ++i) {
-        const uint32_t box_rows = (uint32_t)(i < kNumBoxes - 1 ? (16 << i) : kMaxN);
+template <class C>
+CUresult make_token_maps(TokenMaps<C> &m, void *base, int cols, int rows, CUtensorMapDataType type) {
+    for (int i = 0; i < C::kNumBoxes; ++i) {
         CUresult r = encode_tensor_map_2d(&m.box[i], type, base, (uint64_t)cols, (uint64_t)rows, (uint64_t)cols * 2,
-                                          (uint32_t)kTileK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+                                          (uint32_t)kTileK, (uint32_t)box_rows<C>(i), CU_TENSOR_MAP_SWIZZLE_128B);
         if (r != CUDA_SUCCESS) return r;
     }
     return CUDA_SUCCESS;
 }
 
+template <class C>
+cudaError_t set_smem_attrs() {
+    cudaError_t e = cudaFuncSetAttribute(mma_kernel<C, Proj::GateUp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)mma_smem_bytes<C>());
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(mma_kernel<C, Proj::Down>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)mma_smem_bytes<C>());
+    return e;
+}
+
 }  // namespace
 
 struct MmaMaps {
-    TokenMaps x_perm, act;
+    TokenMaps<BigCfg> x_perm, act;
+    TokenMaps<SmallCfg> x_perm_small, act_small;
 };
+
+bool mma_use_small_tiles(const Layer &L, int T) {
+    return (long long)T * L.desc.top_k <= (long long)kMmaSmallMaxAvgTokens * L.desc.num_experts;
+}
 
 cudaError_t mma_setup(Layer &L)
 {
     const int maxP = L.desc.max_tokens * L.desc.top_k;
+    const int H = L.desc.hidden, I = L.desc.intermediate;
     MmaMaps *mm = new (std::nothrow) MmaMaps();
     if (!mm) return cudaErrorMemoryAllocation;
-    if (make_token_maps(mm->x_perm, L.ws.x_perm, L.desc.hidden, maxP, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) != CUDA_SUCCESS ||
-        make_token_maps(mm->act, L.ws.act, L.desc.intermediate, maxP, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) != CUDA_SUCCESS) {
+    if (make_token_maps(mm->x_perm, L.ws.x_perm, H, maxP, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) != CUDA_SUCCESS ||
+        make_token_maps(mm->act, L.ws.act, I, maxP, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) != CUDA_SUCCESS ||
+        make_token_maps(mm->x_perm_small, L.ws.x_perm, H, maxP, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) != CUDA_SUCCESS ||
+        make_token_maps(mm->act_small, L.ws.act, I, maxP, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) != CUDA_SUCCESS) {
         delete mm;
         return cudaErrorInvalidValue;
     }
     L.mma_maps = mm;
-    cudaError_t e = cudaFuncSetAttribute(mma_kernel<Proj::GateUp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)mma_smem_bytes());
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(mma_kernel<Proj::Down>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)mma_smem_bytes());
+    cudaError_t e = set_smem_attrs<BigCfg>();
+    if (e == cudaSuccess) e = set_smem_attrs<SmallCfg>();
     return e;
 }
 
@@ -566,7 +601,11 @@ cudaError_t launch_mma_gate_up(Layer &L, cudaStream_t s, int *launches)
     a.act_out = L.ws.act;
     a.row_inv_scale = L.ws.row_inv;
     const MmaMaps *mm = static_cast<const MmaMaps *>(L.mma_maps);
-    mma_kernel<Proj::GateUp><<<L.num_sms, kThreads, mma_smem_bytes(), s>>>(mm->x_perm, a);
+    if (L.mma_small)
+        mma_kernel<SmallCfg, Proj::GateUp><<<L.num_sms * SmallCfg::kCtasPerSm, SmallCfg::kThreads,
+                                             mma_smem_bytes<SmallCfg>(), s>>>(mm->x_perm_small, a);
+    else
+        mma_kernel<BigCfg, Proj::GateUp><<<L.num_sms, BigCfg::kThreads, mma_smem_bytes<BigCfg>(), s>>>(mm->x_perm, a);
     *launches += 1;
     return cudaGetLastError();
 }
@@ -580,7 +619,11 @@ cudaError_t launch_mma_down(Layer &L, cudaStream_t s, int *launches)
     a.R = L.desc.hidden; a.K = L.desc.intermediate;
     a.y_out = L.ws.y;
     const MmaMaps *mm = static_cast<const MmaMaps *>(L.mma_maps);
-    mma_kernel<Proj::Down><<<L.num_sms, kThreads, mma_smem_bytes(), s>>>(mm->act, a);
+    if (L.mma_small)
+        mma_kernel<SmallCfg, Proj::Down><<<L.num_sms * SmallCfg::kCtasPerSm, SmallCfg::kThreads,
+                                           mma_smem_bytes<SmallCfg>(), s>>>(mm->act_small, a);
+    else
+        mma_kernel<BigCfg, Proj::Down><<<L.num_sms, BigCfg::kThreads, mma_smem_bytes<BigCfg>(), s>>>(mm->act, a);
     *launches += 1;
     return cudaGetLastError();
 }

@@ -308,10 +308,10 @@ __global__ void __launch_bounds__(256) topk_kernel(
 // the segment, so rows are ordered by (expert, pair index): a stable counting
 // sort. Then every routed expert gets its regime and joins its regime's list.
 struct PlanArgs {
-    int E, gemv_max_tokens;
+    int E, gemv_max_tokens, mma_tile;
     uint32_t flags;
     int32_t *counts, *offsets, *perm, *inv, *regime, *gemv_list, *mma_list, *list_sizes, *err_word;
-    int32_t *mma_entries;   // [max][4]: expert, first permuted row, rows (<= kMmaTileTokens), 0
+    int32_t *mma_entries;   // [max][4]: expert, first permuted row, rows (<= mma_tile), 0
     int debug;
 };
 
@@ -415,7 +415,7 @@ __device__ void plan_block(const int32_t *__restrict__ ids, int P, const PlanArg
             n_mma += __popc(bm);
         }
         if (lane == 0) { pa.list_sizes[0] = n_gemv; pa.list_sizes[1] = n_mma; }
-        // token tiles of the MMA-regime experts: ceil(m_e / kMmaTileTokens) entries per
+        // token tiles of the MMA-regime experts: ceil(m_e / pa.mma_tile) entries per
         // expert, in expert order; lane l handles experts 8l .. 8l+7
         int ntl[8], mine = 0;
 #pragma unroll
@@ -426,7 +426,7 @@ __device__ void plan_block(const int32_t *__restrict__ ids, int P, const PlanArg
                 const int m = tot[e];
                 const bool mma = m > 0 && !(pa.flags & TFMOE_FLAG_FORCE_GEMV) &&
                                  ((pa.flags & TFMOE_FLAG_FORCE_MMA) || m > pa.gemv_max_tokens);
-                n = mma ? (m + kMmaTileTokens - 1) / kMmaTileTokens : 0;
+                n = mma ? (m + pa.mma_tile - 1) / pa.mma_tile : 0;
             }
             ntl[i] = n;
             mine += n;
@@ -444,8 +444,8 @@ __device__ void plan_block(const int32_t *__restrict__ ids, int P, const PlanArg
             for (int j = 0; j < ntl[i]; ++j, ++idx) {
                 int32_t *ent = pa.mma_entries + 4 * (size_t)idx;
                 ent[0] = e;
-                ent[1] = off[e] + j * kMmaTileTokens;
-                ent[2] = min(kMmaTileTokens, tot[e] - j * kMmaTileTokens);
+                ent[1] = off[e] + j * pa.mma_tile;
+                ent[2] = min(pa.mma_tile, tot[e] - j * pa.mma_tile);
                 ent[3] = 0;
             }
         }
@@ -543,6 +543,7 @@ static PlanArgs plan_args(const Layer &L, int T) {
     PlanArgs pa{};
     pa.E = L.desc.num_experts;
     pa.gemv_max_tokens = gemv_threshold(L, T);
+    pa.mma_tile = L.mma_small ? kMmaSmallTileTokens : kMmaTileTokens;
     pa.flags = L.desc.flags;
     pa.counts = L.ws.counts; pa.offsets = L.ws.offsets; pa.perm = L.ws.perm; pa.inv = L.ws.inv;
     pa.regime = L.ws.regime; pa.gemv_list = L.ws.gemv_list; pa.mma_list = L.ws.mma_list;
