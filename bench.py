@@ -120,13 +120,12 @@ def kernel_source_hash(stage: str = "gemv_gate_up"):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(stage: str):
-    """DRAM bytes per launch from a committed ncu capture, if it matches the current kernel source."""
+def ncu_traffic(workload: str, stage: str):
+    """DRAM bytes per launch from a committed ncu capture of this workload, if it matches the current kernel source."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
-    ent = d.get(stage)
+    ent = json.load(open(p)).get(workload, {}).get(stage)
     if not ent or ent.get("kernel_source_hash") != kernel_source_hash(stage):
         return None
     return ent.get("dram_bytes_per_launch")
@@ -151,7 +150,9 @@ def oracle_cpu_sample(shape, layers, xs, seconds: float):
     return tokens / el, oracle.max_threads(), f"{n} oracle forwards, {tokens} tokens, {el:.1f} s"
 
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend: str = "nccl"):
+    """Rank, world size, local rank and the process group (None for one process). Replicas only:
+    the group carries the timing barrier and the max over ranks, never the data path."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -160,23 +161,34 @@ def dist_setup(n_gpus):
         import datetime
 
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
         pg = dist
     return rank, world, local, pg
 
 
-def barrier(pg, torch):
+def barrier(pg, torch, cuda: bool = True):
     if pg is not None:
         pg.barrier()
-    torch.cuda.synchronize()
+    if cuda:
+        torch.cuda.synchronize()
 
 
-def max_over_ranks(pg, torch, v: float) -> float:
+def max_over_ranks(pg, torch, v: float, device: str = "cuda") -> float:
     if pg is None:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_seed(seed: int, rank: int) -> int:
+    """Each replica runs its own seeded layers (rank 0 the listed seeds)."""
+    return seed + 1000 * rank
+
+
+def weak_value(world: int, tokens_per_step: int, steps: int, ms: float) -> float:
+    """Whole-job tokens/s: the tokens all ranks processed over the slowest rank's time."""
+    return world * tokens_per_step * steps / (ms / 1e3)
 
 
 def run_reference(args):
@@ -248,7 +260,7 @@ def main():
     n_x = 8 if T <= 256 else 2
     layers_np, layers, xs = [], [], []
     for s in seeds:
-        lnp = synth.make_layer(shape, s + 1000 * rank) if rank else synth.make_layer(shape, s)
+        lnp = synth.make_layer(shape, replica_seed(s, rank))
         layers_np.append(lnp)
         L = tfmoe.MoELayer(H, I, E, k, T, has_router_bias=lnp["router_bias"] is not None, flags=args.flags,
                            gemv_max_tokens=args.gemv_max_tokens)
@@ -365,12 +377,12 @@ def main():
     clocks = sampler.stop() if sampler else None
     ms_local = ev0.elapsed_time(ev1)
     ms = max_over_ranks(pg, torch, ms_local)
-    value = world * T * args.steps / (ms / 1e3)
+    value = weak_value(world, T, args.steps, ms)
 
     # ---- per-kernel timing for the roofline: one forward per layer on a known batch, then
     # a CUDA graph that re-enqueues one stage of those forwards, rotating over the layers
     # (so consecutive launches read different weights), timed with events on its stream.
-    gemv_units, mma_pairs = [], []
+    gemv_units, mma_pairs, mma_units = [], [], []
     for li, L in enumerate(layers):
         with torch.cuda.stream(stream):
             tfmoe.check(L.forward_raw(xs[li][0].data_ptr(), T, out.data_ptr(), stream.cuda_stream))
@@ -379,6 +391,7 @@ def main():
         cnt = L.buffer_tensor(tfmoe.BUF_EXPERT_COUNTS, torch.int32, (E,)).cpu().numpy()
         gemv_units.append(int(np.sum(reg == 1)))
         mma_pairs.append(int(np.sum(cnt[reg == 2])))
+        mma_units.append(int(np.sum(reg == 2)))
     kernel_us = {}
     for stage in ("gemv_gate_up", "gemv_down", "gather", "mma_gate_up", "mma_down", "combine"):
         sid = tfmoe.STAGE_ID[stage]
@@ -422,24 +435,39 @@ def main():
         alg = float(np.mean(gemv_units)) * rows * NVFP4_BYTES_PER_WEIGHT
         achieved = alg / (kernel_us[dominant] * 1e-6) / 1e9
         roofline = {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                    "frac": achieved / hbm_peak, "traffic": ncu_traffic(dominant),
+                    "frac": achieved / hbm_peak, "traffic": ncu_traffic(args.workload, dominant),
                     "algorithmic_bytes_per_launch": alg, "avg_launch_us": kernel_us[dominant],
                     "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback",
                     "how": how}
     elif dominant in ("mma_gate_up", "mma_down"):
+        # the tensor-core kernel's bound follows its arithmetic intensity: FLOPs per weight
+        # byte against the ratio of the measured peaks (a few tokens per expert stream
+        # weights, hundreds of tokens per expert keep the tensor pipe busy)
         rows = 2 * I if dominant == "mma_gate_up" else H
         kdim = H if dominant == "mma_gate_up" else I
-        alg = 2.0 * float(np.mean(mma_pairs)) * rows * kdim
-        achieved = alg / (kernel_us[dominant] * 1e-6) / 1e12
-        roofline = {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": bf16_peak,
-                    "unit": "TFLOP/s", "frac": achieved / bf16_peak, "traffic": ncu_traffic(dominant),
-                    "algorithmic_flops_per_launch": alg, "avg_launch_us": kernel_us[dominant],
-                    "peak_source": ("measured (MEASURED_PEAKS.json bf16_tflops, burst)" if peak_src == "measured"
-                                    else "fallback"),
-                    "how": how}
+        flops = 2.0 * float(np.mean(mma_pairs)) * rows * kdim
+        wbytes = float(np.mean(mma_units)) * rows * kdim * NVFP4_BYTES_PER_WEIGHT
+        t_s = kernel_us[dominant] * 1e-6
+        if wbytes > 0 and flops / wbytes < (bf16_peak * 1e12) / (hbm_peak * 1e9):
+            achieved = wbytes / t_s / 1e9
+            roofline = {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                        "frac": achieved / hbm_peak, "traffic": ncu_traffic(args.workload, dominant),
+                        "algorithmic_bytes_per_launch": wbytes, "algorithmic_flops_per_launch": flops,
+                        "avg_launch_us": kernel_us[dominant],
+                        "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback",
+                        "how": how}
+        else:
+            achieved = flops / t_s / 1e12
+            roofline = {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": bf16_peak,
+                        "unit": "TFLOP/s", "frac": achieved / bf16_peak, "traffic": ncu_traffic(args.workload, dominant),
+                        "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": wbytes,
+                        "avg_launch_us": kernel_us[dominant],
+                        "peak_source": ("measured (MEASURED_PEAKS.json bf16_tflops, burst)" if peak_src == "measured"
+                                        else "fallback"),
+                        "how": how}
     else:
         roofline = {"bound": "hbm", "kernel": dominant, "achieved": None, "peak": hbm_peak, "unit": "GB/s",
-                    "frac": None, "traffic": ncu_traffic(dominant), "avg_launch_us": kernel_us[dominant]}
+                    "frac": None, "traffic": ncu_traffic(args.workload, dominant), "avg_launch_us": kernel_us[dominant]}
 
     # ---- per-stage times of ordinary (profiled, host-synchronised) forwards; these include
     # host launch gaps and are reported for orientation only
