@@ -48,11 +48,14 @@ constexpr int kThreads = (kComputeWarps + 1) * 32;   // + the control warp
 #endif
 constexpr int kCtasPerSm = TFMOE_GEMV_CTAS_PER_SM;
 #ifndef TFMOE_GEMV_RING
-#define TFMOE_GEMV_RING 6
+#define TFMOE_GEMV_RING 3
 #endif
-constexpr int kChunk = 2;          // column tiles per ring slot of a compute warp
+#ifndef TFMOE_GEMV_CHUNK
+#define TFMOE_GEMV_CHUNK 4
+#endif
+constexpr int kChunk = TFMOE_GEMV_CHUNK;   // column tiles per ring slot of a compute warp
 constexpr int kRing = TFMOE_GEMV_RING;   // ring slots per compute warp (kRing - 1 chunks in flight)
-static_assert(kRing >= 3, "ring depth");
+static_assert(kRing >= 2, "ring depth");
 constexpr int kMaxNT = TFMOE_GEMV_TOKENS_PER_PASS;   // tokens per pass (2 or 4)
 static_assert(kMaxNT == 2 || kMaxNT == 4, "tokens per pass");
 
@@ -412,24 +415,31 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     const uint4 *ring = reinterpret_cast<const uint4 *>(base + lay.ring) + (size_t)warp * kRing * kChunk * 32 + lane;
     const int nch = (KTW + kChunk - 1) / kChunk;
     int ptask = -1, pt0 = 0, pch = 0, slot_fill = 0;
+    const uint8_t *pg = nullptr;                          // next chunk of the stream (this lane's bytes)
     {
         int ft;
-        if (first_pass(ft)) ptask = ft;
+        if (first_pass(ft)) { ptask = ft; pg = lane_codes(ft); }
     }
     auto refill = [&]() {
         if (ptask >= 0) {
-            const uint8_t *g = lane_codes(ptask) + (size_t)pch * kChunk * kTileCodeBytes;
             const int n = min(kChunk, KTW - pch * kChunk);
             uint4 *d = const_cast<uint4 *>(ring) + (size_t)slot_fill * kChunk * 32;
 #pragma unroll
             for (int j = 0; j < kChunk; ++j)
-                if (j < n) cp_async16(d + j * 32, g + (size_t)j * kTileCodeBytes);
+                if (j < n) cp_async16(d + j * 32, pg + (size_t)j * kTileCodeBytes);
+            pg += (size_t)kChunk * kTileCodeBytes;
             if (++pch == nch) {
                 pch = 0;
                 int rb, ntask, nt0;
                 const int m = task_rows(ptask, rb);
-                if (next_pass(ptask, pt0, m, ntask, nt0)) { ptask = ntask; pt0 = nt0; }
-                else ptask = -1;
+                if (next_pass(ptask, pt0, m, ntask, nt0)) {
+                    if (ntask != ptask) pg = lane_codes(ntask);
+                    else pg -= (size_t)nch * kChunk * kTileCodeBytes;   // same task, next tokens
+                    ptask = ntask;
+                    pt0 = nt0;
+                } else {
+                    ptask = -1;
+                }
             }
         }
         cp_async_commit();

@@ -152,7 +152,7 @@ template <int M>
 __global__ void __launch_bounds__(256) router_split_kernel(
     const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, const float *__restrict__ bias,
     float *__restrict__ logits, double *__restrict__ partial, int T, int H, int E, int k_len, int32_t *err_word,
-    int debug)
+    int debug, uint16_t *xq, float *xq_inv)
 {
     constexpr int TT = 16 * M, TE = 16 * M, KC = 32;
     __shared__ double xs[KC][TT + 1];
@@ -214,46 +214,69 @@ __global__ void __launch_bounds__(256) router_split_kernel(
             }
         }
     }
+    // the CTAs of the first expert tile also write the GEMV regime's x operand for their
+    // tokens and hidden-dimension slice (16-element blocks, see block16_bf16_to_f16)
+    if (xq && blockIdx.y == 0) {
+        const int rows = min(TT, T - t_base), blocks = k_len / 16;
+        for (int i = threadIdx.x; i < rows * blocks; i += blockDim.x) {
+            const int t = t_base + i / blocks;
+            const size_t off = (size_t)t * H + k_begin + (size_t)(i % blocks) * 16;
+            xq_inv[off / 16] = block16_bf16_to_f16(x + off, xq + off);
+        }
+    }
 }
 
 // One warp per token: k rounds of a warp arg-max over (logit desc, index asc),
 // then softmax over the selected logits (max-subtracted, fp32).
 constexpr int kMaxEPerLane = 8;   // E <= 256
-__device__ __forceinline__ void topk_warp(const float *row, int E, int k, int32_t *ids_row, float *w_row)
+
+// Order-preserving key of a finite fp32 logit: a larger logit has a larger key, and -0
+// counts as +0 (equal logits tie). No finite logit maps to key 0.
+__device__ __forceinline__ uint32_t logit_key(float v) {
+    uint32_t b = __float_as_uint(v);
+    if ((b << 1) == 0u) b = 0u;
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// One warp selects a token's top k experts: k rounds, each a lane-local best (largest key,
+// lowest expert on ties) followed by a warp-wide max of the keys and a min of the expert ids
+// that hold it (two redux.sync), so ties go to the lower expert index.
+__device__ __forceinline__ void topk_warp(const float *row, int E, int k, int32_t *ids_row, float *w_row,
+                                          int32_t *ids_copy = nullptr)
 {
     const int lane = threadIdx.x & 31;
     float v[kMaxEPerLane];
+    uint32_t key[kMaxEPerLane];
+    uint32_t taken = 0;                       // bit i: candidate lane + 32 i used or absent
 #pragma unroll
     for (int i = 0; i < kMaxEPerLane; ++i) {
         const int e = lane + 32 * i;
-        v[i] = (e < E) ? __ldcg(row + e) : -INFINITY;
+        v[i] = (e < E) ? __ldcg(row + e) : 0.f;
+        key[i] = logit_key(v[i]);
+        if (e >= E) taken |= 1u << i;
     }
-    uint32_t taken = 0;
     float sel_first = 0.f, my_sel = 0.f;
     int my_id = -1;
     for (int s = 0; s < k; ++s) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
+        uint32_t bk = 0u;
+        float bv = 0.f;
 #pragma unroll
         for (int i = 0; i < kMaxEPerLane; ++i) {
-            const int e = lane + 32 * i;
-            if (e < E && !(taken & (1u << i)) && (v[i] > bv || (v[i] == bv && e < bi) || bi == 0x7fffffff)) {
+            if (!(taken & (1u << i)) && key[i] > bk) {   // strict: the lower i (lower expert) keeps ties
+                bk = key[i];
                 bv = v[i];
-                bi = e;
             }
         }
+        const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
+        uint32_t mine = 0xffffffffu;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
-                bv = ov;
-                bi = oi;
-            }
-        }
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-        if (s == 0) sel_first = bv;
-        if (lane == s) { my_sel = bv; my_id = bi; }
+        for (int i = kMaxEPerLane - 1; i >= 0; --i)
+            if (!(taken & (1u << i)) && key[i] == mk) mine = (uint32_t)(lane + 32 * i);
+        const uint32_t win = __reduce_min_sync(0xffffffffu, mine);
+        const float wv = __shfl_sync(0xffffffffu, bv, (int)(win & 31u));
+        if ((int)(win & 31u) == lane) taken |= 1u << (win >> 5);
+        if (s == 0) sel_first = wv;
+        if (lane == s) { my_sel = wv; my_id = (int)win; }
     }
     const float ex = (lane < k) ? expf(my_sel - sel_first) : 0.f;
     float den = ex;
@@ -262,6 +285,7 @@ __device__ __forceinline__ void topk_warp(const float *row, int E, int k, int32_
     if (lane < k) {
         ids_row[lane] = my_id;
         w_row[lane] = ex / den;
+        if (ids_copy) ids_copy[lane] = my_id;
     }
 }
 
@@ -317,6 +341,33 @@ struct PlanArgs {
 
 __host__ __device__ constexpr size_t plan_smem_ints(int warps, int E) { return (size_t)warps * E + 2 * E + 1; }
 
+// ids: the pairs' expert ids, written by an earlier kernel (global) or by this CTA (shared).
+// Exclusive scan of tot[0..E) into off[0..E] by one warp (E <= 256: 8 experts per lane).
+__device__ __forceinline__ void scan_experts_warp(const int32_t *tot, int32_t *off, int E) {
+    const int lane = threadIdx.x & 31;
+    int local[8], s = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = lane * 8 + i;
+        local[i] = (e < E) ? tot[e] : 0;
+        s += local[i];
+    }
+    int incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    int run = incl - s;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = lane * 8 + i;
+        if (e < E) off[e] = run;
+        run += local[i];
+    }
+    if (lane == 31) off[E] = incl;
+}
+
 __device__ void plan_block(const int32_t *__restrict__ ids, int P, const PlanArgs &pa, int32_t *sm)
 {
     const int E = pa.E;
@@ -325,74 +376,85 @@ __device__ void plan_block(const int32_t *__restrict__ ids, int P, const PlanArg
     int32_t *tot = sm + W * E;       // [E]
     int32_t *off = tot + E;          // [E+1]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int i = threadIdx.x; i < W * E; i += blockDim.x) cnt[i] = 0;
-    __syncthreads();
-    const int seg = (P + W - 1) / W;
-    const int p_begin = min(P, warp * seg), p_end = min(P, p_begin + seg);
-    int32_t *my_cnt = cnt + warp * E;
-    for (int p0 = p_begin; p0 < p_end; p0 += 32) {
-        const int p = p0 + lane;
-        int e = (p < p_end) ? __ldcg(ids + p) : -1;
-        if (e >= E || (e < 0 && p < p_end)) {
-            if (pa.debug) atomicOr(pa.err_word, DEV_ERR_BAD_EXPERT);
-            e = -1;
+    if (P <= (int)blockDim.x && P <= W * E) {
+        // small batches: one thread per pair; the count comes from shared atomics and the
+        // stable rank from the earlier pairs with the same expert, read from a shared copy
+        int32_t *ids_s = cnt;
+        for (int e = threadIdx.x; e < E; e += blockDim.x) tot[e] = 0;
+        for (int i = threadIdx.x; i < P; i += blockDim.x) ids_s[i] = ids[i];
+        __syncthreads();
+        const int p = threadIdx.x;
+        int e = -1;
+        if (p < P) {
+            e = ids_s[p];
+            if (e >= E || e < 0) {
+                if (pa.debug) atomicOr(pa.err_word, DEV_ERR_BAD_EXPERT);
+                e = -1;
+            } else {
+                atomicAdd(&tot[e], 1);
+            }
         }
-        const uint32_t m = __match_any_sync(0xffffffffu, e);
-        if (e >= 0 && lane == __ffs(m) - 1) my_cnt[e] += __popc(m);
-        __syncwarp();
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int run = 0;
-        for (int w = 0; w < W; ++w) {
-            const int c = cnt[w * E + e];
-            cnt[w * E + e] = run;
-            run += c;
-        }
-        tot[e] = run;
-    }
-    __syncthreads();
-    if (warp == 0) {   // exclusive scan of tot over experts, E <= 256: 8 per lane
-        int local[8], s = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int e = lane * 8 + i;
-            local[i] = (e < E) ? tot[e] : 0;
-            s += local[i];
-        }
-        int incl = s;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        int run = incl - s;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int e = lane * 8 + i;
-            if (e < E) off[e] = run;
-            run += local[i];
-        }
-        if (lane == 31) off[E] = incl;
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < W * E; i += blockDim.x) cnt[i] += off[i % E];
-    for (int e = threadIdx.x; e <= E; e += blockDim.x) pa.offsets[e] = off[e];
-    __syncthreads();
-    for (int p0 = p_begin; p0 < p_end; p0 += 32) {
-        const int p = p0 + lane;
-        int e = (p < p_end) ? __ldcg(ids + p) : -1;
-        if (e >= E) e = -1;
-        const uint32_t m = __match_any_sync(0xffffffffu, e);
+        __syncthreads();
+        if (warp == 0) scan_experts_warp(tot, off, E);
+        __syncthreads();
+        for (int i = threadIdx.x; i <= E; i += blockDim.x) pa.offsets[i] = off[i];
         if (e >= 0) {
-            const int rank = __popc(m & ((1u << lane) - 1u));
-            const int r = my_cnt[e] + rank;
+            int rank = 0;
+            for (int q = 0; q < p; ++q) rank += (ids_s[q] == e);
+            const int r = off[e] + rank;
             pa.perm[r] = p;
             pa.inv[p] = r;
         }
-        __syncwarp();
-        if (e >= 0 && lane == __ffs(m) - 1) my_cnt[e] += __popc(m);
-        __syncwarp();
+    } else {
+        // P contiguous pairs split into W warp segments: count per (segment, expert), scan,
+        // then place each pair at its segment's base + its rank among same-expert pairs
+        for (int i = threadIdx.x; i < W * E; i += blockDim.x) cnt[i] = 0;
+        __syncthreads();
+        const int seg = (P + W - 1) / W;
+        const int p_begin = min(P, warp * seg), p_end = min(P, p_begin + seg);
+        int32_t *my_cnt = cnt + warp * E;
+        for (int p0 = p_begin; p0 < p_end; p0 += 32) {
+            const int p = p0 + lane;
+            int e = (p < p_end) ? ids[p] : -1;
+            if (e >= E || (e < 0 && p < p_end)) {
+                if (pa.debug) atomicOr(pa.err_word, DEV_ERR_BAD_EXPERT);
+                e = -1;
+            }
+            const uint32_t m = __match_any_sync(0xffffffffu, e);
+            if (e >= 0 && lane == __ffs(m) - 1) my_cnt[e] += __popc(m);
+            __syncwarp();
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            int run = 0;
+            for (int w = 0; w < W; ++w) {
+                const int c = cnt[w * E + e];
+                cnt[w * E + e] = run;
+                run += c;
+            }
+            tot[e] = run;
+        }
+        __syncthreads();
+        if (warp == 0) scan_experts_warp(tot, off, E);
+        __syncthreads();
+        for (int i = threadIdx.x; i < W * E; i += blockDim.x) cnt[i] += off[i % E];
+        for (int e = threadIdx.x; e <= E; e += blockDim.x) pa.offsets[e] = off[e];
+        __syncthreads();
+        for (int p0 = p_begin; p0 < p_end; p0 += 32) {
+            const int p = p0 + lane;
+            int e = (p < p_end) ? ids[p] : -1;
+            if (e >= E) e = -1;
+            const uint32_t m = __match_any_sync(0xffffffffu, e);
+            if (e >= 0) {
+                const int rank = __popc(m & ((1u << lane) - 1u));
+                const int r = my_cnt[e] + rank;
+                pa.perm[r] = p;
+                pa.inv[p] = r;
+            }
+            __syncwarp();
+            if (e >= 0 && lane == __ffs(m) - 1) my_cnt[e] += __popc(m);
+            __syncwarp();
+        }
     }
     if (warp == 0) {
         int n_gemv = 0, n_mma = 0;
@@ -475,53 +537,42 @@ __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(
     PlanArgs pa, int32_t *counter, uint16_t *xq, float *xq_inv)
 {
     extern __shared__ int32_t sm[];
-    __shared__ double red[kFusedThreads / 32][kFusedMaxT];
     __shared__ int is_last;
     const int E = pa.E, e = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    double acc[kFusedMaxT];
-#pragma unroll
-    for (int t = 0; t < kFusedMaxT; ++t) acc[t] = 0.0;
+    // logits of expert e: warp w takes tokens w, w + 8 (T <= 16); lane l covers 8 columns per
+    // 256-column step, and the warp adds its lanes in a fixed shuffle order
     const uint16_t *wrow = wr + (size_t)e * H;
-    for (int c = threadIdx.x * 8; c < H; c += kFusedThreads * 8) {
-        const uint4 wv = *reinterpret_cast<const uint4 *>(wrow + c);
-        const uint32_t wu[4] = {wv.x, wv.y, wv.z, wv.w};
-        double w[8];
+    for (int t = warp; t < T; t += kFusedThreads / 32) {
+        const uint16_t *xrow = x + (size_t)t * H;
+        double acc = 0.0;
+        for (int c0 = lane * 8; c0 < H; c0 += 256 * 8) {
+            uint4 wv[8], xv[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            w[2 * i] = (double)bf16_bits_to_float(wu[i] & 0xFFFFu);
-            w[2 * i + 1] = (double)bf16_bits_to_float(wu[i] >> 16);
-        }
+            for (int u = 0; u < 8; ++u) {
+                const int c = c0 + u * 256;
+                wv[u] = (c < H) ? *reinterpret_cast<const uint4 *>(wrow + c) : make_uint4(0, 0, 0, 0);
+                xv[u] = (c < H) ? *reinterpret_cast<const uint4 *>(xrow + c) : make_uint4(0, 0, 0, 0);
+            }
 #pragma unroll
-        for (int t = 0; t < kFusedMaxT; ++t) {
-            if (t < T) {
-                const uint4 xv = *reinterpret_cast<const uint4 *>(x + (size_t)t * H + c);
-                const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
+            for (int u = 0; u < 8; ++u) {
+                const uint32_t wu[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
+                const uint32_t xu[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    acc[t] = fma((double)bf16_bits_to_float(xu[i] & 0xFFFFu), w[2 * i], acc[t]);
-                    acc[t] = fma((double)bf16_bits_to_float(xu[i] >> 16), w[2 * i + 1], acc[t]);
+                    acc = fma((double)bf16_bits_to_float(xu[i] & 0xFFFFu), (double)bf16_bits_to_float(wu[i] & 0xFFFFu), acc);
+                    acc = fma((double)bf16_bits_to_float(xu[i] >> 16), (double)bf16_bits_to_float(wu[i] >> 16), acc);
                 }
             }
         }
-    }
 #pragma unroll
-    for (int t = 0; t < kFusedMaxT; ++t) {
-        if (t < T) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
-            if (lane == 0) red[warp][t] = acc[t];
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) {
+            float l = (float)acc;
+            if (bias) l = l + bias[e];
+            if (pa.debug && !isfinite(l)) atomicOr(pa.err_word, DEV_ERR_NONFINITE);
+            logits[(size_t)t * E + e] = l;
         }
-    }
-    __syncthreads();
-    if (threadIdx.x < T) {
-        double v = 0.0;
-#pragma unroll
-        for (int w = 0; w < kFusedThreads / 32; ++w) v += red[w][threadIdx.x];
-        float l = (float)v;
-        if (bias) l = l + bias[e];
-        if (pa.debug && !isfinite(l)) atomicOr(pa.err_word, DEV_ERR_NONFINITE);
-        logits[(size_t)threadIdx.x * E + e] = l;
     }
     if (xq) convert_x_blocks(x, T, H, xq, xq_inv);
     __threadfence();
@@ -530,10 +581,12 @@ __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(
     __syncthreads();
     if (!is_last) return;
     __threadfence();
+    // the ids stay in shared memory for the plan: no global round trip on the serial tail
+    __shared__ int32_t ids_sm[kFusedMaxT * 32];
     for (int t = warp; t < T; t += kFusedThreads / 32)
-        topk_warp(logits + (size_t)t * E, E, k, ids + (size_t)t * k, wts + (size_t)t * k);
+        topk_warp(logits + (size_t)t * E, E, k, ids + (size_t)t * k, wts + (size_t)t * k, ids_sm + t * k);
     __syncthreads();
-    plan_block(ids, T * k, pa, sm);
+    plan_block(ids_sm, T * k, pa, sm);
     if (threadIdx.x == 0) *counter = 0;
 }
 
@@ -585,16 +638,15 @@ cudaError_t launch_router(Layer &L, const uint16_t *x, int T, cudaStream_t s, in
         dim3 grid((T + tile - 1) / tile, (E + tile - 1) / tile, S);
         if (M == 4)
             router_split_kernel<4><<<grid, 256, 0, s>>>(x, L.w.router_w, bias, L.ws.logits, partial, T, H, E, H / S,
-                                                        L.ws.err_word, debug);
+                                                        L.ws.err_word, debug, gemv ? L.ws.xq : nullptr, L.ws.xq_inv);
         else
             router_split_kernel<2><<<grid, 256, 0, s>>>(x, L.w.router_w, bias, L.ws.logits, partial, T, H, E, H / S,
-                                                        L.ws.err_word, debug);
+                                                        L.ws.err_word, debug, gemv ? L.ws.xq : nullptr, L.ws.xq_inv);
     }
     {
         StageTimer timer(L, TFMOE_STAGE_TOPK, s);
-        topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(L.ws.logits, L.ws.ids, L.ws.topk_w, T, E, k, x, H,
-                                                  gemv ? L.ws.xq : nullptr, L.ws.xq_inv, partial, S, bias,
-                                                  L.ws.err_word, debug);
+        topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(L.ws.logits, L.ws.ids, L.ws.topk_w, T, E, k, x, H, nullptr, nullptr,
+                                                  partial, S, bias, L.ws.err_word, debug);
     }
     *launches += 2;
     return cudaGetLastError();
