@@ -77,6 +77,10 @@ void carve_workspace(Layer &L, uint8_t *base, size_t *total) {
     c.take(&w.list_sizes, 4, base);
     c.take(&w.err_word, 1, base);
     c.take(&w.route_counter, 1, base);
+    c.take(&w.seg_cnt, ((T + 7) / 8) * E, base);
+    c.take(&w.seg_base, ((T + 7) / 8) * E, base);
+    c.take(&w.plan_tot, E, base);
+    c.take(&w.plan_counter, 1, base);
     c.take(&w.mma_entries, 4 * max_mma_entries(P, E), base);
     c.take(&w.x_perm, P * H, base);
     c.take(&w.row_inv, P, base);
@@ -191,6 +195,7 @@ tfmoe_status tfmoe_create(const tfmoe_layer_desc *desc, tfmoe_layer **out)
     carve_weights(L, static_cast<uint8_t *>(L.w_block), &L.w_bytes);
     e = cudaMemset(L.ws.err_word, 0, sizeof(int32_t));
     if (e == cudaSuccess) e = cudaMemset(L.ws.route_counter, 0, sizeof(int32_t));
+    if (e == cudaSuccess) e = cudaMemset(L.ws.plan_counter, 0, sizeof(int32_t));
     if (e == cudaSuccess) e = gemv_setup(L);
     if (e == cudaSuccess) e = mma_setup(L);
     if (e != cudaSuccess) {

@@ -43,6 +43,10 @@ constexpr int kDefaultGemvMaxTokens = 2;
 constexpr int kRouterMaxSlices = 16;
 constexpr size_t kRouterPartialMax = size_t(1) << 22;
 
+// Batches with more than this many (token, expert) pairs build the plan with a
+// multi-CTA scan instead of one CTA.
+constexpr int kLargePlanPairs = 4096;
+
 // Tokens per tensor-core tile (the MMA N dimension): up to kMmaTileTokens with one CTA
 // per SM, or up to kMmaSmallTileTokens with two CTAs per SM when a batch averages at most
 // kMmaSmallMaxAvgTokens tokens per expert.
@@ -66,6 +70,10 @@ struct Workspace {
     int32_t *list_sizes = nullptr;  // [4]   n_gemv, n_mma, n_mma_entries, (reserved)
     int32_t *err_word = nullptr;    // [1]
     int32_t *route_counter = nullptr; // [1] arrivals of the fused routing kernel (left at 0)
+    int32_t *seg_cnt = nullptr;     // [ceil(maxT/8)][E] per-segment expert counts (large-batch plan)
+    int32_t *seg_base = nullptr;    // [ceil(maxT/8)][E] per-segment first ranks
+    int32_t *plan_tot = nullptr;    // [E]
+    int32_t *plan_counter = nullptr; // [1] arrivals of the plan scan (left at 0)
     int32_t *mma_entries = nullptr; // [max_mma_entries][4] token tiles of the MMA regime
     uint16_t *x_perm = nullptr;     // [maxP][H] f16 activation rows (times 2^sh) in permuted order (MMA regime)
     float *row_inv = nullptr;       // [maxP] 2^-sh of each x_perm row

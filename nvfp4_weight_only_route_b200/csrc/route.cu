@@ -303,27 +303,44 @@ __device__ __forceinline__ void convert_x_blocks(const uint16_t *__restrict__ x,
 // One warp per token; with xq given, the grid also writes the GEMV regime's x operand.
 // With S > 1 fp64 partial sums [S][T][E], the warp first adds them in slice order,
 // rounds once to fp32, adds the bias and stores the token's logits.
+// Tokens per top-k CTA (one warp each); a CTA's pairs form one segment of the plan.
+constexpr int kTopkTokens = 8;
+
 __global__ void __launch_bounds__(256) topk_kernel(
     float *__restrict__ logits, int32_t *__restrict__ ids, float *__restrict__ wts, int T, int E, int k,
     const uint16_t *__restrict__ x, int H, uint16_t *xq, float *xq_inv, const double *__restrict__ partial, int S,
-    const float *__restrict__ bias, int32_t *err_word, int debug)
+    const float *__restrict__ bias, int32_t *err_word, int debug, int32_t *seg_cnt)
 {
+    __shared__ int32_t ids_s[kTopkTokens * 32];
+    __shared__ int32_t cnt_s[256];
     if (xq) convert_x_blocks(x, T, H, xq, xq_inv);
-    const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    if (t >= T) return;
-    if (partial) {
-        for (int e = threadIdx.x & 31; e < E; e += 32) {
-            double v = 0.0;
-            for (int z = 0; z < S; ++z) v += partial[((size_t)z * T + t) * E + e];
-            float l = (float)v;
-            if (bias) l = l + bias[e];
-            if (debug && !isfinite(l)) atomicOr(err_word, DEV_ERR_NONFINITE);
-            logits[(size_t)t * E + e] = l;
+    if (seg_cnt)
+        for (int e = threadIdx.x; e < E; e += blockDim.x) cnt_s[e] = 0;
+    const int warp = threadIdx.x >> 5;
+    const int t = blockIdx.x * kTopkTokens + warp;
+    if (t < T) {
+        if (partial) {
+            for (int e = threadIdx.x & 31; e < E; e += 32) {
+                double v = 0.0;
+                for (int z = 0; z < S; ++z) v += partial[((size_t)z * T + t) * E + e];
+                float l = (float)v;
+                if (bias) l = l + bias[e];
+                if (debug && !isfinite(l)) atomicOr(err_word, DEV_ERR_NONFINITE);
+                logits[(size_t)t * E + e] = l;
+            }
+            __syncwarp();
         }
-        __syncwarp();
+        topk_warp(logits + (size_t)t * E, E, k, ids + (size_t)t * k, wts + (size_t)t * k, ids_s + warp * k);
     }
-    topk_warp(logits + (size_t)t * E, E, k, ids + (size_t)t * k, wts + (size_t)t * k);
+    if (!seg_cnt) return;
+    // this segment's expert histogram, for the multi-CTA plan
+    __syncthreads();
+    const int n = min(kTopkTokens, T - (int)blockIdx.x * kTopkTokens) * k;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) atomicAdd(&cnt_s[ids_s[i]], 1);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) seg_cnt[(size_t)blockIdx.x * E + e] = cnt_s[e];
 }
+
 
 // The expert plan, computed by one CTA of W warps. Pairs p = t*k + s are split
 // into W contiguous segments, one per warp. Pass 1 counts per (segment,
@@ -341,7 +358,6 @@ struct PlanArgs {
 
 __host__ __device__ constexpr size_t plan_smem_ints(int warps, int E) { return (size_t)warps * E + 2 * E + 1; }
 
-// ids: the pairs' expert ids, written by an earlier kernel (global) or by this CTA (shared).
 // Exclusive scan of tot[0..E) into off[0..E] by one warp (E <= 256: 8 experts per lane).
 __device__ __forceinline__ void scan_experts_warp(const int32_t *tot, int32_t *off, int E) {
     const int lane = threadIdx.x & 31;
@@ -368,6 +384,69 @@ __device__ __forceinline__ void scan_experts_warp(const int32_t *tot, int32_t *o
     if (lane == 31) off[E] = incl;
 }
 
+// Regime of every expert, the per-regime expert lists and the tensor-core token tiles,
+// from the per-expert totals and offsets; run by one warp.
+__device__ void plan_tail_warp(const int32_t *tot, const int32_t *off, const PlanArgs &pa)
+{
+    const int E = pa.E, lane = threadIdx.x & 31;
+    int n_gemv = 0, n_mma = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        const int m = (e < E) ? tot[e] : 0;
+        int reg = 0;
+        if (m > 0) {
+            if (pa.flags & TFMOE_FLAG_FORCE_GEMV) reg = 1;
+            else if (pa.flags & TFMOE_FLAG_FORCE_MMA) reg = 2;
+            else reg = (m <= pa.gemv_max_tokens) ? 1 : 2;
+        }
+        if (e < E) { pa.regime[e] = reg; pa.counts[e] = m; }
+        const uint32_t bg = __ballot_sync(0xffffffffu, reg == 1);
+        const uint32_t bm = __ballot_sync(0xffffffffu, reg == 2);
+        const uint32_t lt = (1u << lane) - 1u;
+        if (reg == 1) pa.gemv_list[n_gemv + __popc(bg & lt)] = e;
+        if (reg == 2) pa.mma_list[n_mma + __popc(bm & lt)] = e;
+        n_gemv += __popc(bg);
+        n_mma += __popc(bm);
+    }
+    if (lane == 0) { pa.list_sizes[0] = n_gemv; pa.list_sizes[1] = n_mma; }
+    // token tiles of the MMA-regime experts: ceil(m_e / pa.mma_tile) entries per
+    // expert, in expert order; lane l handles experts 8l .. 8l+7
+    int ntl[8], mine = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = lane * 8 + i;
+        int n = 0;
+        if (e < E) {
+            const int m = tot[e];
+            const bool mma = m > 0 && !(pa.flags & TFMOE_FLAG_FORCE_GEMV) &&
+                             ((pa.flags & TFMOE_FLAG_FORCE_MMA) || m > pa.gemv_max_tokens);
+            n = mma ? (m + pa.mma_tile - 1) / pa.mma_tile : 0;
+        }
+        ntl[i] = n;
+        mine += n;
+    }
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    int idx = incl - mine;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = lane * 8 + i;
+        for (int j = 0; j < ntl[i]; ++j, ++idx) {
+            int32_t *ent = pa.mma_entries + 4 * (size_t)idx;
+            ent[0] = e;
+            ent[1] = off[e] + j * pa.mma_tile;
+            ent[2] = min(pa.mma_tile, tot[e] - j * pa.mma_tile);
+            ent[3] = 0;
+        }
+    }
+    if (lane == 31) pa.list_sizes[2] = incl;
+}
+
+// ids: the pairs' expert ids, written by an earlier kernel (global) or by this CTA (shared).
 __device__ void plan_block(const int32_t *__restrict__ ids, int P, const PlanArgs &pa, int32_t *sm)
 {
     const int E = pa.E;
@@ -456,69 +535,86 @@ __device__ void plan_block(const int32_t *__restrict__ ids, int P, const PlanArg
             __syncwarp();
         }
     }
-    if (warp == 0) {
-        int n_gemv = 0, n_mma = 0;
-        for (int e0 = 0; e0 < E; e0 += 32) {
-            const int e = e0 + lane;
-            const int m = (e < E) ? tot[e] : 0;
-            int reg = 0;
-            if (m > 0) {
-                if (pa.flags & TFMOE_FLAG_FORCE_GEMV) reg = 1;
-                else if (pa.flags & TFMOE_FLAG_FORCE_MMA) reg = 2;
-                else reg = (m <= pa.gemv_max_tokens) ? 1 : 2;
-            }
-            if (e < E) { pa.regime[e] = reg; pa.counts[e] = m; }
-            const uint32_t bg = __ballot_sync(0xffffffffu, reg == 1);
-            const uint32_t bm = __ballot_sync(0xffffffffu, reg == 2);
-            const uint32_t lt = (1u << lane) - 1u;
-            if (reg == 1) pa.gemv_list[n_gemv + __popc(bg & lt)] = e;
-            if (reg == 2) pa.mma_list[n_mma + __popc(bm & lt)] = e;
-            n_gemv += __popc(bg);
-            n_mma += __popc(bm);
-        }
-        if (lane == 0) { pa.list_sizes[0] = n_gemv; pa.list_sizes[1] = n_mma; }
-        // token tiles of the MMA-regime experts: ceil(m_e / pa.mma_tile) entries per
-        // expert, in expert order; lane l handles experts 8l .. 8l+7
-        int ntl[8], mine = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int e = lane * 8 + i;
-            int n = 0;
-            if (e < E) {
-                const int m = tot[e];
-                const bool mma = m > 0 && !(pa.flags & TFMOE_FLAG_FORCE_GEMV) &&
-                                 ((pa.flags & TFMOE_FLAG_FORCE_MMA) || m > pa.gemv_max_tokens);
-                n = mma ? (m + pa.mma_tile - 1) / pa.mma_tile : 0;
-            }
-            ntl[i] = n;
-            mine += n;
-        }
-        int incl = mine;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        int idx = incl - mine;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int e = lane * 8 + i;
-            for (int j = 0; j < ntl[i]; ++j, ++idx) {
-                int32_t *ent = pa.mma_entries + 4 * (size_t)idx;
-                ent[0] = e;
-                ent[1] = off[e] + j * pa.mma_tile;
-                ent[2] = min(pa.mma_tile, tot[e] - j * pa.mma_tile);
-                ent[3] = 0;
-            }
-        }
-        if (lane == 31) pa.list_sizes[2] = incl;
-    }
+    if (warp == 0) plan_tail_warp(tot, off, pa);
 }
 
 __global__ void __launch_bounds__(1024) permute_kernel(const int32_t *__restrict__ ids, int P, PlanArgs pa)
 {
     extern __shared__ int32_t sm[];
     plan_block(ids, P, pa, sm);
+}
+
+// Multi-CTA plan, step 1 (large batches): CTA e scans expert e's counts over the segments
+// (exclusive prefix = the segment's first rank among the expert's rows) and stores the
+// total; the last CTA to arrive turns the totals into offsets and runs the plan's tail.
+__global__ void __launch_bounds__(256) plan_scan_kernel(const int32_t *__restrict__ seg_cnt, int nseg,
+                                                        int32_t *seg_base, int32_t *tot_g, int32_t *counter,
+                                                        PlanArgs pa)
+{
+    __shared__ int32_t wsum[8];
+    __shared__ int32_t tot[256], off[257];
+    __shared__ int is_last;
+    const int E = pa.E, e = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int carry = 0;
+    for (int s0 = 0; s0 < nseg; s0 += blockDim.x) {
+        const int sidx = s0 + threadIdx.x;
+        const int v = (sidx < nseg) ? seg_cnt[(size_t)sidx * E + e] : 0;
+        int incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
+        }
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        int before = 0, all = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+            if (w < warp) before += wsum[w];
+            all += wsum[w];
+        }
+        if (sidx < nseg) seg_base[(size_t)sidx * E + e] = carry + before + incl - v;
+        carry += all;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) tot_g[e] = carry;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = (atomicAdd(counter, 1) == (int)gridDim.x - 1);
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    for (int i = threadIdx.x; i < E; i += blockDim.x) tot[i] = __ldcg(tot_g + i);
+    __syncthreads();
+    if (warp == 0) scan_experts_warp(tot, off, E);
+    __syncthreads();
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) pa.offsets[i] = off[i];
+    if (warp == 0) plan_tail_warp(tot, off, pa);
+    if (threadIdx.x == 0) *counter = 0;
+}
+
+// Multi-CTA plan, step 2: CTA s places the pairs of segment s at the expert's offset plus
+// the segment's base plus the pair's rank among the segment's same-expert pairs, which
+// keeps the rows ordered by (expert, pair index).
+__global__ void __launch_bounds__(256) plan_place_kernel(const int32_t *__restrict__ ids, int P, int k,
+                                                         const int32_t *__restrict__ seg_base,
+                                                         const int32_t *__restrict__ offsets, int E,
+                                                         int32_t *__restrict__ perm, int32_t *__restrict__ inv)
+{
+    __shared__ int32_t ids_s[kTopkTokens * 32];
+    const int p0 = blockIdx.x * kTopkTokens * k;
+    const int n = min(kTopkTokens * k, P - p0);
+    for (int i = threadIdx.x; i < n; i += blockDim.x) ids_s[i] = ids[p0 + i];
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int e = ids_s[i];
+        if (e < 0 || e >= E) continue;
+        int rank = 0;
+        for (int q = 0; q < i; ++q) rank += (ids_s[q] == e);
+        const int r = offsets[e] + seg_base[(size_t)blockIdx.x * E + e] + rank;
+        perm[r] = p0 + i;
+        inv[p0 + i] = r;
+    }
 }
 
 // Decode-sized batches (T <= 16): router, top-k and plan in one launch.
@@ -608,6 +704,10 @@ static PlanArgs plan_args(const Layer &L, int T) {
 
 bool route_fused_applies(const Layer &L, int T) { return T <= kFusedMaxT; }
 
+static bool large_plan(const Layer &L, int T) {
+    return T > kFusedMaxT && (long long)T * L.desc.top_k > kLargePlanPairs;
+}
+
 cudaError_t launch_router(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches)
 {
     const int H = L.desc.hidden, E = L.desc.num_experts, k = L.desc.top_k;
@@ -645,8 +745,9 @@ cudaError_t launch_router(Layer &L, const uint16_t *x, int T, cudaStream_t s, in
     }
     {
         StageTimer timer(L, TFMOE_STAGE_TOPK, s);
-        topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(L.ws.logits, L.ws.ids, L.ws.topk_w, T, E, k, x, H, nullptr, nullptr,
-                                                  partial, S, bias, L.ws.err_word, debug);
+        topk_kernel<<<(T + kTopkTokens - 1) / kTopkTokens, 256, 0, s>>>(
+            L.ws.logits, L.ws.ids, L.ws.topk_w, T, E, k, x, H, nullptr, nullptr, partial, S, bias, L.ws.err_word, debug,
+            large_plan(L, T) ? L.ws.seg_cnt : nullptr);
     }
     *launches += 2;
     return cudaGetLastError();
@@ -657,6 +758,15 @@ cudaError_t launch_permute(Layer &L, int T, cudaStream_t s, int *launches)
     if (route_fused_applies(L, T)) return cudaSuccess;
     StageTimer timer(L, TFMOE_STAGE_PERMUTE, s);
     const int E = L.desc.num_experts, P = T * L.desc.top_k;
+    if (large_plan(L, T)) {
+        const int nseg = (T + kTopkTokens - 1) / kTopkTokens;
+        plan_scan_kernel<<<E, 256, 0, s>>>(L.ws.seg_cnt, nseg, L.ws.seg_base, L.ws.plan_tot, L.ws.plan_counter,
+                                           plan_args(L, T));
+        plan_place_kernel<<<nseg, 256, 0, s>>>(L.ws.ids, P, L.desc.top_k, L.ws.seg_base, L.ws.offsets, E, L.ws.perm,
+                                               L.ws.inv);
+        *launches += 2;
+        return cudaGetLastError();
+    }
     const size_t smem = sizeof(int32_t) * plan_smem_ints(32, E);
     permute_kernel<<<1, 1024, smem, s>>>(L.ws.ids, P, plan_args(L, T));
     *launches += 1;
@@ -739,7 +849,7 @@ extern "C" tfmoe_status tfmoe_route_noalloc(const uint16_t *x, int32_t T, int32_
         router_tiled_kernel<<<grid, 256, 0, s>>>(x, router_w, router_bias, logits, T, H, E, nullptr, 0);
     }
     topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(logits, ids_out, weights_out, T, E, k, x, H, nullptr, nullptr, nullptr,
-                                            1, nullptr, nullptr, 0);
+                                            1, nullptr, nullptr, 0, nullptr);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return record_error(TFMOE_ERR_CUDA, "tfmoe_route_noalloc: launch: %s", cudaGetErrorString(e));

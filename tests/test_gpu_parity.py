@@ -208,8 +208,13 @@ def _sampled_check(oracle_mod, run, layer, x, k, n_sample, seed):
     o = oracle_mod.forward(layer, x[idx], top_k=k, intermediates=True)
     assert np.array_equal(g["ids"][idx], o["ids"])
     assert np.array_equal(g["logits"][idx], o["logits"])
-    # every pair's row is where the permutation says, and the counts add up
-    assert g["counts"].sum() == T * k and np.array_equal(np.sort(g["perm"]), np.arange(T * k))
+    # the plan of the whole batch, from the GPU's own ids: rows ordered by (expert, pair index)
+    ids_all = g["ids"].ravel()
+    E = g["counts"].shape[0]
+    counts = np.bincount(ids_all, minlength=E)
+    assert np.array_equal(g["counts"], counts)
+    assert np.array_equal(g["offsets"], np.concatenate([[0], np.cumsum(counts)]))
+    assert np.array_equal(g["perm"], np.argsort(ids_all, kind="stable"))
     assert np.array_equal(g["inv"][g["perm"]], np.arange(T * k))
     return check_output(g["out"][idx], o)
 
@@ -233,5 +238,23 @@ def test_large_layer_sweep_sampled(oracle_mod):
         for T in s.T:
             x = synth.make_x(s, 6, T)
             _sampled_check(oracle_mod, run, layer, x, s.k, 8, T)
+    finally:
+        run.close()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("regime", ["auto", "gemv"])
+def test_large_batch_plan(oracle_mod, regime):
+    """More than 4096 (token, expert) pairs: the plan is built by the multi-CTA scan; 601
+    tokens leave a ragged last segment of one token."""
+    s = synth.custom_shape(H=256, I=128, E=64, k=8)
+    layer = synth.make_layer(s, 21)
+    x = synth.make_x(s, 21, 601)
+    run = GpuRun(layer, s.H, s.I, s.E, s.k, 601, flags=REGIMES[regime])
+    try:
+        g = run.forward(x, intermediates=True)
+        o = oracle_mod.forward(layer, x, top_k=s.k, intermediates=True)
+        check_routing(g, o, s.E, s.k)
+        check_output(g["out"], o)
     finally:
         run.close()
