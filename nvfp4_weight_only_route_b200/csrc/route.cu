@@ -226,6 +226,97 @@ __global__ void __launch_bounds__(256) router_split_kernel(
     }
 }
 
+// Layer path for larger batches on the fp64 tensor cores: mma.sync m8n8k4 f64 (each
+// product of two bf16 values is exact in fp64, sums accumulate in fp64 as in the scalar
+// kernel). CTA tile 64 tokens x 64 experts over a z-slice of the hidden dimension, staged
+// 32 columns at a time as fp64 in shared memory; warp (wm, wn) of 2 x 4 owns 32 tokens x
+// 16 experts = 4 x 2 tiles of 8 x 8. Output as router_split_kernel (fp32 logits + bias, or
+// fp64 partials [z][T][E]) and the same x conversion by the first expert-tile column.
+__device__ __forceinline__ void dmma_8x8x4(double &d0, double &d1, double a, double b) {
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                 : "+d"(d0), "+d"(d1) : "d"(a), "d"(b));
+}
+
+__global__ void __launch_bounds__(256) router_dmma_kernel(
+    const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, const float *__restrict__ bias,
+    float *__restrict__ logits, double *__restrict__ partial, int T, int H, int E, int k_len, int32_t *err_word,
+    int debug, uint16_t *xq, float *xq_inv)
+{
+    constexpr int TT = 64, TE = 64, KC = 32, LD = KC + 2;   // row stride in doubles
+    __shared__ double xs[TT * LD];
+    __shared__ double ws[TE * LD];
+    const int t_base = blockIdx.x * TT, e_base = blockIdx.y * TE, k_begin = blockIdx.z * k_len;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int wm = warp >> 2, wn = warp & 3;                 // 2 x 4 warps
+    const int g = lane >> 2, q = lane & 3;                   // fragment row group / thread in group
+    double acc[4][2][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
+    for (int k0 = k_begin; k0 < k_begin + k_len; k0 += KC) {
+        // 64 rows x 32 columns of x and of wr, 8 bf16 per item, converted to fp64
+        for (int i = threadIdx.x; i < TT * KC / 8; i += 256) {
+            const int row = i / (KC / 8), col = (i % (KC / 8)) * 8;
+            const int t = t_base + row, e = e_base + row;
+            uint4 xv = make_uint4(0, 0, 0, 0), wv = make_uint4(0, 0, 0, 0);
+            if (t < T) xv = *reinterpret_cast<const uint4 *>(x + (size_t)t * H + k0 + col);
+            if (e < E) wv = *reinterpret_cast<const uint4 *>(wr + (size_t)e * H + k0 + col);
+            const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w}, wu[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                xs[row * LD + col + 2 * j] = (double)bf16_bits_to_float(xu[j] & 0xFFFFu);
+                xs[row * LD + col + 2 * j + 1] = (double)bf16_bits_to_float(xu[j] >> 16);
+                ws[row * LD + col + 2 * j] = (double)bf16_bits_to_float(wu[j] & 0xFFFFu);
+                ws[row * LD + col + 2 * j + 1] = (double)bf16_bits_to_float(wu[j] >> 16);
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < KC; kk += 4) {
+            double a[4], b[2];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = xs[(wm * 32 + i * 8 + g) * LD + kk + q];      // A[token g][k q]
+#pragma unroll
+            for (int j = 0; j < 2; ++j) b[j] = ws[(wn * 16 + j * 8 + g) * LD + kk + q];      // B[k q][expert g]
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) dmma_8x8x4(acc[i][j][0], acc[i][j][1], a[i], b[j]);
+        }
+        __syncthreads();
+    }
+    // D[row g][col 2q + c] of each 8 x 8 tile
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int t = t_base + wm * 32 + i * 8 + g;
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const int e = e_base + wn * 16 + j * 8 + 2 * q + c;
+                if (e >= E) continue;
+                if (partial) {
+                    partial[((size_t)blockIdx.z * T + t) * E + e] = acc[i][j][c];
+                } else {
+                    float l = (float)acc[i][j][c];
+                    if (bias) l = l + bias[e];
+                    if (debug && !isfinite(l)) atomicOr(err_word, DEV_ERR_NONFINITE);
+                    logits[(size_t)t * E + e] = l;
+                }
+            }
+    }
+    if (xq && blockIdx.y == 0) {
+        const int rows = min(TT, T - t_base), blocks = k_len / 16;
+        for (int i = threadIdx.x; i < rows * blocks; i += blockDim.x) {
+            const int t = t_base + i / blocks;
+            const size_t off = (size_t)t * H + k_begin + (size_t)(i % blocks) * 16;
+            xq_inv[off / 16] = block16_bf16_to_f16(x + off, xq + off);
+        }
+    }
+}
+
 // One warp per token: k rounds of a warp arg-max over (logit desc, index asc),
 // then softmax over the selected logits (max-subtracted, fp32).
 constexpr int kMaxEPerLane = 8;   // E <= 256
@@ -626,6 +717,11 @@ __global__ void __launch_bounds__(256) plan_place_kernel(const int32_t *__restri
 // block is the launch-saving shape proposed in TensorFold issue #627 (comment
 // on the fused tf_nemo_route_row experiment).
 constexpr int kFusedMaxT = 16;
+#ifndef TFMOE_ROUTER_DMMA_MIN_TOKENS
+#define TFMOE_ROUTER_DMMA_MIN_TOKENS 128
+#endif
+// Batches of at least this many tokens take the router on the fp64 tensor cores.
+constexpr int kRouterDmmaMinTokens = TFMOE_ROUTER_DMMA_MIN_TOKENS;
 constexpr int kFusedThreads = 256;
 __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(
     const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, const float *__restrict__ bias,
@@ -725,7 +821,8 @@ cudaError_t launch_router(Layer &L, const uint16_t *x, int T, cudaStream_t s, in
         return cudaGetLastError();
     }
     // tile size and hidden-dimension slices: enough CTAs for two per SM where possible
-    const int M = (T >= 2048) ? 4 : 2, tile = 16 * M;
+    const bool dmma = T >= kRouterDmmaMinTokens;
+    const int M = (T >= 2048) ? 4 : 2, tile = dmma ? 64 : 16 * M;
     const int tiles = ((T + tile - 1) / tile) * ((E + tile - 1) / tile);
     int S = 1;
     if (tiles < 2 * L.num_sms) {
@@ -736,7 +833,10 @@ cudaError_t launch_router(Layer &L, const uint16_t *x, int T, cudaStream_t s, in
     {
         StageTimer timer(L, TFMOE_STAGE_ROUTER, s);
         dim3 grid((T + tile - 1) / tile, (E + tile - 1) / tile, S);
-        if (M == 4)
+        if (dmma)
+            router_dmma_kernel<<<grid, 256, 0, s>>>(x, L.w.router_w, bias, L.ws.logits, partial, T, H, E, H / S,
+                                                    L.ws.err_word, debug, gemv ? L.ws.xq : nullptr, L.ws.xq_inv);
+        else if (M == 4)
             router_split_kernel<4><<<grid, 256, 0, s>>>(x, L.w.router_w, bias, L.ws.logits, partial, T, H, E, H / S,
                                                         L.ws.err_word, debug, gemv ? L.ws.xq : nullptr, L.ws.xq_inv);
         else
