@@ -71,7 +71,7 @@ struct MmaCfg {
     static_assert(kBStageBytes % 1024 == 0, "token stages must stay 1 KB aligned");
 };
 using BigCfg = MmaCfg<kMmaTileTokens, 5, 5, 16, 2, 2, 1>;       // 640 threads, 512 TMEM columns
-using SmallCfg = MmaCfg<kMmaSmallTileTokens, 3, 4, 12, 1, 1, 2>; // 384 threads, 256 TMEM columns
+using SmallCfg = MmaCfg<kMmaSmallTileTokens, 3, 4, 12, 2, 1, 2>; // 512 threads, 256 TMEM columns
 
 template <class C>
 struct MmaSmem {
