@@ -74,6 +74,13 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
         : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs) : "memory");
     return ok != 0;
 }
+// Programmatic dependent launch. A grid launched with programmatic stream
+// serialisation may start once every CTA of the grid before it has called
+// launch_dependents (or exited); grid_dep_wait returns when that grid has completed
+// and its memory is visible. Both are no-ops for a grid launched normally.
+__device__ __forceinline__ void grid_dep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Bounded wait: returns false (and sets the error word) when the limit passes.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, int32_t *err_word) {
     if (mbar_try_wait(bar, parity)) return true;

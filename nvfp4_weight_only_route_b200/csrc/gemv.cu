@@ -53,6 +53,9 @@ constexpr int kCtasPerSm = TFMOE_GEMV_CTAS_PER_SM;
 #ifndef TFMOE_GEMV_CHUNK
 #define TFMOE_GEMV_CHUNK 4
 #endif
+#ifndef TFMOE_GEMV_DOWN_EARLY
+#define TFMOE_GEMV_DOWN_EARLY 1
+#endif
 constexpr int kChunk = TFMOE_GEMV_CHUNK;   // column tiles per ring slot of a compute warp
 constexpr int kRing = TFMOE_GEMV_RING;   // ring slots per compute warp (kRing - 1 chunks in flight)
 static_assert(kRing >= 2, "ring depth");
@@ -243,6 +246,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     const int RT = a.R / kTileRows, tpe = a.R / rows_task;
     const int n_list = __ldg(a.list_size);
     const int n_tasks = n_list * tpe;
+    // The down launch depends on this grid programmatically: its CTAs may take the
+    // slots of gate/up CTAs that finished and fetch weights while the rest still run.
+    if (P == Proj::GateUp) grid_dep_launch_dependents();
     if ((int)blockIdx.x >= n_tasks) return;
 
     const SmemLayout lay(K, KS, RG);
@@ -301,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
         const uint32_t scale_tx = (uint32_t)(KT * rows_task * 4);
         int last_s = -1, last_x = -1;                 // barriers of the latest copies issued
         uint32_t last_s_par = 0, last_x_par = 0;
-        auto issue = [&](int task, int t0, int tn, int p) {
+        auto issue = [&](int task, int t0, int tn, int p, bool first) {
             int r_begin;
             const int m = task_rows(task, r_begin);
             const int nt = min(kMaxNT, m - t0);
@@ -320,6 +326,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
                     last_s = sb;
                     last_s_par = (tn >> 1) & 1;
                 }
+            }
+            // the down pass reads aq, which the gate/up grid writes: wait for that grid here,
+            // after the first scale copy and before the first activation copy
+            if (P == Proj::Down && first) {
+                __syncwarp();
+                grid_dep_wait();
+            }
+            if (lane == 0) {
                 mbar_arrive_expect_tx(&xfull[xb], (uint32_t)nt * (uint32_t)(K * 2 + K / 4));
                 last_x = xb;
                 last_x_par = (p >> 1) & 1;
@@ -335,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
         };
         int ftask;
         if (first_pass(ftask)) {
-            issue(ftask, 0, 0, 0);
+            issue(ftask, 0, 0, 0, true);
             int p = 0, tn = 0;
             for (int task = ftask; task < n_tasks; task += gridDim.x) {
                 int r_begin;
@@ -346,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
                     const int nt = min(kMaxNT, m - t0);
                     int ntask, nt0;
                     // the buffers of pass p+1 were last read in pass p-1, whose sums were consumed below
-                    if (next_pass(task, t0, m, ntask, nt0)) issue(ntask, nt0, ntask == task ? tn : tn + 1, p + 1);
+                    if (next_pass(task, t0, m, ntask, nt0)) issue(ntask, nt0, ntask == task ? tn : tn + 1, p + 1, false);
                     wait_or_abort(&full[p & 1], (p >> 1) & 1, abort_flag, a.err_word);
                     const float *rb = red(p & 1);
                     if (P == Proj::GateUp) {
@@ -446,6 +460,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
         slot_fill = (slot_fill + 1 == kRing) ? 0 : slot_fill + 1;
     };
     for (int i = 0; i < kRing - 1; ++i) refill();
+    // weights only so far; the bounded waits below start after the gate/up grid is done
+    if (P == Proj::Down && ptask >= 0) grid_dep_wait();
 
     int slot_use = 0;
     int p = 0, tn = 0;
@@ -573,9 +589,19 @@ cudaError_t launch_gemv_down(Layer &L, cudaStream_t s, int *launches)
     d.KS = gm->g_down.KS; d.RG = gm->g_down.RG;
     d.src = L.ws.aq; d.src_inv = L.ws.aq_inv;
     d.y_out = L.ws.y;
-    gemv_kernel<Proj::Down><<<L.gemv_grid_down, kThreads, gemv_smem_bytes(d.K, gm->g_down), s>>>(gm->down, d);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(L.gemv_grid_down);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = gemv_smem_bytes(d.K, gm->g_down);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = TFMOE_GEMV_DOWN_EARLY;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_kernel<Proj::Down>, gm->down, d);
     *launches += 1;
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_gemv(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches)
