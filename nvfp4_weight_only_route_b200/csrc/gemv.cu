@@ -126,8 +126,31 @@ size_t gemv_smem_bytes(int K, Geometry g) { return 128 + SmemLayout(K, g.KS, g.R
 
 // 16-byte asynchronous copy global -> shared (cp.async, bypassing L1): the code stream
 // stays 128-bit coalesced loads while the data waits in shared memory, not registers.
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+__device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void *gmem_src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(gmem_src) : "memory");
+}
+// Shared-memory loads by 32-bit address: the inner loop's addresses are a few
+// per-pass bases plus constant offsets, with no generic-pointer arithmetic.
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float2 lds64f(uint32_t a) {
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+// The E4M3 pair in bits [sh, sh + 16) of w -> two floats (exact).
+__device__ __forceinline__ float2 e4m3_pair_at(uint32_t w, uint32_t sh) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}" : "=r"(h2) : "r"(w >> sh));
+    return f16x2_to_float2(h2);
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -142,23 +165,25 @@ __device__ __forceinline__ float fma2_f16_f32(uint32_t w2, uint32_t x2, float ac
     return acc;
 }
 
-// One lane's share of n <= kChunk column tiles for NT tokens. cs points at the lane's
-// 16 code bytes of the chunk's first tile in its ring slot (tiles 32 x 16 bytes apart);
-// tile0 indexes that tile inside the warp's slice; xs / xis point (in shared memory) at
-// token 0's activation values / inverse scales at the slice's first tile and the lane's
-// half; token t's row starts K values (K/16 inverse scales) further on.
+// One lane's share of n <= kChunk column tiles for NT tokens, all operands in shared
+// memory addressed by 32-bit bases:
+//   cs  the lane's 16 code bytes of the chunk's first tile (tiles 512 bytes apart);
+//   sc  the lane's 4 scale bytes of that tile (tiles sc_step bytes apart; the lane's
+//       half takes bits [hsh, hsh + 16));
+//   xa  token 0's 32 activation values of the lane's half of that tile (tiles 128
+//       bytes apart, tokens x_tok bytes apart); xia their two inverse scales (tiles
+//       16 bytes apart, tokens xi_tok bytes apart).
 template <int NT>
-__device__ __forceinline__ void chunk_compute(const uint4 *cs, int n, int tile0, const uint32_t *sc, int rows_task,
-                                              int h, const uint16_t *xs, const float *xis, int K,
+__device__ __forceinline__ void chunk_compute(uint32_t cs, int n, uint32_t sc, uint32_t sc_step, uint32_t hsh,
+                                              uint32_t xa, uint32_t xia, uint32_t x_tok, uint32_t xi_tok,
                                               float (&acc)[kMaxNT])
 {
 #pragma unroll
     for (int j = 0; j < kChunk; ++j) {
         if (j >= n) break;
-        const int tw = tile0 + j;
-        const uint32_t s4 = sc[tw * rows_task];
-        const float2 s = f16x2_to_float2(e4m3x2_to_f16x2(h ? (s4 >> 16) : (s4 & 0xFFFFu)));
-        const uint4 cw = cs[j * 32];
+        const float2 s = e4m3_pair_at(lds32(sc), hsh);
+        sc += sc_step;
+        const uint4 cw = lds128(cs + j * 512);
         const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
         float p[NT][2];
 #pragma unroll
@@ -170,7 +195,7 @@ __device__ __forceinline__ void chunk_compute(const uint4 *cs, int n, int tile0,
             e2m1x8_to_f16x2x4(words[q], wp);
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
-                const uint4 xv = *(reinterpret_cast<const uint4 *>(xs + t * K + tw * kTileK) + q);
+                const uint4 xv = lds128(xa + t * x_tok + j * 128 + q * 16);
                 float &pp = p[t][q >> 1];
                 pp = fma2_f16_f32(wp[0], xv.x, pp);
                 pp = fma2_f16_f32(wp[1], xv.y, pp);
@@ -180,7 +205,7 @@ __device__ __forceinline__ void chunk_compute(const uint4 *cs, int n, int tile0,
         }
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-            const float2 inv = *reinterpret_cast<const float2 *>(xis + t * (K / 16) + tw * (kTileK / 16));
+            const float2 inv = lds64f(xia + t * xi_tok + j * 16);
             acc[t] = fmaf(p[t][0], s.x * inv.x, acc[t]);
             acc[t] = fmaf(p[t][1], s.y * inv.y, acc[t]);
         }
@@ -190,17 +215,20 @@ __device__ __forceinline__ void chunk_compute(const uint4 *cs, int n, int tile0,
 // All column chunks of one pass: wait for the lane's oldest copies, compute, and let
 // `refill` put the next chunk of the stream into the slot freed by the previous one.
 template <int NT, class Refill>
-__device__ __forceinline__ void pass_run(const uint4 *ring, int &slot_use, int KTW, const uint32_t *sc, int rows_task,
-                                         int h, const uint16_t *xs, const float *xis, int K, float (&acc)[kMaxNT],
-                                         Refill &refill)
+__device__ __forceinline__ void pass_run(uint32_t ring, int &slot_use, int KTW, uint32_t sc, uint32_t sc_step,
+                                         uint32_t hsh, uint32_t xa, uint32_t xia, uint32_t x_tok, uint32_t xi_tok,
+                                         float (&acc)[kMaxNT], Refill &refill)
 {
     const int nch = (KTW + kChunk - 1) / kChunk;
     for (int ch = 0; ch < nch; ++ch) {
         cp_async_wait<kRing - 2>();
-        chunk_compute<NT>(ring + (size_t)slot_use * kChunk * 32, min(kChunk, KTW - ch * kChunk), ch * kChunk, sc,
-                          rows_task, h, xs, xis, K, acc);
+        chunk_compute<NT>(ring + (uint32_t)slot_use * (kChunk * 512), min(kChunk, KTW - ch * kChunk), sc, sc_step, hsh,
+                          xa, xia, x_tok, xi_tok, acc);
         refill();
         slot_use = (slot_use + 1 == kRing) ? 0 : slot_use + 1;
+        sc += kChunk * sc_step;
+        xa += kChunk * 128;
+        xia += kChunk * 16;
     }
 }
 
@@ -426,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     // The warp's code stream: the (task, pass, chunk) sequence it consumes, kRing - 1
     // chunks ahead. Each lane copies and later reads only its own 16-byte pieces, so a
     // lane's cp.async.wait_group is all the synchronisation the ring needs.
-    const uint4 *ring = reinterpret_cast<const uint4 *>(base + lay.ring) + (size_t)warp * kRing * kChunk * 32 + lane;
+    const uint32_t ring = smem_u32(base + lay.ring) + (uint32_t)(warp * kRing * kChunk * 32 + lane) * 16u;
     const int nch = (KTW + kChunk - 1) / kChunk;
     int ptask = -1, pt0 = 0, pch = 0, slot_fill = 0;
     const uint8_t *pg = nullptr;                          // next chunk of the stream (this lane's bytes)
@@ -437,10 +465,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     auto refill = [&]() {
         if (ptask >= 0) {
             const int n = min(kChunk, KTW - pch * kChunk);
-            uint4 *d = const_cast<uint4 *>(ring) + (size_t)slot_fill * kChunk * 32;
+            const uint32_t d = ring + (uint32_t)slot_fill * (kChunk * 512);
 #pragma unroll
             for (int j = 0; j < kChunk; ++j)
-                if (j < n) cp_async16(d + j * 32, pg + (size_t)j * kTileCodeBytes);
+                if (j < n) cp_async16(d + j * 512, pg + (size_t)j * kTileCodeBytes);
             pg += (size_t)kChunk * kTileCodeBytes;
             if (++pch == nch) {
                 pch = 0;
@@ -465,25 +493,29 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
 
     int slot_use = 0;
     int p = 0, tn = 0;
+    const uint32_t sc_step = (uint32_t)rows_task * 4u, hsh = (uint32_t)h * 16u;
+    const uint32_t x_tok = (uint32_t)K * 2u, xi_tok = (uint32_t)(K / 16) * 4u;
     for (int task = blockIdx.x; task < n_tasks; task += gridDim.x) {
         int r_begin;
         const int m = task_rows(task, r_begin);
         if (m <= 0) continue;
         const int sb = tn & 1;
-        const uint32_t *sc = sbuf(sb) + (size_t)(ks * KTW) * rows_task + lrow;
+        const uint32_t sc = smem_u32(sbuf(sb)) + (uint32_t)((ks * KTW) * rows_task + lrow) * 4u;
         wait_or_abort(&sfull[sb], (tn >> 1) & 1, abort_flag, a.err_word);
         for (int t0 = 0; t0 < m; t0 += kMaxNT, ++p) {
             const int nt = min(kMaxNT, m - t0);
             const int xb = p & 1;
             wait_or_abort(&xfull[xb], (p >> 1) & 1, abort_flag, a.err_word);
-            const uint16_t *xs = xbuf(xb) + col0;
-            const float *xis = xibuf(xb) + col0 / 16;
+            const uint32_t xa = smem_u32(xbuf(xb)) + (uint32_t)col0 * 2u;
+            const uint32_t xia = smem_u32(xibuf(xb)) + (uint32_t)(col0 / 16) * 4u;
             float acc[kMaxNT] = {};
             switch (nt) {
-            case 1: pass_run<1>(ring, slot_use, KTW, sc, rows_task, h, xs, xis, K, acc, refill); break;
-            case 2: pass_run<2>(ring, slot_use, KTW, sc, rows_task, h, xs, xis, K, acc, refill); break;
-            case 3: pass_run<(kMaxNT > 2 ? 3 : 2)>(ring, slot_use, KTW, sc, rows_task, h, xs, xis, K, acc, refill); break;
-            default: pass_run<kMaxNT>(ring, slot_use, KTW, sc, rows_task, h, xs, xis, K, acc, refill); break;
+            case 1: pass_run<1>(ring, slot_use, KTW, sc, sc_step, hsh, xa, xia, x_tok, xi_tok, acc, refill); break;
+            case 2: pass_run<2>(ring, slot_use, KTW, sc, sc_step, hsh, xa, xia, x_tok, xi_tok, acc, refill); break;
+            case 3:
+                pass_run<(kMaxNT > 2 ? 3 : 2)>(ring, slot_use, KTW, sc, sc_step, hsh, xa, xia, x_tok, xi_tok, acc, refill);
+                break;
+            default: pass_run<kMaxNT>(ring, slot_use, KTW, sc, sc_step, hsh, xa, xia, x_tok, xi_tok, acc, refill); break;
             }
 #pragma unroll
             for (int t = 0; t < kMaxNT; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 16);
