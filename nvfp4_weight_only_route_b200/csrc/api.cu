@@ -277,9 +277,9 @@ tfmoe_status tfmoe_forward(tfmoe_layer *layer, const uint16_t *x, int32_t T, uin
     if (e == cudaSuccess) e = launch_permute(L, T, s, &n);
     if (e == cudaSuccess && use_mma) e = launch_gather(L, x, T, s, &n);
     if (e == cudaSuccess && use_mma) e = launch_mma_gate_up(L, s, &n);
-    if (e == cudaSuccess && use_gemv) e = launch_gemv_gate_up(L, x, s, &n);
+    if (e == cudaSuccess && use_gemv) e = launch_gemv_gate_up(L, x, T, s, &n);
     if (e == cudaSuccess && use_mma) e = launch_mma_down(L, s, &n);
-    if (e == cudaSuccess && use_gemv) e = launch_gemv_down(L, s, &n);
+    if (e == cudaSuccess && use_gemv) e = launch_gemv_down(L, T, s, &n);
     if (e == cudaSuccess) e = launch_combine(L, T, out, s, &n);
     L.last_use_mma = use_mma;
     L.last_use_gemv = use_gemv;
@@ -397,10 +397,10 @@ tfmoe_status tfmoe_forward_stage(tfmoe_layer *layer, int32_t stage, const uint16
     switch (stage) {
     case TFMOE_STAGE_GEMV_GATE_UP:
         if (!x) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward_stage: x is NULL");
-        if (L.last_use_gemv) e = launch_gemv_gate_up(L, x, s, &n);
+        if (L.last_use_gemv) e = launch_gemv_gate_up(L, x, T, s, &n);
         break;
     case TFMOE_STAGE_GEMV_DOWN:
-        if (L.last_use_gemv) e = launch_gemv_down(L, s, &n);
+        if (L.last_use_gemv) e = launch_gemv_down(L, T, s, &n);
         break;
     case TFMOE_STAGE_GATHER:
         if (!x) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward_stage: x is NULL");

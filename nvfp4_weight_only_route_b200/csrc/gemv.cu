@@ -29,6 +29,7 @@
 // one mixed-precision fma.rn.f32.f16, so a 16-element partial sum is an fp32
 // sum of exact products; it is scaled by (E4M3 block scale * inverse power of
 // two of the activation block, an exact product) into the fp32 row accumulator.
+#include <algorithm>
 #include <new>
 
 #include "common.cuh"
@@ -64,6 +65,11 @@ static_assert(kMaxNT == 2 || kMaxNT == 4, "tokens per pass");
 
 enum class Proj { GateUp, Down };
 
+// A GEMV task: id = li * tpe + sub (entry li of the GEMV list, row group sub).
+struct Cursor {
+    int id, li, sub;
+};
+
 struct GemvArgs {
     const uint8_t *codes;       // tiled codes of all experts
     const float *glob0;         // gate (GateUp) or down (Down) per-tensor scale [E]
@@ -91,6 +97,22 @@ struct Geometry {
 
 // Gate/up tasks hold at least two 16-row groups (32 interleaved rows = 16 SwiGLU
 // outputs = one 16-element block of a). KT = K / 64 is even there (H % 128 == 0).
+// Each projection has two task shapes: the default one (more, shorter tasks) and a
+// long one (each warp streams more column tiles per pass, so the per-pass costs are
+// spread over more weights), used when the batch gives every CTA enough tasks.
+#ifndef TFMOE_GEMV_GU_LONG_KS
+#define TFMOE_GEMV_GU_LONG_KS 4
+#endif
+#ifndef TFMOE_GEMV_DOWN_LONG_KS
+#define TFMOE_GEMV_DOWN_LONG_KS 2
+#endif
+constexpr int kLongTasksPerCta = 4;   // the long shape needs this many tasks per CTA (estimated)
+Geometry geometry_from(int ks_start, int K) {
+    const int KT = K / kTileK;
+    int KS = ks_start;
+    while (KT % KS) KS >>= 1;
+    return {KS, kWarps / KS};
+}
 Geometry geometry(bool gate_up, int K) {
     const int KT = K / kTileK;
     int KS = gate_up ? 4 : 8;
@@ -271,6 +293,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     const int K = a.K, KT = K / kTileK, KS = a.KS, RG = a.RG;
     const int rows_task = 16 * RG, KTW = KT / KS;
+    const int rt_log2 = 31 - __clz(rows_task);            // rows_task is a power of two
     const int RT = a.R / kTileRows, tpe = a.R / rows_task;
     const int n_list = __ldg(a.list_size);
     const int n_tasks = n_list * tpe;
@@ -310,24 +333,34 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     }
     __syncthreads();
 
-    auto task_expert = [&](int task) { return tab[task / tpe]; };
-    auto task_rows = [&](int task, int &r_begin) {
-        r_begin = tab[n_list + task / tpe];
-        return tab[2 * n_list + task / tpe];
+    // The CTA's tasks are blockIdx.x + i * gridDim.x. A cursor carries a task's list
+    // entry (li = task / tpe) and row group (sub = task % tpe) and steps without dividing.
+    const int g_li = (int)gridDim.x / tpe, g_sub = (int)gridDim.x % tpe;
+    const Cursor c0{(int)blockIdx.x, (int)blockIdx.x / tpe, (int)blockIdx.x % tpe};
+    auto advance = [&](Cursor &c) {
+        c.id += gridDim.x;
+        c.li += g_li;
+        c.sub += g_sub;
+        if (c.sub >= tpe) { c.sub -= tpe; ++c.li; }
     };
-    // the pass after (task, t0) in this CTA's sequence; tasks without rows have no pass
-    auto next_pass = [&](int task, int t0, int m, int &ntask, int &nt0) {
-        if (t0 + kMaxNT < m) { ntask = task; nt0 = t0 + kMaxNT; return true; }
-        for (int tk = task + (int)gridDim.x; tk < n_tasks; tk += gridDim.x) {
+    auto task_rows = [&](const Cursor &c, int &r_begin) {
+        r_begin = tab[n_list + c.li];
+        return tab[2 * n_list + c.li];
+    };
+    // the pass after (task c, t0) in this CTA's sequence; tasks without rows have no pass
+    auto next_pass = [&](const Cursor &c, int t0, int m, Cursor &nc, int &nt0) {
+        if (t0 + kMaxNT < m) { nc = c; nt0 = t0 + kMaxNT; return true; }
+        Cursor k = c;
+        for (advance(k); k.id < n_tasks; advance(k)) {
             int rb;
-            if (task_rows(tk, rb) > 0) { ntask = tk; nt0 = 0; return true; }
+            if (task_rows(k, rb) > 0) { nc = k; nt0 = 0; return true; }
         }
         return false;
     };
-    auto first_pass = [&](int &ftask) {
+    auto first_pass = [&](Cursor &fc) {
         int rb, t0;
-        if (task_rows(blockIdx.x, rb) > 0) { ftask = blockIdx.x; return true; }
-        return next_pass(blockIdx.x, 0, 0, ftask, t0);
+        if (task_rows(c0, rb) > 0) { fc = c0; return true; }
+        return next_pass(c0, 0, 0, fc, t0);
     };
 
     if (warp == kComputeWarps) {
@@ -335,9 +368,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
         const uint32_t scale_tx = (uint32_t)(KT * rows_task * 4);
         int last_s = -1, last_x = -1;                 // barriers of the latest copies issued
         uint32_t last_s_par = 0, last_x_par = 0;
-        auto issue = [&](int task, int t0, int tn, int p, bool first) {
+        auto issue = [&](const Cursor &c, int t0, int tn, int p, bool first) {
             int r_begin;
-            const int m = task_rows(task, r_begin);
+            const int m = task_rows(c, r_begin);
             const int nt = min(kMaxNT, m - t0);
             int row = 0;
             if (lane < nt) {
@@ -347,9 +380,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
             const int xb = p & 1;
             if (lane == 0) {
                 if (t0 == 0) {
-                    const int sb = tn & 1, row0 = (task % tpe) * rows_task;
+                    const int sb = tn & 1, row0 = c.sub * rows_task;
                     mbar_arrive_expect_tx(&sfull[sb], scale_tx);
-                    tma_load_2d(sbuf(sb), &smap, row0 % kTileRows, (task_expert(task) * RT + row0 / kTileRows) * KT,
+                    tma_load_2d(sbuf(sb), &smap, row0 % kTileRows, (tab[c.li] * RT + row0 / kTileRows) * KT,
                                 &sfull[sb]);
                     last_s = sb;
                     last_s_par = (tn >> 1) & 1;
@@ -375,27 +408,28 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
                 }
             }
         };
-        int ftask;
-        if (first_pass(ftask)) {
-            issue(ftask, 0, 0, 0, true);
+        Cursor fc;
+        if (first_pass(fc)) {
+            issue(fc, 0, 0, 0, true);
             int p = 0, tn = 0;
-            for (int task = ftask; task < n_tasks; task += gridDim.x) {
+            for (Cursor c = fc; c.id < n_tasks; advance(c)) {
                 int r_begin;
-                const int m = task_rows(task, r_begin);
+                const int m = task_rows(c, r_begin);
                 if (m <= 0) continue;
-                const int e = task_expert(task), row0 = (task % tpe) * rows_task;
+                const int e = tab[c.li], row0 = c.sub * rows_task;
                 for (int t0 = 0; t0 < m; t0 += kMaxNT, ++p) {
                     const int nt = min(kMaxNT, m - t0);
-                    int ntask, nt0;
+                    Cursor nc;
+                    int nt0;
                     // the buffers of pass p+1 were last read in pass p-1, whose sums were consumed below
-                    if (next_pass(task, t0, m, ntask, nt0)) issue(ntask, nt0, ntask == task ? tn : tn + 1, p + 1, false);
+                    if (next_pass(c, t0, m, nc, nt0)) issue(nc, nt0, nc.id == c.id ? tn : tn + 1, p + 1, false);
                     wait_or_abort(&full[p & 1], (p >> 1) & 1, abort_flag, a.err_word);
                     const float *rb = red(p & 1);
                     if (P == Proj::GateUp) {
                         // rows_task is a multiple of 32: a round covers 32 rows (16 gate/up pairs) of one token
                         const float g0 = __ldg(a.glob0 + e), g1 = __ldg(a.glob1 + e);
                         for (int i0 = 0; i0 < rows_task * nt; i0 += 32) {
-                            const int i = i0 + lane, t = i / rows_task, rl = i % rows_task;
+                            const int i = i0 + lane, t = i >> rt_log2, rl = i & (rows_task - 1);
                             float v = 0.f;
                             for (int s = 0; s < KS; ++s) v += rb[((size_t)s * rows_task + rl) * kMaxNT + t];
                             const int grow = row0 + rl;
@@ -421,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
                     } else {
                         const float gs = __ldg(a.glob0 + e);
                         for (int i = lane; i < rows_task * nt; i += 32) {
-                            const int t = i / rows_task, rl = i % rows_task;
+                            const int t = i >> rt_log2, rl = i & (rows_task - 1);
                             float v = 0.f;
                             for (int s = 0; s < KS; ++s) v += rb[((size_t)s * rows_task + rl) * kMaxNT + t];
                             a.y_out[(size_t)(r_begin + t0 + t) * a.R + row0 + rl] = v * gs;
@@ -446,9 +480,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     const int h = lane >> 4;
     const int lrow = rgl * 16 + (lane & 15);              // row of the lane inside the task
     const int col0 = ks * KTW * kTileK + h * 32;          // first column of the lane's slice and half
-    auto lane_codes = [&](int task) -> const uint8_t * {
-        const int row0 = (task % tpe) * rows_task;
-        return a.codes + ((size_t)(task_expert(task) * RT + row0 / kTileRows) * KT + (size_t)ks * KTW) *
+    auto lane_codes = [&](const Cursor &c) -> const uint8_t * {
+        const int row0 = c.sub * rows_task;
+        return a.codes + ((size_t)(tab[c.li] * RT + row0 / kTileRows) * KT + (size_t)ks * KTW) *
                    kTileCodeBytes + h * 2048 + (row0 % kTileRows + lrow) * 16;
     };
     // The warp's code stream: the (task, pass, chunk) sequence it consumes, kRing - 1
@@ -456,14 +490,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     // lane's cp.async.wait_group is all the synchronisation the ring needs.
     const uint32_t ring = smem_u32(base + lay.ring) + (uint32_t)(warp * kRing * kChunk * 32 + lane) * 16u;
     const int nch = (KTW + kChunk - 1) / kChunk;
-    int ptask = -1, pt0 = 0, pch = 0, slot_fill = 0;
+    Cursor pc{};                                          // task of the next chunk of the stream
+    bool pvalid = false;
+    int pt0 = 0, pch = 0, slot_fill = 0;
     const uint8_t *pg = nullptr;                          // next chunk of the stream (this lane's bytes)
     {
-        int ft;
-        if (first_pass(ft)) { ptask = ft; pg = lane_codes(ft); }
+        Cursor ft;
+        if (first_pass(ft)) { pc = ft; pvalid = true; pg = lane_codes(ft); }
     }
     auto refill = [&]() {
-        if (ptask >= 0) {
+        if (pvalid) {
             const int n = min(kChunk, KTW - pch * kChunk);
             const uint32_t d = ring + (uint32_t)slot_fill * (kChunk * 512);
 #pragma unroll
@@ -472,15 +508,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
             pg += (size_t)kChunk * kTileCodeBytes;
             if (++pch == nch) {
                 pch = 0;
-                int rb, ntask, nt0;
-                const int m = task_rows(ptask, rb);
-                if (next_pass(ptask, pt0, m, ntask, nt0)) {
-                    if (ntask != ptask) pg = lane_codes(ntask);
+                int rb, nt0;
+                Cursor nc;
+                const int m = task_rows(pc, rb);
+                if (next_pass(pc, pt0, m, nc, nt0)) {
+                    if (nc.id != pc.id) pg = lane_codes(nc);
                     else pg -= (size_t)nch * kChunk * kTileCodeBytes;   // same task, next tokens
-                    ptask = ntask;
+                    pc = nc;
                     pt0 = nt0;
                 } else {
-                    ptask = -1;
+                    pvalid = false;
                 }
             }
         }
@@ -489,15 +526,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     };
     for (int i = 0; i < kRing - 1; ++i) refill();
     // weights only so far; the bounded waits below start after the gate/up grid is done
-    if (P == Proj::Down && ptask >= 0) grid_dep_wait();
+    if (P == Proj::Down && pvalid) grid_dep_wait();
 
     int slot_use = 0;
     int p = 0, tn = 0;
     const uint32_t sc_step = (uint32_t)rows_task * 4u, hsh = (uint32_t)h * 16u;
     const uint32_t x_tok = (uint32_t)K * 2u, xi_tok = (uint32_t)(K / 16) * 4u;
-    for (int task = blockIdx.x; task < n_tasks; task += gridDim.x) {
+    for (Cursor c = c0; c.id < n_tasks; advance(c)) {
         int r_begin;
-        const int m = task_rows(task, r_begin);
+        const int m = task_rows(c, r_begin);
         if (m <= 0) continue;
         const int sb = tn & 1;
         const uint32_t sc = smem_u32(sbuf(sb)) + (uint32_t)((ks * KTW) * rows_task + lrow) * 4u;
@@ -543,10 +580,23 @@ int gemv_grid(int K, Geometry g, int num_sms) {
     return per_sm * num_sms;
 }
 
-struct GemvMaps {
-    CUtensorMap gu, down;
-    Geometry g_gu, g_down;
+struct GemvShape {
+    CUtensorMap map;   // the scales, box = one task's rows x all column tiles
+    Geometry g;
+    int grid;
+    size_t smem;
 };
+struct GemvMaps {
+    GemvShape gu[2], down[2];   // [0] default, [1] long
+};
+
+// The shape for a batch of T tokens: long when the GEMV list (at most min(E, T k)
+// experts) gives each CTA kLongTasksPerCta long tasks.
+const GemvShape &pick_shape(const Layer &L, const GemvShape (&sh)[2], int R, int T) {
+    const int experts = min(L.desc.num_experts, T * L.desc.top_k);
+    const long long tasks = (long long)experts * (R / (16 * sh[1].g.RG));
+    return (sh[1].g.KS != sh[0].g.KS && tasks >= (long long)kLongTasksPerCta * sh[1].grid) ? sh[1] : sh[0];
+}
 
 }  // namespace
 
@@ -555,27 +605,37 @@ cudaError_t gemv_setup(Layer &L)
     const int H = L.desc.hidden, I = L.desc.intermediate, E = L.desc.num_experts;
     GemvMaps *gm = new (std::nothrow) GemvMaps();
     if (!gm) return cudaErrorMemoryAllocation;
-    gm->g_gu = geometry(true, H);
-    gm->g_down = geometry(false, I);
+    gm->gu[0].g = geometry(true, H);
+    gm->gu[1].g = geometry_from(TFMOE_GEMV_GU_LONG_KS, H);
+    gm->down[0].g = geometry(false, I);
+    gm->down[1].g = geometry_from(TFMOE_GEMV_DOWN_LONG_KS, I);
     // scale slabs viewed as [E * RT * KT][128 rows] of u32; a task's box is 16*RG rows x all KT slabs
     const uint64_t slabs_gu = (uint64_t)E * (2 * I / kTileRows) * (H / kTileK);
     const uint64_t slabs_d = (uint64_t)E * (H / kTileRows) * (I / kTileK);
-    if (encode_tensor_map_2d(&gm->gu, CU_TENSOR_MAP_DATA_TYPE_UINT32, L.w.gu_scales, kTileRows, slabs_gu,
-                             kTileScaleBytes, 16 * gm->g_gu.RG, H / kTileK, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
-        encode_tensor_map_2d(&gm->down, CU_TENSOR_MAP_DATA_TYPE_UINT32, L.w.d_scales, kTileRows, slabs_d,
-                             kTileScaleBytes, 16 * gm->g_down.RG, I / kTileK, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS) {
-        delete gm;
-        return cudaErrorInvalidValue;
+    for (int v = 0; v < 2; ++v) {
+        if (encode_tensor_map_2d(&gm->gu[v].map, CU_TENSOR_MAP_DATA_TYPE_UINT32, L.w.gu_scales, kTileRows, slabs_gu,
+                                 kTileScaleBytes, 16 * gm->gu[v].g.RG, H / kTileK,
+                                 CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
+            encode_tensor_map_2d(&gm->down[v].map, CU_TENSOR_MAP_DATA_TYPE_UINT32, L.w.d_scales, kTileRows, slabs_d,
+                                 kTileScaleBytes, 16 * gm->down[v].g.RG, I / kTileK,
+                                 CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS) {
+            delete gm;
+            return cudaErrorInvalidValue;
+        }
+        gm->gu[v].smem = gemv_smem_bytes(H, gm->gu[v].g);
+        gm->down[v].smem = gemv_smem_bytes(I, gm->down[v].g);
     }
     L.gemv_maps = gm;
     cudaError_t e = cudaFuncSetAttribute(gemv_kernel<Proj::GateUp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)gemv_smem_bytes(H, gm->g_gu));
+                                         (int)std::max(gm->gu[0].smem, gm->gu[1].smem));
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(gemv_kernel<Proj::Down>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)gemv_smem_bytes(I, gm->g_down));
+                                 (int)std::max(gm->down[0].smem, gm->down[1].smem));
     if (e != cudaSuccess) return e;
-    L.gemv_grid_gu = gemv_grid<Proj::GateUp>(H, gm->g_gu, L.num_sms);
-    L.gemv_grid_down = gemv_grid<Proj::Down>(I, gm->g_down, L.num_sms);
+    for (int v = 0; v < 2; ++v) {
+        gm->gu[v].grid = gemv_grid<Proj::GateUp>(H, gm->gu[v].g, L.num_sms);
+        gm->down[v].grid = gemv_grid<Proj::Down>(I, gm->down[v].g, L.num_sms);
+    }
     return cudaSuccess;
 }
 
@@ -593,7 +653,7 @@ static GemvArgs common_args(const Layer &L) {
     return g;
 }
 
-cudaError_t launch_gemv_gate_up(Layer &L, const uint16_t *x, cudaStream_t s, int *launches)
+cudaError_t launch_gemv_gate_up(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches)
 {
     (void)x;   // the routing kernels left x in block-scaled f16 form in ws.xq
     StageTimer timer(L, TFMOE_STAGE_GEMV_GATE_UP, s);
@@ -602,15 +662,16 @@ cudaError_t launch_gemv_gate_up(Layer &L, const uint16_t *x, cudaStream_t s, int
     g.codes = L.w.gu_codes;
     g.glob0 = L.w.gate_global; g.glob1 = L.w.up_global;
     g.R = 2 * L.desc.intermediate; g.K = L.desc.hidden;
-    g.KS = gm->g_gu.KS; g.RG = gm->g_gu.RG;
+    const GemvShape &sh = pick_shape(L, gm->gu, g.R, T);
+    g.KS = sh.g.KS; g.RG = sh.g.RG;
     g.src = L.ws.xq; g.src_inv = L.ws.xq_inv;
     g.act_out = L.ws.act; g.aq_out = L.ws.aq; g.aq_inv_out = L.ws.aq_inv;
-    gemv_kernel<Proj::GateUp><<<L.gemv_grid_gu, kThreads, gemv_smem_bytes(g.K, gm->g_gu), s>>>(gm->gu, g);
+    gemv_kernel<Proj::GateUp><<<sh.grid, kThreads, sh.smem, s>>>(sh.map, g);
     *launches += 1;
     return cudaGetLastError();
 }
 
-cudaError_t launch_gemv_down(Layer &L, cudaStream_t s, int *launches)
+cudaError_t launch_gemv_down(Layer &L, int T, cudaStream_t s, int *launches)
 {
     StageTimer timer(L, TFMOE_STAGE_GEMV_DOWN, s);
     const GemvMaps *gm = static_cast<const GemvMaps *>(L.gemv_maps);
@@ -618,29 +679,29 @@ cudaError_t launch_gemv_down(Layer &L, cudaStream_t s, int *launches)
     d.codes = L.w.d_codes;
     d.glob0 = L.w.down_global; d.glob1 = nullptr;
     d.R = L.desc.hidden; d.K = L.desc.intermediate;
-    d.KS = gm->g_down.KS; d.RG = gm->g_down.RG;
+    const GemvShape &sh = pick_shape(L, gm->down, d.R, T);
+    d.KS = sh.g.KS; d.RG = sh.g.RG;
     d.src = L.ws.aq; d.src_inv = L.ws.aq_inv;
     d.y_out = L.ws.y;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(L.gemv_grid_down);
+    cfg.gridDim = dim3(sh.grid);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = gemv_smem_bytes(d.K, gm->g_down);
+    cfg.dynamicSmemBytes = sh.smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = TFMOE_GEMV_DOWN_EARLY;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_kernel<Proj::Down>, gm->down, d);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_kernel<Proj::Down>, sh.map, d);
     *launches += 1;
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_gemv(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches)
 {
-    (void)T;
-    cudaError_t e = launch_gemv_gate_up(L, x, s, launches);
-    if (e == cudaSuccess) e = launch_gemv_down(L, s, launches);
+    cudaError_t e = launch_gemv_gate_up(L, x, T, s, launches);
+    if (e == cudaSuccess) e = launch_gemv_down(L, T, s, launches);
     return e;
 }
 

@@ -115,7 +115,6 @@ struct Layer {
     int32_t last_T = -1;            // T of the last successful forward (stage replays need it)
     bool last_use_mma = false, last_use_gemv = false;
     bool mma_small = false;         // the tensor-core regime of the current forward uses small tiles
-    int gemv_grid_gu = 0, gemv_grid_down = 0;
     size_t router_partial_cap = 0;  // doubles in ws.router_partial
     void *gemv_maps = nullptr;      // tensor maps of the GEMV regime's scale slabs
     void *mma_maps = nullptr;       // tensor maps of the MMA regime's token operands
@@ -151,8 +150,8 @@ inline int gemv_threshold(const Layer &L, int T) {
 cudaError_t launch_router(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches);
 cudaError_t launch_permute(Layer &L, int T, cudaStream_t s, int *launches);
 cudaError_t launch_gemv(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches);
-cudaError_t launch_gemv_gate_up(Layer &L, const uint16_t *x, cudaStream_t s, int *launches);
-cudaError_t launch_gemv_down(Layer &L, cudaStream_t s, int *launches);
+cudaError_t launch_gemv_gate_up(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches);
+cudaError_t launch_gemv_down(Layer &L, int T, cudaStream_t s, int *launches);
 cudaError_t launch_combine(Layer &L, int T, uint16_t *out, cudaStream_t s, int *launches);
 cudaError_t launch_repack(const Layer &L, const tfmoe_weights &src, cudaStream_t s);
 cudaError_t gemv_setup(Layer &L);
