@@ -44,9 +44,6 @@ constexpr int kThreads = (kComputeWarps + 1) * 32;   // + the control warp
 #ifndef TFMOE_GEMV_CTAS_PER_SM
 #define TFMOE_GEMV_CTAS_PER_SM 2
 #endif
-#ifndef TFMOE_GEMV_TOKENS_PER_PASS
-#define TFMOE_GEMV_TOKENS_PER_PASS 2
-#endif
 constexpr int kCtasPerSm = TFMOE_GEMV_CTAS_PER_SM;
 #ifndef TFMOE_GEMV_RING
 #define TFMOE_GEMV_RING 3
@@ -60,8 +57,7 @@ constexpr int kCtasPerSm = TFMOE_GEMV_CTAS_PER_SM;
 constexpr int kChunk = TFMOE_GEMV_CHUNK;   // column tiles per ring slot of a compute warp
 constexpr int kRing = TFMOE_GEMV_RING;   // ring slots per compute warp (kRing - 1 chunks in flight)
 static_assert(kRing >= 2, "ring depth");
-constexpr int kMaxNT = TFMOE_GEMV_TOKENS_PER_PASS;   // tokens per pass (2 or 4)
-static_assert(kMaxNT == 2 || kMaxNT == 4, "tokens per pass");
+constexpr int kMaxNT = 2;   // tokens per pass (the partial sums of a pass are one f32 pair per lane)
 
 enum class Proj { GateUp, Down };
 
@@ -163,6 +159,9 @@ __device__ __forceinline__ float2 lds64f(uint32_t a) {
     asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
     return v;
 }
+__device__ __forceinline__ void sts_f32x2(uint32_t a, float v0, float v1) {
+    asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(a), "f"(v0), "f"(v1) : "memory");
+}
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
@@ -244,8 +243,12 @@ __device__ __forceinline__ void pass_run(uint32_t ring, int &slot_use, int KTW, 
     const int nch = (KTW + kChunk - 1) / kChunk;
     for (int ch = 0; ch < nch; ++ch) {
         cp_async_wait<kRing - 2>();
-        chunk_compute<NT>(ring + (uint32_t)slot_use * (kChunk * 512), min(kChunk, KTW - ch * kChunk), sc, sc_step, hsh,
-                          xa, xia, x_tok, xi_tok, acc);
+        const uint32_t cs = ring + (uint32_t)slot_use * (kChunk * 512);
+        const int n = KTW - ch * kChunk;
+        if (n >= kChunk)   // full chunk: the tile count is a constant
+            chunk_compute<NT>(cs, kChunk, sc, sc_step, hsh, xa, xia, x_tok, xi_tok, acc);
+        else
+            chunk_compute<NT>(cs, n, sc, sc_step, hsh, xa, xia, x_tok, xi_tok, acc);
         refill();
         slot_use = (slot_use + 1 == kRing) ? 0 : slot_use + 1;
         sc += kChunk * sc_step;
@@ -500,11 +503,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     }
     auto refill = [&]() {
         if (pvalid) {
-            const int n = min(kChunk, KTW - pch * kChunk);
+            const int n = KTW - pch * kChunk;
             const uint32_t d = ring + (uint32_t)slot_fill * (kChunk * 512);
+            if (n >= kChunk) {
 #pragma unroll
-            for (int j = 0; j < kChunk; ++j)
-                if (j < n) cp_async16(d + j * 512, pg + (size_t)j * kTileCodeBytes);
+                for (int j = 0; j < kChunk; ++j) cp_async16(d + j * 512, pg + (size_t)j * kTileCodeBytes);
+            } else {
+#pragma unroll
+                for (int j = 0; j < kChunk - 1; ++j)
+                    if (j < n) cp_async16(d + j * 512, pg + (size_t)j * kTileCodeBytes);
+            }
             pg += (size_t)kChunk * kTileCodeBytes;
             if (++pch == nch) {
                 pch = 0;
@@ -532,37 +540,35 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     int p = 0, tn = 0;
     const uint32_t sc_step = (uint32_t)rows_task * 4u, hsh = (uint32_t)h * 16u;
     const uint32_t x_tok = (uint32_t)K * 2u, xi_tok = (uint32_t)(K / 16) * 4u;
+    // this lane's addresses in buffer 0 of each double buffer; buffer 1 is one size further
+    const uint32_t sm0 = smem_u32(base);
+    const uint32_t sc0 = sm0 + (uint32_t)lay.sc + (uint32_t)((ks * KTW) * rows_task + lrow) * 4u;
+    const uint32_t x0 = sm0 + (uint32_t)lay.x + (uint32_t)col0 * 2u;
+    const uint32_t xi0 = sm0 + (uint32_t)lay.xi + (uint32_t)(col0 / 16) * 4u;
+    const uint32_t red0 = sm0 + (uint32_t)lay.red + (uint32_t)(ks * rows_task + lrow) * (kMaxNT * 4u);
     for (Cursor c = c0; c.id < n_tasks; advance(c)) {
         int r_begin;
         const int m = task_rows(c, r_begin);
         if (m <= 0) continue;
         const int sb = tn & 1;
-        const uint32_t sc = smem_u32(sbuf(sb)) + (uint32_t)((ks * KTW) * rows_task + lrow) * 4u;
+        const uint32_t sc = sc0 + (uint32_t)sb * (uint32_t)lay.sc_sz;
         wait_or_abort(&sfull[sb], (tn >> 1) & 1, abort_flag, a.err_word);
         for (int t0 = 0; t0 < m; t0 += kMaxNT, ++p) {
             const int nt = min(kMaxNT, m - t0);
             const int xb = p & 1;
             wait_or_abort(&xfull[xb], (p >> 1) & 1, abort_flag, a.err_word);
-            const uint32_t xa = smem_u32(xbuf(xb)) + (uint32_t)col0 * 2u;
-            const uint32_t xia = smem_u32(xibuf(xb)) + (uint32_t)(col0 / 16) * 4u;
+            const uint32_t xa = x0 + (uint32_t)xb * (uint32_t)lay.x_sz;
+            const uint32_t xia = xi0 + (uint32_t)xb * (uint32_t)lay.xi_sz;
             float acc[kMaxNT] = {};
-            switch (nt) {
-            case 1: pass_run<1>(ring, slot_use, KTW, sc, sc_step, hsh, xa, xia, x_tok, xi_tok, acc, refill); break;
-            case 2: pass_run<2>(ring, slot_use, KTW, sc, sc_step, hsh, xa, xia, x_tok, xi_tok, acc, refill); break;
-            case 3:
-                pass_run<(kMaxNT > 2 ? 3 : 2)>(ring, slot_use, KTW, sc, sc_step, hsh, xa, xia, x_tok, xi_tok, acc, refill);
-                break;
-            default: pass_run<kMaxNT>(ring, slot_use, KTW, sc, sc_step, hsh, xa, xia, x_tok, xi_tok, acc, refill); break;
-            }
+            if (nt == 1)
+                pass_run<1>(ring, slot_use, KTW, sc, sc_step, hsh, xa, xia, x_tok, xi_tok, acc, refill);
+            else
+                pass_run<2>(ring, slot_use, KTW, sc, sc_step, hsh, xa, xia, x_tok, xi_tok, acc, refill);
 #pragma unroll
             for (int t = 0; t < kMaxNT; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 16);
             // the control warp has consumed what pass p-2 left in this buffer
             if (p >= 2) wait_or_abort(&rfree[xb], ((p - 2) >> 1) & 1, abort_flag, a.err_word);
-            float *rb = red(xb);
-            if (h == 0) {
-#pragma unroll
-                for (int t = 0; t < kMaxNT; ++t) rb[((size_t)ks * rows_task + lrow) * kMaxNT + t] = acc[t];
-            }
+            if (h == 0) sts_f32x2(red0 + (uint32_t)xb * (uint32_t)lay.red_sz, acc[0], acc[1]);
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[xb]);
         }
