@@ -119,7 +119,7 @@ Geometry geometry(bool gate_up, int K) {
 // Shared memory of a CTA, in bytes from a 128-byte aligned base: two buffers each of
 // the task's scales [KT][16*RG] u32, the partial sums [KS][16*RG][kMaxNT] f32, the
 // pass's activation rows [kMaxNT][K] f16 and their inverse scales [kMaxNT][K/16] f32;
-// the GEMV list table [3][<= 256] i32; per compute warp a ring of kRing code chunks
+// the GEMV list table [5][<= 256] (expert, first row, rows, per-tensor scales); per compute warp a ring of kRing code chunks
 // (kChunk tiles x 32 lanes x 16 bytes); 8 mbarriers and an abort flag.
 constexpr int kMaxList = 256;
 struct SmemLayout {
@@ -135,7 +135,7 @@ struct SmemLayout {
         x = red + 2 * red_sz;
         xi = x + 2 * x_sz;
         tab = xi + 2 * xi_sz;
-        ring = tab + 3 * kMaxList * 4;
+        ring = tab + 5 * kMaxList * 4;
         bar = ring + (size_t)kComputeWarps * kRing * kChunk * 32 * 16;
         total = bar + 9 * sizeof(uint64_t);
     }
@@ -144,8 +144,11 @@ size_t gemv_smem_bytes(int K, Geometry g) { return 128 + SmemLayout(K, g.KS, g.R
 
 // 16-byte asynchronous copy global -> shared (cp.async, bypassing L1): the code stream
 // stays 128-bit coalesced loads while the data waits in shared memory, not registers.
+// The offsets are immediates of the instruction: a chunk's copies share two base registers.
+template <int DOFF, int SOFF>
 __device__ __forceinline__ void cp_async16(uint32_t smem_dst, const void *gmem_src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_dst), "l"(gmem_src) : "memory");
+    asm volatile("cp.async.cg.shared.global [%0+%2], [%1+%3], 16;" ::"r"(smem_dst), "l"(gmem_src), "n"(DOFF),
+                 "n"(SOFF) : "memory");
 }
 // Shared-memory loads by 32-bit address: the inner loop's addresses are a few
 // per-pass bases plus constant offsets, with no generic-pointer arithmetic.
@@ -154,17 +157,20 @@ __device__ __forceinline__ uint32_t lds32(uint32_t a) {
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
     return v;
 }
+template <int OFF>
 __device__ __forceinline__ float2 lds64f(uint32_t a) {
     float2 v;
-    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2+%3];" : "=f"(v.x), "=f"(v.y) : "r"(a), "n"(OFF));
     return v;
 }
 __device__ __forceinline__ void sts_f32x2(uint32_t a, float v0, float v1) {
     asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(a), "f"(v0), "f"(v1) : "memory");
 }
+template <int OFF>
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
     uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4+%5];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a), "n"(OFF));
     return v;
 }
 // The E4M3 pair in bits [sh, sh + 16) of w -> two floats (exact).
@@ -186,86 +192,100 @@ __device__ __forceinline__ float fma2_f16_f32(uint32_t w2, uint32_t x2, float ac
     return acc;
 }
 
-// One lane's share of n <= kChunk column tiles for NT tokens, all operands in shared
-// memory addressed by 32-bit bases:
-//   cs  the lane's 16 code bytes of the chunk's first tile (tiles 512 bytes apart);
-//   sc  the lane's 4 scale bytes of that tile (tiles sc_step bytes apart; the lane's
-//       half takes bits [hsh, hsh + 16));
-//   xa  token 0's 32 activation values of the lane's half of that tile (tiles 128
-//       bytes apart, tokens x_tok bytes apart); xia their two inverse scales (tiles
-//       16 bytes apart, tokens xi_tok bytes apart).
+// Eight weights (one code word) against the matching 8 activations of each token:
+// XOFF is the byte offset of those activations from the chunk's bases xa0 / xa1.
+template <int NT, int XOFF>
+__device__ __forceinline__ void word8(uint32_t w, uint32_t xa0, uint32_t xa1, float (&pp)[NT]) {
+    uint32_t wp[4];
+    e2m1x8_to_f16x2x4(w, wp);
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        const uint4 xv = lds128<XOFF>(t == 0 ? xa0 : xa1);
+        pp[t] = fma2_f16_f32(wp[0], xv.x, pp[t]);
+        pp[t] = fma2_f16_f32(wp[1], xv.y, pp[t]);
+        pp[t] = fma2_f16_f32(wp[2], xv.z, pp[t]);
+        pp[t] = fma2_f16_f32(wp[3], xv.w, pp[t]);
+    }
+}
+
+// Tile J of a chunk: the lane's 32 weights (16 code bytes at cs + 512 J) against NT
+// tokens. Activations of token t start at xa_t + 128 J (32 f16 values, 4 per word
+// pair) with their two inverse block scales at xi_t + 16 J; the lane's two E4M3
+// scales are bits [hsh, hsh + 16) of the word at sc.
+template <int NT, int J>
+__device__ __forceinline__ void tile_compute(uint32_t cs, uint32_t sc, uint32_t hsh, uint32_t xa0, uint32_t xa1,
+                                             uint32_t xi0, uint32_t xi1, float (&acc)[kMaxNT])
+{
+    const float2 s = e4m3_pair_at(lds32(sc), hsh);
+    const uint4 cw = lds128<J * 512>(cs);
+    float p0[NT], p1[NT];   // 16-column blocks 0 and 1 of the lane's 32 columns
+#pragma unroll
+    for (int t = 0; t < NT; ++t) p0[t] = p1[t] = 0.f;
+    word8<NT, J * 128 + 0>(cw.x, xa0, xa1, p0);
+    word8<NT, J * 128 + 16>(cw.y, xa0, xa1, p0);
+    word8<NT, J * 128 + 32>(cw.z, xa0, xa1, p1);
+    word8<NT, J * 128 + 48>(cw.w, xa0, xa1, p1);
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        const float2 inv = lds64f<J * 16>(t == 0 ? xi0 : xi1);
+        acc[t] = fmaf(p0[t], s.x * inv.x, acc[t]);
+        acc[t] = fmaf(p1[t], s.y * inv.y, acc[t]);
+    }
+}
+
+// The n <= kChunk tiles of one chunk (n is a constant for full chunks).
+static_assert(kChunk == 4, "tile_compute is unrolled for 4-tile chunks");
 template <int NT>
 __device__ __forceinline__ void chunk_compute(uint32_t cs, int n, uint32_t sc, uint32_t sc_step, uint32_t hsh,
-                                              uint32_t xa, uint32_t xia, uint32_t x_tok, uint32_t xi_tok,
+                                              uint32_t xa0, uint32_t xa1, uint32_t xi0, uint32_t xi1,
                                               float (&acc)[kMaxNT])
 {
-#pragma unroll
-    for (int j = 0; j < kChunk; ++j) {
-        if (j >= n) break;
-        const float2 s = e4m3_pair_at(lds32(sc), hsh);
-        sc += sc_step;
-        const uint4 cw = lds128(cs + j * 512);
-        const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-        float p[NT][2];
-#pragma unroll
-        for (int t = 0; t < NT; ++t) p[t][0] = p[t][1] = 0.f;
-        // word q holds columns 8q .. 8q+7 of the lane's 32 (16-column block q / 2)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            uint32_t wp[4];
-            e2m1x8_to_f16x2x4(words[q], wp);
-#pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                const uint4 xv = lds128(xa + t * x_tok + j * 128 + q * 16);
-                float &pp = p[t][q >> 1];
-                pp = fma2_f16_f32(wp[0], xv.x, pp);
-                pp = fma2_f16_f32(wp[1], xv.y, pp);
-                pp = fma2_f16_f32(wp[2], xv.z, pp);
-                pp = fma2_f16_f32(wp[3], xv.w, pp);
-            }
-        }
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            const float2 inv = lds64f(xia + t * xi_tok + j * 16);
-            acc[t] = fmaf(p[t][0], s.x * inv.x, acc[t]);
-            acc[t] = fmaf(p[t][1], s.y * inv.y, acc[t]);
-        }
-    }
+    tile_compute<NT, 0>(cs, sc, hsh, xa0, xa1, xi0, xi1, acc);
+    if (n > 1) tile_compute<NT, 1>(cs, sc + sc_step, hsh, xa0, xa1, xi0, xi1, acc);
+    if (n > 2) tile_compute<NT, 2>(cs, sc + 2 * sc_step, hsh, xa0, xa1, xi0, xi1, acc);
+    if (n > 3) tile_compute<NT, 3>(cs, sc + 3 * sc_step, hsh, xa0, xa1, xi0, xi1, acc);
+}
+
+// A lane's position in its code stream. The ring holds kRing chunk slots of
+// kChunk * 512 bytes; `use` and `fill` are byte offsets of the slot read next and
+// the slot filled next (kRing - 1 slots apart).
+constexpr uint32_t kSlotBytes = kChunk * 512;
+__device__ __forceinline__ uint32_t next_slot(uint32_t off) {
+    return off == (kRing - 1) * kSlotBytes ? 0u : off + kSlotBytes;
 }
 
 // All column chunks of one pass: wait for the lane's oldest copies, compute, and let
 // `refill` put the next chunk of the stream into the slot freed by the previous one.
 template <int NT, class Refill>
-__device__ __forceinline__ void pass_run(uint32_t ring, int &slot_use, int KTW, uint32_t sc, uint32_t sc_step,
-                                         uint32_t hsh, uint32_t xa, uint32_t xia, uint32_t x_tok, uint32_t xi_tok,
-                                         float (&acc)[kMaxNT], Refill &refill)
+__device__ __forceinline__ void pass_run(uint32_t ring, uint32_t &use, int nch, int n_last, uint32_t sc,
+                                         uint32_t sc_step, uint32_t hsh, uint32_t xa0, uint32_t xa1, uint32_t xi0,
+                                         uint32_t xi1, float (&acc)[kMaxNT], Refill &refill)
 {
-    const int nch = (KTW + kChunk - 1) / kChunk;
     for (int ch = 0; ch < nch; ++ch) {
         cp_async_wait<kRing - 2>();
-        const uint32_t cs = ring + (uint32_t)slot_use * (kChunk * 512);
-        const int n = KTW - ch * kChunk;
-        if (n >= kChunk)   // full chunk: the tile count is a constant
-            chunk_compute<NT>(cs, kChunk, sc, sc_step, hsh, xa, xia, x_tok, xi_tok, acc);
+        if (ch + 1 < nch || n_last == kChunk)
+            chunk_compute<NT>(ring + use, kChunk, sc, sc_step, hsh, xa0, xa1, xi0, xi1, acc);
         else
-            chunk_compute<NT>(cs, n, sc, sc_step, hsh, xa, xia, x_tok, xi_tok, acc);
+            chunk_compute<NT>(ring + use, n_last, sc, sc_step, hsh, xa0, xa1, xi0, xi1, acc);
         refill();
-        slot_use = (slot_use + 1 == kRing) ? 0 : slot_use + 1;
+        use = next_slot(use);
         sc += kChunk * sc_step;
-        xa += kChunk * 128;
-        xia += kChunk * 16;
+        xa0 += kChunk * 128;
+        xa1 += kChunk * 128;
+        xi0 += kChunk * 16;
+        xi1 += kChunk * 16;
     }
 }
 
 // Bounded mbarrier wait shared by every role of the CTA: gives up (returning false)
 // once another thread has flagged an abort or after kWaitLimitNs, flagging it itself.
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int32_t *abort_flag,
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int32_t *abort_flag,
                                               int32_t *err_word) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_at(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
         for (int i = 0; i < 4; ++i)
-            if (mbar_try_wait_sleep(bar, parity)) return true;
+            if (mbar_try_wait_sleep_at(bar, parity)) return true;
         if (*abort_flag) return false;
         if (global_timer_ns() - t0 > kWaitLimitNs) {
             atomicOr(err_word, DEV_ERR_WAIT_TIMEOUT);
@@ -310,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     auto red = [&](int b) { return reinterpret_cast<float *>(base + lay.red + b * lay.red_sz); };
     auto xbuf = [&](int b) { return reinterpret_cast<uint16_t *>(base + lay.x + b * lay.x_sz); };
     auto xibuf = [&](int b) { return reinterpret_cast<float *>(base + lay.xi + b * lay.xi_sz); };
-    int32_t *tab = reinterpret_cast<int32_t *>(base + lay.tab);     // [3][n_list]: expert, first row, rows
+    int32_t *tab = reinterpret_cast<int32_t *>(base + lay.tab);     // [5][n_list]: expert, first row, rows, g0, g1
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + lay.bar);
     uint64_t *sfull = bars, *xfull = bars + 2, *full = bars + 4, *rfree = bars + 6;
     volatile int32_t *abort_flag = reinterpret_cast<volatile int32_t *>(bars + 8);
@@ -333,6 +353,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
         tab[i] = e;
         tab[n_list + i] = rb;
         tab[2 * n_list + i] = __ldg(a.offsets + e + 1) - rb;
+        tab[3 * n_list + i] = __float_as_int(__ldg(a.glob0 + e));
+        tab[4 * n_list + i] = P == Proj::GateUp ? __float_as_int(__ldg(a.glob1 + e)) : 0;
     }
     __syncthreads();
 
@@ -411,26 +433,46 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
                 }
             }
         };
+        // The issue cursor runs two passes ahead of the pass being consumed: pass p+2's
+        // copies go out as soon as pass p's partial sums are in (its buffers were last
+        // read by pass p), before pass p's epilogue.
+        Cursor ic;
+        bool ivalid = first_pass(ic);
+        int it0 = 0, itn = 0, ip = 0;
+        auto issue_next = [&](bool first) {
+            if (!ivalid) return;
+            int rb;
+            const int m = task_rows(ic, rb);
+            issue(ic, it0, itn, ip, first);
+            Cursor nc;
+            int nt0;
+            if (next_pass(ic, it0, m, nc, nt0)) {
+                if (nc.id != ic.id) ++itn;
+                ic = nc;
+                it0 = nt0;
+            } else {
+                ivalid = false;
+            }
+            ++ip;
+        };
         Cursor fc;
         if (first_pass(fc)) {
-            issue(fc, 0, 0, 0, true);
-            int p = 0, tn = 0;
+            issue_next(true);
+            issue_next(false);
+            int p = 0;
             for (Cursor c = fc; c.id < n_tasks; advance(c)) {
                 int r_begin;
                 const int m = task_rows(c, r_begin);
                 if (m <= 0) continue;
-                const int e = tab[c.li], row0 = c.sub * rows_task;
+                const int row0 = c.sub * rows_task;
                 for (int t0 = 0; t0 < m; t0 += kMaxNT, ++p) {
                     const int nt = min(kMaxNT, m - t0);
-                    Cursor nc;
-                    int nt0;
-                    // the buffers of pass p+1 were last read in pass p-1, whose sums were consumed below
-                    if (next_pass(c, t0, m, nc, nt0)) issue(nc, nt0, nc.id == c.id ? tn : tn + 1, p + 1, false);
-                    wait_or_abort(&full[p & 1], (p >> 1) & 1, abort_flag, a.err_word);
+                    wait_or_abort(smem_u32(&full[p & 1]), (p >> 1) & 1, abort_flag, a.err_word);
+                    issue_next(false);
                     const float *rb = red(p & 1);
                     if (P == Proj::GateUp) {
                         // rows_task is a multiple of 32: a round covers 32 rows (16 gate/up pairs) of one token
-                        const float g0 = __ldg(a.glob0 + e), g1 = __ldg(a.glob1 + e);
+                        const float g0 = __int_as_float(tab[3 * n_list + c.li]), g1 = __int_as_float(tab[4 * n_list + c.li]);
                         for (int i0 = 0; i0 < rows_task * nt; i0 += 32) {
                             const int i = i0 + lane, t = i >> rt_log2, rl = i & (rows_task - 1);
                             float v = 0.f;
@@ -456,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
                             if (lane == 0) a.aq_inv_out[r * (a.I / 16) + (j >> 4)] = __int_as_float((127 - sh) << 23);
                         }
                     } else {
-                        const float gs = __ldg(a.glob0 + e);
+                        const float gs = __int_as_float(tab[3 * n_list + c.li]);
                         for (int i = lane; i < rows_task * nt; i += 32) {
                             const int t = i >> rt_log2, rl = i & (rows_task - 1);
                             float v = 0.f;
@@ -467,7 +509,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&rfree[p & 1]);
                 }
-                ++tn;
             }
         }
         // after an abort, let the latest copies land before the CTA exits (bounded)
@@ -483,60 +524,76 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     const int h = lane >> 4;
     const int lrow = rgl * 16 + (lane & 15);              // row of the lane inside the task
     const int col0 = ks * KTW * kTileK + h * 32;          // first column of the lane's slice and half
-    auto lane_codes = [&](const Cursor &c) -> const uint8_t * {
-        const int row0 = c.sub * rows_task;
-        return a.codes + ((size_t)(tab[c.li] * RT + row0 / kTileRows) * KT + (size_t)ks * KTW) *
-                   kTileCodeBytes + h * 2048 + (row0 % kTileRows + lrow) * 16;
+    const int nch = (KTW + kChunk - 1) / kChunk, n_last = KTW - (nch - 1) * kChunk;
+    // the lane's bytes of a task's first code tile: tile (e, rt, ks * KTW), half h, row lrow
+    const uint32_t lane_off = (uint32_t)(ks * KTW) * kTileCodeBytes + (uint32_t)h * 2048u + (uint32_t)lrow * 16u;
+    auto task_codes = [&](const Cursor &c) -> const uint8_t * {
+        const int row0 = c.sub << rt_log2;
+        return a.codes + (size_t)((tab[c.li] * RT + (row0 >> 7)) * KT) * kTileCodeBytes + lane_off +
+               (uint32_t)(row0 & (kTileRows - 1)) * 16u;
     };
     // The warp's code stream: the (task, pass, chunk) sequence it consumes, kRing - 1
     // chunks ahead. Each lane copies and later reads only its own 16-byte pieces, so a
     // lane's cp.async.wait_group is all the synchronisation the ring needs.
     const uint32_t ring = smem_u32(base + lay.ring) + (uint32_t)(warp * kRing * kChunk * 32 + lane) * 16u;
-    const int nch = (KTW + kChunk - 1) / kChunk;
     Cursor pc{};                                          // task of the next chunk of the stream
     bool pvalid = false;
-    int pt0 = 0, pch = 0, slot_fill = 0;
+    int pt0 = 0, pm = 0, pleft = nch;                     // its first token, rows, chunks left in the pass
+    uint32_t fill = 0;
     const uint8_t *pg = nullptr;                          // next chunk of the stream (this lane's bytes)
     {
         Cursor ft;
-        if (first_pass(ft)) { pc = ft; pvalid = true; pg = lane_codes(ft); }
+        if (first_pass(ft)) {
+            int rb;
+            pc = ft;
+            pvalid = true;
+            pm = task_rows(ft, rb);
+            pg = task_codes(ft);
+        }
     }
     auto refill = [&]() {
         if (pvalid) {
-            const int n = KTW - pch * kChunk;
-            const uint32_t d = ring + (uint32_t)slot_fill * (kChunk * 512);
-            if (n >= kChunk) {
-#pragma unroll
-                for (int j = 0; j < kChunk; ++j) cp_async16(d + j * 512, pg + (size_t)j * kTileCodeBytes);
+            const uint32_t d = ring + fill;
+            if (pleft > 1 || n_last == kChunk) {
+                cp_async16<0, 0>(d, pg);
+                cp_async16<512, kTileCodeBytes>(d, pg);
+                cp_async16<1024, 2 * kTileCodeBytes>(d, pg);
+                cp_async16<1536, 3 * kTileCodeBytes>(d, pg);
             } else {
-#pragma unroll
-                for (int j = 0; j < kChunk - 1; ++j)
-                    if (j < n) cp_async16(d + j * 512, pg + (size_t)j * kTileCodeBytes);
+                cp_async16<0, 0>(d, pg);
+                if (n_last > 1) cp_async16<512, kTileCodeBytes>(d, pg);
+                if (n_last > 2) cp_async16<1024, 2 * kTileCodeBytes>(d, pg);
             }
-            pg += (size_t)kChunk * kTileCodeBytes;
-            if (++pch == nch) {
-                pch = 0;
-                int rb, nt0;
-                Cursor nc;
-                const int m = task_rows(pc, rb);
-                if (next_pass(pc, pt0, m, nc, nt0)) {
-                    if (nc.id != pc.id) pg = lane_codes(nc);
-                    else pg -= (size_t)nch * kChunk * kTileCodeBytes;   // same task, next tokens
-                    pc = nc;
-                    pt0 = nt0;
+            pg += kChunk * kTileCodeBytes;
+            if (--pleft == 0) {
+                pleft = nch;
+                if (pt0 + kMaxNT < pm) {                  // same task, next tokens
+                    pt0 += kMaxNT;
+                    pg -= (size_t)nch * kChunk * kTileCodeBytes;
                 } else {
-                    pvalid = false;
+                    Cursor nc;
+                    int nt0;
+                    if (next_pass(pc, pt0, pm, nc, nt0)) {
+                        int rb;
+                        pc = nc;
+                        pt0 = 0;
+                        pm = task_rows(nc, rb);
+                        pg = task_codes(nc);
+                    } else {
+                        pvalid = false;
+                    }
                 }
             }
         }
         cp_async_commit();
-        slot_fill = (slot_fill + 1 == kRing) ? 0 : slot_fill + 1;
+        fill = next_slot(fill);
     };
+    const bool has_work = pvalid;
     for (int i = 0; i < kRing - 1; ++i) refill();
     // weights only so far; the bounded waits below start after the gate/up grid is done
-    if (P == Proj::Down && pvalid) grid_dep_wait();
+    if (P == Proj::Down && has_work) grid_dep_wait();
 
-    int slot_use = 0;
+    uint32_t use = 0;
     int p = 0, tn = 0;
     const uint32_t sc_step = (uint32_t)rows_task * 4u, hsh = (uint32_t)h * 16u;
     const uint32_t x_tok = (uint32_t)K * 2u, xi_tok = (uint32_t)(K / 16) * 4u;
@@ -546,31 +603,31 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     const uint32_t x0 = sm0 + (uint32_t)lay.x + (uint32_t)col0 * 2u;
     const uint32_t xi0 = sm0 + (uint32_t)lay.xi + (uint32_t)(col0 / 16) * 4u;
     const uint32_t red0 = sm0 + (uint32_t)lay.red + (uint32_t)(ks * rows_task + lrow) * (kMaxNT * 4u);
+    const uint32_t bar0 = smem_u32(bars);                 // sfull, xfull, full, rfree: 2 each, 8 bytes apart
     for (Cursor c = c0; c.id < n_tasks; advance(c)) {
         int r_begin;
         const int m = task_rows(c, r_begin);
         if (m <= 0) continue;
         const int sb = tn & 1;
         const uint32_t sc = sc0 + (uint32_t)sb * (uint32_t)lay.sc_sz;
-        wait_or_abort(&sfull[sb], (tn >> 1) & 1, abort_flag, a.err_word);
+        wait_or_abort(bar0 + 8u * sb, (tn >> 1) & 1, abort_flag, a.err_word);
         for (int t0 = 0; t0 < m; t0 += kMaxNT, ++p) {
-            const int nt = min(kMaxNT, m - t0);
             const int xb = p & 1;
-            wait_or_abort(&xfull[xb], (p >> 1) & 1, abort_flag, a.err_word);
+            wait_or_abort(bar0 + 16u + 8u * xb, (p >> 1) & 1, abort_flag, a.err_word);
             const uint32_t xa = x0 + (uint32_t)xb * (uint32_t)lay.x_sz;
             const uint32_t xia = xi0 + (uint32_t)xb * (uint32_t)lay.xi_sz;
             float acc[kMaxNT] = {};
-            if (nt == 1)
-                pass_run<1>(ring, slot_use, KTW, sc, sc_step, hsh, xa, xia, x_tok, xi_tok, acc, refill);
+            if (m - t0 == 1)
+                pass_run<1>(ring, use, nch, n_last, sc, sc_step, hsh, xa, xa + x_tok, xia, xia + xi_tok, acc, refill);
             else
-                pass_run<2>(ring, slot_use, KTW, sc, sc_step, hsh, xa, xia, x_tok, xi_tok, acc, refill);
+                pass_run<2>(ring, use, nch, n_last, sc, sc_step, hsh, xa, xa + x_tok, xia, xia + xi_tok, acc, refill);
 #pragma unroll
             for (int t = 0; t < kMaxNT; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], 16);
             // the control warp has consumed what pass p-2 left in this buffer
-            if (p >= 2) wait_or_abort(&rfree[xb], ((p - 2) >> 1) & 1, abort_flag, a.err_word);
+            if (p >= 2) wait_or_abort(bar0 + 48u + 8u * xb, ((p - 2) >> 1) & 1, abort_flag, a.err_word);
             if (h == 0) sts_f32x2(red0 + (uint32_t)xb * (uint32_t)lay.red_sz, acc[0], acc[1]);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&full[xb]);
+            if (lane == 0) mbar_arrive_at(bar0 + 32u + 8u * xb);
         }
         ++tn;
     }
