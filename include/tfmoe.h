@@ -210,7 +210,10 @@ typedef enum {
  * must be its input (read by the gate/up stages); out receives the combine
  * stage's result. Supported stages: GEMV_GATE_UP, GEMV_DOWN, MMA_GATE_UP,
  * MMA_DOWN, GATHER, COMBINE (others return TFMOE_ERR_UNSUPPORTED); a stage
- * whose kernels the forward did not use enqueues nothing.
+ * whose kernels the forward did not use enqueues nothing. Stage kernels are
+ * launched in plain stream order (tfmoe_forward lets the down projection and
+ * the combine start early, as programmatic dependents of the kernel before
+ * them), so back-to-back replays of one stage do not overlap.
  */
 TFMOE_API tfmoe_status tfmoe_forward_stage(tfmoe_layer *layer, int32_t stage, const uint16_t *x, int32_t T,
                                            uint16_t *out, void *cuda_stream);

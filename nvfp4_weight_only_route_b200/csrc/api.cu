@@ -394,6 +394,11 @@ tfmoe_status tfmoe_forward_stage(tfmoe_layer *layer, int32_t stage, const uint16
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
     int n = 0;
     cudaError_t e = cudaSuccess;
+    struct PlainOrder {   // for this call only, whatever path it returns by
+        Layer &L;
+        explicit PlainOrder(Layer &l) : L(l) { L.plain_order = true; }
+        ~PlainOrder() { L.plain_order = false; }
+    } plain(L);
     switch (stage) {
     case TFMOE_STAGE_GEMV_GATE_UP:
         if (!x) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward_stage: x is NULL");

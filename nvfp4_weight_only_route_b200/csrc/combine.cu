@@ -7,6 +7,10 @@
 #include "common.cuh"
 #include "internal.h"
 
+#ifndef TFMOE_COMBINE_EARLY
+#define TFMOE_COMBINE_EARLY 1
+#endif
+
 namespace tfmoe {
 namespace {
 
@@ -16,6 +20,8 @@ __global__ void __launch_bounds__(256) combine_kernel(
     const float *__restrict__ y, const float *__restrict__ g, const int32_t *__restrict__ inv,
     uint16_t *__restrict__ out, int T, int H, int k, int P, int32_t *err_word, int debug)
 {
+    // launched as a programmatic dependent of the down projection: y is final past this wait
+    grid_dep_wait();
     const int per_token = H / 8;
     const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (size_t)T * per_token) return;
@@ -50,10 +56,19 @@ cudaError_t launch_combine(Layer &L, int T, uint16_t *out, cudaStream_t s, int *
     const int H = L.desc.hidden, k = L.desc.top_k;
     const size_t n = (size_t)T * (H / 8);
     const int debug = (L.desc.flags & TFMOE_FLAG_DEBUG_CHECKS) ? 1 : 0;
-    combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(L.ws.y, L.ws.topk_w, L.ws.inv, out, T, H, k,
-                                                               T * k, L.ws.err_word, debug);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)((n + 255) / 256));
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = L.plain_order ? 0 : TFMOE_COMBINE_EARLY;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, combine_kernel, (const float *)L.ws.y, (const float *)L.ws.topk_w,
+                                             (const int32_t *)L.ws.inv, out, T, H, k, T * k, L.ws.err_word, debug);
     *launches += 1;
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace tfmoe

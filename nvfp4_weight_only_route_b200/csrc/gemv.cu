@@ -320,9 +320,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     const int RT = a.R / kTileRows, tpe = a.R / rows_task;
     const int n_list = __ldg(a.list_size);
     const int n_tasks = n_list * tpe;
-    // The down launch depends on this grid programmatically: its CTAs may take the
-    // slots of gate/up CTAs that finished and fetch weights while the rest still run.
-    if (P == Proj::GateUp) grid_dep_launch_dependents();
+    // The next launch (down after gate/up, the combine after down) depends on this grid
+    // programmatically: its CTAs may start while this grid runs and wait for it there.
+    grid_dep_launch_dependents();
     if ((int)blockIdx.x >= n_tasks) return;
 
     const SmemLayout lay(K, KS, RG);
@@ -753,7 +753,7 @@ cudaError_t launch_gemv_down(Layer &L, int T, cudaStream_t s, int *launches)
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = TFMOE_GEMV_DOWN_EARLY;
+    attr[0].val.programmaticStreamSerializationAllowed = L.plain_order ? 0 : TFMOE_GEMV_DOWN_EARLY;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_kernel<Proj::Down>, sh.map, d);

@@ -120,6 +120,7 @@ struct Layer {
     void *mma_maps = nullptr;       // tensor maps of the MMA regime's token operands
     // per-stage profiling (tfmoe_profile_enable)
     bool profiling = false;
+    bool plain_order = false;       // launch every kernel in plain stream order (stage replays)
     cudaEvent_t prof_ev[TFMOE_STAGE_COUNT][2] = {};
     bool prof_used[TFMOE_STAGE_COUNT] = {};
     float prof_ms[TFMOE_STAGE_COUNT] = {};

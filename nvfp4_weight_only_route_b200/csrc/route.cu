@@ -547,30 +547,34 @@ __device__ void plan_block(const int32_t *__restrict__ ids, int P, const PlanArg
     int32_t *off = tot + E;          // [E+1]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (P <= (int)blockDim.x && P <= W * E) {
-        // small batches: one thread per pair; the count comes from shared atomics and the
-        // stable rank from the earlier pairs with the same expert, read from a shared copy
-        int32_t *ids_s = cnt;
+        // small batches: one thread per pair. Warp w holds pairs 32w .. 32w+31; its lanes
+        // with the same expert find each other with match_any, the first of them records
+        // the warp's count of that expert, and a pair's stable rank is its rank inside the
+        // warp plus the counts of the earlier warps.
+        for (int i = threadIdx.x; i < W * E; i += blockDim.x) cnt[i] = 0;
         for (int e = threadIdx.x; e < E; e += blockDim.x) tot[e] = 0;
-        for (int i = threadIdx.x; i < P; i += blockDim.x) ids_s[i] = ids[i];
         __syncthreads();
         const int p = threadIdx.x;
         int e = -1;
         if (p < P) {
-            e = ids_s[p];
+            e = ids[p];
             if (e >= E || e < 0) {
                 if (pa.debug) atomicOr(pa.err_word, DEV_ERR_BAD_EXPERT);
                 e = -1;
-            } else {
-                atomicAdd(&tot[e], 1);
             }
+        }
+        const uint32_t same = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && lane == __ffs(same) - 1) {
+            cnt[warp * E + e] = __popc(same);
+            atomicAdd(&tot[e], __popc(same));
         }
         __syncthreads();
         if (warp == 0) scan_experts_warp(tot, off, E);
         __syncthreads();
         for (int i = threadIdx.x; i <= E; i += blockDim.x) pa.offsets[i] = off[i];
         if (e >= 0) {
-            int rank = 0;
-            for (int q = 0; q < p; ++q) rank += (ids_s[q] == e);
+            int rank = __popc(same & ((1u << lane) - 1u));
+            for (int w = 0; w < warp; ++w) rank += cnt[w * E + e];
             const int r = off[e] + rank;
             pa.perm[r] = p;
             pa.inv[p] = r;
