@@ -112,11 +112,36 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def code_only(text: str) -> str:
+    """C/CUDA source with comments, trailing blanks and empty lines removed (string literals kept)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"':                                   # string literal, escapes included
+            j = i + 1
+            while j < n and text[j] != '"':
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return "\n".join(l.rstrip() for l in "".join(out).splitlines() if l.strip())
+
+
 def kernel_source_hash(stage: str = "gemv_gate_up"):
+    """Hash of the code (not the comments) of the stage's kernel file + common.cuh + internal.h."""
     h = hashlib.sha256()
     files = ("mma.cu",) if stage.startswith("mma") else ("gemv.cu",)
     for f in files + ("common.cuh", "internal.h"):
-        h.update(open(os.path.join(ROOT, "nvfp4_weight_only_route_b200", "csrc", f), "rb").read())
+        src = open(os.path.join(ROOT, "nvfp4_weight_only_route_b200", "csrc", f), encoding="utf-8").read()
+        h.update(code_only(src).encode())
     return h.hexdigest()[:16]
 
 

@@ -7,10 +7,14 @@
 // compute-bound"); the expert up/down kernels are the largest share of decode
 // GPU time in TensorFold issue #627 (comment with the RTX 4090 per-launch
 // table). So the kernel is built around the memory stream: the packed codes
-// arrive with 128-bit coalesced loads, double-buffered in registers across
-// column chunks and prefetched across tasks; each task's E4M3 block scales
-// arrive in shared memory with one 2-D tensor copy (TMA) issued a task ahead;
-// the inner loop spends about one instruction per weight and token.
+// arrive with 128-bit coalesced loads (16-byte cp.async per lane) into a
+// per-warp shared-memory ring that runs two 4-tile chunks ahead, across passes
+// and tasks; each task's E4M3 block scales arrive in shared memory with one
+// 2-D tensor copy (TMA), and each pass's activation rows with bulk copies,
+// both issued two passes ahead by a control warp. Per weight and token the
+// inner loop spends one mixed-precision FMA and half an E2M1 conversion; the
+// addresses are 32-bit shared-memory bases with immediate offsets, so little
+// else is issued.
 //
 // Task = (expert of the GEMV list, 16*RG consecutive weight rows). The 8 warps
 // of a CTA split it as RG row groups x KS column slices (RG * KS = 8): lane l
@@ -20,7 +24,9 @@
 // slices), added in a fixed order; then the epilogue threads (one per row and
 // token) apply the per-tensor scale and either SwiGLU (gate/up) or the fp32
 // store (down). Tasks are small so that the few waves of a decode step stay
-// balanced across the CTAs.
+// balanced across the CTAs; when a batch gives every CTA several tasks, the
+// down projection switches to longer ones (fewer column slices, more tiles per
+// warp and pass).
 //
 // Arithmetic: the activation operand is an f16 tensor with one power of two
 // per 16 elements (exact for every bf16 element within 2^28 of its block's
@@ -296,10 +302,11 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
 }
 
 // CTA = 8 compute warps + 1 control warp. The compute warps only stream codes and
-// do arithmetic: they never wait for one another. The control warp runs one pass
-// ahead issuing the tensor/bulk copies of scales and activation rows, and one pass
-// behind adding the compute warps' partial sums (in slice order) and storing the
-// outputs, so no warp holds a CTA-wide barrier per pass.
+// do arithmetic: they never wait for one another. The control warp issues the
+// tensor/bulk copies of scales and activation rows two passes ahead (pass p+2's as
+// soon as pass p's partial sums are in) and runs one pass behind adding the compute
+// warps' partial sums (in slice order) and storing the outputs, so no warp holds a
+// CTA-wide barrier per pass.
 //
 // Barriers (parity = use count / 2 mod 2, every barrier alternating between 2 buffers):
 //   sfull[b]  scales of task #i landed (b = i & 1; expect-tx by the control warp)
