@@ -180,8 +180,18 @@ def test_forward_host_matches_device(oracle_mod):
         dev = run.forward(x, intermediates=False)["out"]
         xh = torch.from_numpy(x.view(np.int16)).pin_memory()
         oh = torch.empty((8, s.H), dtype=torch.int16).pin_memory()
-        run.layer.forward_host(xh, oh)
+        stream = torch.cuda.Stream()
+        run.layer.forward_host(xh, oh, stream=stream)
         assert np.array_equal(oh.numpy().view(np.uint16), dev)
+        # another input (pageable buffers), then the first again: no state leaks between calls
+        x2 = synth.make_x(s, 11, 8)
+        dev2 = run.forward(x2, intermediates=False)["out"]
+        oh2 = torch.empty((8, s.H), dtype=torch.int16)
+        run.layer.forward_host(torch.from_numpy(x2.view(np.int16)), oh2, stream=stream)
+        assert np.array_equal(oh2.numpy().view(np.uint16), dev2)
+        run.layer.forward_host(xh, oh, stream=stream)
+        assert np.array_equal(oh.numpy().view(np.uint16), dev)
+        assert run.layer.last_launch_count() > 0
     finally:
         run.close()
 
