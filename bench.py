@@ -156,6 +156,50 @@ def ncu_traffic(workload: str, stage: str):
     return ent.get("dram_bytes_per_launch")
 
 
+def work_per_forward(mean_active: float, T: int, H: int, I: int, E: int, k: int):
+    """Algorithmic bytes and FLOPs of one forward: the active experts' NVFP4 weights read
+    once (3 H I weights each), the bf16 router weights, x in and out; expert and router FLOPs.
+    The intermediates and the routing state are implementation traffic, not counted."""
+    nbytes = mean_active * 3 * H * I * NVFP4_BYTES_PER_WEIGHT + E * H * 2 + T * H * 2 * 2
+    flops = 2.0 * T * k * 3 * H * I + 2.0 * T * H * E
+    return nbytes, flops
+
+
+def roofline_for(kernel: str, us: float, H: int, I: int, gemv_experts: float, mma_pairs: float, mma_experts: float,
+                 hbm_peak: float, bf16_peak: float, measured: bool, traffic, how: str) -> dict:
+    """The roofline object of the dominant kernel from its average launch time `us`.
+    GEMV launches read gemv_experts x rows x K weights (HBM bound). A tensor-core launch
+    does 2 x pairs x rows x K FLOPs on mma_experts x rows x K weights; its bound follows
+    its arithmetic intensity against the ratio of the measured peaks."""
+    hbm_src = "measured (MEASURED_PEAKS.json hbm_gbs)" if measured else "fallback"
+    if kernel in ("gemv_gate_up", "gemv_down"):
+        alg = gemv_experts * (2 * I * H if kernel == "gemv_gate_up" else H * I) * NVFP4_BYTES_PER_WEIGHT
+        achieved = alg / (us * 1e-6) / 1e9
+        return {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": traffic, "algorithmic_bytes_per_launch": alg,
+                "avg_launch_us": us, "peak_source": hbm_src, "how": how}
+    if kernel in ("mma_gate_up", "mma_down"):
+        rows = 2 * I if kernel == "mma_gate_up" else H
+        kdim = H if kernel == "mma_gate_up" else I
+        flops = 2.0 * mma_pairs * rows * kdim
+        wbytes = mma_experts * rows * kdim * NVFP4_BYTES_PER_WEIGHT
+        t_s = us * 1e-6
+        if wbytes > 0 and flops / wbytes < (bf16_peak * 1e12) / (hbm_peak * 1e9):
+            achieved = wbytes / t_s / 1e9
+            return {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": achieved / hbm_peak, "traffic": traffic, "algorithmic_bytes_per_launch": wbytes,
+                    "algorithmic_flops_per_launch": flops, "avg_launch_us": us, "peak_source": hbm_src,
+                    "how": how}
+        achieved = flops / t_s / 1e12
+        return {"bound": "tensor", "kernel": kernel, "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
+                "frac": achieved / bf16_peak, "traffic": traffic, "algorithmic_flops_per_launch": flops,
+                "algorithmic_bytes_per_launch": wbytes, "avg_launch_us": us,
+                "peak_source": "measured (MEASURED_PEAKS.json bf16_tflops, burst)" if measured else "fallback",
+                "how": how}
+    return {"bound": "hbm", "kernel": kernel, "achieved": None, "peak": hbm_peak, "unit": "GB/s", "frac": None,
+            "traffic": traffic, "avg_launch_us": us}
+
+
 def oracle_cpu_sample(shape, layers, xs, seconds: float):
     """Time the fp64 oracle on whole decode batches (or single tokens for big shapes)."""
     from oracle import oracle
@@ -343,9 +387,7 @@ def main():
         gemv_experts.append(int(np.sum(reg == 1)))
     mean_active = float(np.mean(active))
     mean_gemv = float(np.mean(gemv_experts))
-    weight_bytes_expert = 3 * H * I * NVFP4_BYTES_PER_WEIGHT
-    bytes_per_fwd = mean_active * weight_bytes_expert + E * H * 2 + T * H * 2 * 2
-    flops_per_fwd = 2.0 * T * k * 3 * H * I + 2.0 * T * H * E
+    bytes_per_fwd, flops_per_fwd = work_per_forward(mean_active, T, H, I, E, k)
 
     # ---- CUDA graphs of consecutive forwards, all captured before timing. Each graph
     # starts at input index 0 and holds a whole number of input cycles when it can.
@@ -455,44 +497,9 @@ def main():
     dominant = max(kernel_us, key=kernel_us.get)
     how = (f"median of 5 replays of a graph of back-to-back launches rotating {len(layers)} layer(s), "
            "CUDA events on the launch stream")
-    if dominant in ("gemv_gate_up", "gemv_down"):
-        rows = 2 * I * H if dominant == "gemv_gate_up" else H * I
-        alg = float(np.mean(gemv_units)) * rows * NVFP4_BYTES_PER_WEIGHT
-        achieved = alg / (kernel_us[dominant] * 1e-6) / 1e9
-        roofline = {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                    "frac": achieved / hbm_peak, "traffic": ncu_traffic(args.workload, dominant),
-                    "algorithmic_bytes_per_launch": alg, "avg_launch_us": kernel_us[dominant],
-                    "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback",
-                    "how": how}
-    elif dominant in ("mma_gate_up", "mma_down"):
-        # the tensor-core kernel's bound follows its arithmetic intensity: FLOPs per weight
-        # byte against the ratio of the measured peaks (a few tokens per expert stream
-        # weights, hundreds of tokens per expert keep the tensor pipe busy)
-        rows = 2 * I if dominant == "mma_gate_up" else H
-        kdim = H if dominant == "mma_gate_up" else I
-        flops = 2.0 * float(np.mean(mma_pairs)) * rows * kdim
-        wbytes = float(np.mean(mma_units)) * rows * kdim * NVFP4_BYTES_PER_WEIGHT
-        t_s = kernel_us[dominant] * 1e-6
-        if wbytes > 0 and flops / wbytes < (bf16_peak * 1e12) / (hbm_peak * 1e9):
-            achieved = wbytes / t_s / 1e9
-            roofline = {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                        "frac": achieved / hbm_peak, "traffic": ncu_traffic(args.workload, dominant),
-                        "algorithmic_bytes_per_launch": wbytes, "algorithmic_flops_per_launch": flops,
-                        "avg_launch_us": kernel_us[dominant],
-                        "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback",
-                        "how": how}
-        else:
-            achieved = flops / t_s / 1e12
-            roofline = {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": bf16_peak,
-                        "unit": "TFLOP/s", "frac": achieved / bf16_peak, "traffic": ncu_traffic(args.workload, dominant),
-                        "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": wbytes,
-                        "avg_launch_us": kernel_us[dominant],
-                        "peak_source": ("measured (MEASURED_PEAKS.json bf16_tflops, burst)" if peak_src == "measured"
-                                        else "fallback"),
-                        "how": how}
-    else:
-        roofline = {"bound": "hbm", "kernel": dominant, "achieved": None, "peak": hbm_peak, "unit": "GB/s",
-                    "frac": None, "traffic": ncu_traffic(args.workload, dominant), "avg_launch_us": kernel_us[dominant]}
+    roofline = roofline_for(dominant, kernel_us[dominant], H, I, float(np.mean(gemv_units)),
+                            float(np.mean(mma_pairs)), float(np.mean(mma_units)), hbm_peak, bf16_peak,
+                            peak_src == "measured", ncu_traffic(args.workload, dominant), how)
 
     # ---- per-stage times of ordinary (profiled, host-synchronised) forwards; these include
     # host launch gaps and are reported for orientation only
