@@ -21,7 +21,7 @@
 // reduction in stages of 64. One persistent CTA per SM, 20 warps:
 //   warp 0       producer of the token tiles (TMA, 128-byte swizzle, box 64 x N)
 //                into a 5-stage ring that the MMA commit frees
-//   warp 2       producer of the 4 KB code tiles + 2 x 256 B scales (bulk copies)
+//   warp 2       producer of the 4 KB code tiles + their 512 B scale slabs (bulk copies)
 //                into a 16-stage ring that the decoders free once they have read it
 //   warp 1       allocates tensor memory; lane 0 issues the MMAs and commits. Each
 //                tcgen05.mma costs the issuing thread ~100 cycles whatever N is, so
