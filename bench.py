@@ -156,6 +156,11 @@ def ncu_traffic(workload: str, stage: str):
     return ent.get("dram_bytes_per_launch")
 
 
+def workload_label(name: str, H: int, I: int, E: int, k: int, T: int, seeds) -> str:
+    """config.workload of both arms: the workload named by what it is, with its sizes."""
+    return f"{name}: H={H} I={I} E={E} top-{k} T={T} tokens/forward, seeds {list(seeds)} rotated"
+
+
 def work_per_forward(mean_active: float, T: int, H: int, I: int, E: int, k: int):
     """Algorithmic bytes and FLOPs of one forward: the active experts' NVFP4 weights read
     once (3 H I weights each), the bf16 router weights, x in and out; expert and router FLOPs.
@@ -288,8 +293,9 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{args.workload}: H={shape.H} I={shape.I} E={shape.E} top-{shape.k} T={T}, seeds {list(seeds)}",
-                   "reference": "fp64 CPU oracle, one token of the workload per step"},
+        "config": {"workload": workload_label(args.workload, shape.H, shape.I, shape.E, shape.k, T, seeds),
+                   "global_batch": T, "parallelism": "single GPU",
+                   "reference": "fp64 CPU oracle on the host cores, one token of the workload per step"},
         "cpu_baseline": {"value": value, "unit": "tok/s", "cores": oracle.max_threads(), "kind": "oracle",
                          "sample": f"{args.steps} steps of one token each"},
         "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -545,8 +551,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16 activations, nvfp4 weights, fp32 accumulate", "data": "synthetic",
-            "config": {"workload": f"{args.workload}: H={H} I={I} E={E} top-{k} T={T} tokens/forward, "
-                                   f"seeds {list(seeds)} rotated", "global_batch": T * world,
+            "config": {"workload": workload_label(args.workload, H, I, E, k, T, seeds), "global_batch": T * world,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2: rotating seeded layers / full weight sets exceed 126 MB",
                        "flags": args.flags, "gemv_max_tokens": args.gemv_max_tokens or "default",

@@ -63,3 +63,9 @@ def test_other_kernels_report_no_fraction():
     b = _load_bench()
     r = b.roofline_for("combine", 3.0, 2048, 768, 0, 0, 0, 6555.5, 1636.3, True, None, "t")
     assert r["frac"] is None and r["achieved"] is None and r["avg_launch_us"] == 3.0
+
+
+def test_both_arms_name_the_workload_alike():
+    b = _load_bench()
+    assert (b.workload_label("decode", 2048, 768, 128, 8, 8, (1, 2, 3))
+            == "decode: H=2048 I=768 E=128 top-8 T=8 tokens/forward, seeds [1, 2, 3] rotated")
