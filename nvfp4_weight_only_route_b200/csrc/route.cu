@@ -802,7 +802,7 @@ static PlanArgs plan_args(const Layer &L, int T) {
     return pa;
 }
 
-bool route_fused_applies(const Layer &L, int T) { return T <= kFusedMaxT; }
+bool route_fused_applies(const Layer &, int T) { return T <= kFusedMaxT; }
 
 static bool large_plan(const Layer &L, int T) {
     return T > kFusedMaxT && (long long)T * L.desc.top_k > kLargePlanPairs;
