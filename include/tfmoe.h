@@ -65,6 +65,11 @@ typedef struct tfmoe_layer tfmoe_layer;   /* opaque */
 #define TFMOE_FLAG_FORCE_GEMV    0x1u  /* every expert uses the CUDA-core GEMV regime */
 #define TFMOE_FLAG_FORCE_MMA     0x2u  /* every expert uses the tcgen05 tensor-core regime */
 #define TFMOE_FLAG_DEBUG_CHECKS  0x4u  /* kernels bounds-check ids/rows and set the error word */
+/* Test aid for the failure path: in every forward that runs the GEMV gate/up kernel,
+ * one thread of its first CTA waits 1 ms on a barrier that nothing completes and then
+ * takes the timeout path (error word, abort). That forward's output is undefined;
+ * tfmoe_sync_status reports TFMOE_ERR_TIMEOUT. Not for production use. */
+#define TFMOE_FLAG_TEST_TIMEOUT  0x8u
 
 /*
  * Layer shape. Requirements (else TFMOE_ERR_INVALID_ARG):

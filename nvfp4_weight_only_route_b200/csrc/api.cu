@@ -153,7 +153,7 @@ tfmoe_status tfmoe_create(const tfmoe_layer_desc *desc, tfmoe_layer **out)
     if (d.max_tokens <= 0) return fail(TFMOE_ERR_INVALID_ARG, "max_tokens (%d) must be >= 1", d.max_tokens);
     if ((d.flags & TFMOE_FLAG_FORCE_GEMV) && (d.flags & TFMOE_FLAG_FORCE_MMA))
         return fail(TFMOE_ERR_INVALID_ARG, "FORCE_GEMV and FORCE_MMA are exclusive");
-    if (d.flags & ~(TFMOE_FLAG_FORCE_GEMV | TFMOE_FLAG_FORCE_MMA | TFMOE_FLAG_DEBUG_CHECKS))
+    if (d.flags & ~(TFMOE_FLAG_FORCE_GEMV | TFMOE_FLAG_FORCE_MMA | TFMOE_FLAG_DEBUG_CHECKS | TFMOE_FLAG_TEST_TIMEOUT))
         return fail(TFMOE_ERR_INVALID_ARG, "unknown flag bits 0x%x", d.flags);
     if (d.hidden % 128 || d.intermediate % 64)
         return fail(TFMOE_ERR_UNSUPPORTED, "this build needs hidden %% 128 == 0 and intermediate %% 64 == 0 (got %d, %d)",

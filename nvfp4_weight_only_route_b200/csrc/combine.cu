@@ -7,9 +7,6 @@
 #include "common.cuh"
 #include "internal.h"
 
-#ifndef TFMOE_COMBINE_EARLY
-#define TFMOE_COMBINE_EARLY 1
-#endif
 
 namespace tfmoe {
 namespace {
@@ -62,7 +59,7 @@ cudaError_t launch_combine(Layer &L, int T, uint16_t *out, cudaStream_t s, int *
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = L.plain_order ? 0 : TFMOE_COMBINE_EARLY;
+    attr[0].val.programmaticStreamSerializationAllowed = L.plain_order ? 0 : 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, combine_kernel, (const float *)L.ws.y, (const float *)L.ws.topk_w,

@@ -47,23 +47,12 @@ namespace {
 constexpr int kWarps = 8;                       // compute warps (column slices x row groups)
 constexpr int kComputeWarps = kWarps;
 constexpr int kThreads = (kComputeWarps + 1) * 32;   // + the control warp
-#ifndef TFMOE_GEMV_CTAS_PER_SM
-#define TFMOE_GEMV_CTAS_PER_SM 2
-#endif
-constexpr int kCtasPerSm = TFMOE_GEMV_CTAS_PER_SM;
-#ifndef TFMOE_GEMV_RING
-#define TFMOE_GEMV_RING 3
-#endif
-#ifndef TFMOE_GEMV_CHUNK
-#define TFMOE_GEMV_CHUNK 4
-#endif
-#ifndef TFMOE_GEMV_DOWN_EARLY
-#define TFMOE_GEMV_DOWN_EARLY 1
-#endif
-constexpr int kChunk = TFMOE_GEMV_CHUNK;   // column tiles per ring slot of a compute warp
-constexpr int kRing = TFMOE_GEMV_RING;   // ring slots per compute warp (kRing - 1 chunks in flight)
+constexpr int kCtasPerSm = 2;
+constexpr int kChunk = 4;   // column tiles per ring slot of a compute warp
+constexpr int kRing = 3;    // ring slots per compute warp (kRing - 1 chunks in flight)
 static_assert(kRing >= 2, "ring depth");
-constexpr int kMaxNT = 2;   // tokens per pass (the partial sums of a pass are one f32 pair per lane)
+constexpr int kMaxNT = 2;
+constexpr uint32_t kTestWaitNs = 1000000;   // the forced-timeout test's wait: 1 ms   // tokens per pass (the partial sums of a pass are one f32 pair per lane)
 
 enum class Proj { GateUp, Down };
 
@@ -91,6 +80,7 @@ struct GemvArgs {
     float *y_out;               // Down output [P][H]
     int I;
     int32_t *err_word;
+    uint32_t test_wait_ns;      // > 0: CTA 0 first waits this long on a barrier nothing completes
 };
 
 struct Geometry {
@@ -102,12 +92,8 @@ struct Geometry {
 // Each projection has two task shapes: the default one (more, shorter tasks) and a
 // long one (each warp streams more column tiles per pass, so the per-pass costs are
 // spread over more weights), used when the batch gives every CTA enough tasks.
-#ifndef TFMOE_GEMV_GU_LONG_KS
-#define TFMOE_GEMV_GU_LONG_KS 4
-#endif
-#ifndef TFMOE_GEMV_DOWN_LONG_KS
-#define TFMOE_GEMV_DOWN_LONG_KS 2
-#endif
+constexpr int kGateUpLongKS = 4;     // column slices of the long gate/up task shape
+constexpr int kDownLongKS = 2;       // column slices of the long down task shape
 constexpr int kLongTasksPerCta = 4;   // the long shape needs this many tasks per CTA (estimated)
 Geometry geometry_from(int ks_start, int K) {
     const int KT = K / kTileK;
@@ -126,7 +112,8 @@ Geometry geometry(bool gate_up, int K) {
 // the task's scales [KT][16*RG] u32, the partial sums [KS][16*RG][kMaxNT] f32, the
 // pass's activation rows [kMaxNT][K] f16 and their inverse scales [kMaxNT][K/16] f32;
 // the GEMV list table [5][<= 256] (expert, first row, rows, per-tensor scales); per compute warp a ring of kRing code chunks
-// (kChunk tiles x 32 lanes x 16 bytes); 8 mbarriers and an abort flag.
+// (kChunk tiles x 32 lanes x 16 bytes); 8 mbarriers, an abort flag and a barrier that
+// nothing completes (the forced-timeout test).
 constexpr int kMaxList = 256;
 struct SmemLayout {
     size_t sc_sz, red_sz, x_sz, xi_sz;
@@ -143,7 +130,7 @@ struct SmemLayout {
         tab = xi + 2 * xi_sz;
         ring = tab + 5 * kMaxList * 4;
         bar = ring + (size_t)kComputeWarps * kRing * kChunk * 32 * 16;
-        total = bar + 9 * sizeof(uint64_t);
+        total = bar + 10 * sizeof(uint64_t);
     }
 };
 size_t gemv_smem_bytes(int K, Geometry g) { return 128 + SmemLayout(K, g.KS, g.RG).total; }
@@ -341,6 +328,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + lay.bar);
     uint64_t *sfull = bars, *xfull = bars + 2, *full = bars + 4, *rfree = bars + 6;
     volatile int32_t *abort_flag = reinterpret_cast<volatile int32_t *>(bars + 8);
+    uint64_t *never = bars + 9;                           // no thread ever arrives on it
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -350,6 +338,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
             mbar_init(&full[i], kComputeWarps);
             mbar_init(&rfree[i], 1);
         }
+        mbar_init(never, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -398,8 +387,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     if (warp == kComputeWarps) {
         // ------------------------------------------------------------ control warp
         const uint32_t scale_tx = (uint32_t)(KT * rows_task * 4);
-        int last_s = -1, last_x = -1;                 // barriers of the latest copies issued
-        uint32_t last_s_par = 0, last_x_par = 0;
+        // per buffer: whether a copy was issued into it and the phase parity of the latest
+        // one. A buffer is refilled only after every compute warp waited for (or, aborting,
+        // gave up on) its previous copy, and after an abort nothing is issued, so each of
+        // the four barriers has at most one phase in flight: its latest.
+        bool s_used[2] = {false, false}, x_used[2] = {false, false};
+        uint32_t s_par[2] = {0u, 0u}, x_par[2] = {0u, 0u};
         auto issue = [&](const Cursor &c, int t0, int tn, int p, bool first) {
             int r_begin;
             const int m = task_rows(c, r_begin);
@@ -416,8 +409,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
                     mbar_arrive_expect_tx(&sfull[sb], scale_tx);
                     tma_load_2d(sbuf(sb), &smap, row0 % kTileRows, (tab[c.li] * RT + row0 / kTileRows) * KT,
                                 &sfull[sb]);
-                    last_s = sb;
-                    last_s_par = (tn >> 1) & 1;
+                    s_used[sb] = true;
+                    s_par[sb] = (tn >> 1) & 1;
                 }
             }
             // the down pass reads aq, which the gate/up grid writes: wait for that grid here,
@@ -428,8 +421,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
             }
             if (lane == 0) {
                 mbar_arrive_expect_tx(&xfull[xb], (uint32_t)nt * (uint32_t)(K * 2 + K / 4));
-                last_x = xb;
-                last_x_par = (p >> 1) & 1;
+                x_used[xb] = true;
+                x_par[xb] = (p >> 1) & 1;
             }
             for (int t = 0; t < nt; ++t) {
                 const int rr = __shfl_sync(0xffffffffu, row, t);
@@ -447,7 +440,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
         bool ivalid = first_pass(ic);
         int it0 = 0, itn = 0, ip = 0;
         auto issue_next = [&](bool first) {
-            if (!ivalid) return;
+            // after an abort no copy is issued: a compute warp may have stopped waiting for
+            // the copy that last filled the buffer (its arrive on full[] publishes the flag)
+            if (!ivalid || *abort_flag) return;
             int rb;
             const int m = task_rows(ic, rb);
             issue(ic, it0, itn, ip, first);
@@ -518,10 +513,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
                 }
             }
         }
-        // after an abort, let the latest copies land before the CTA exits (bounded)
+        // after an abort, let every copy still in flight land before the CTA exits (bounded)
         if (lane == 0 && *abort_flag) {
-            if (last_s >= 0) mbar_wait_bounded(&sfull[last_s], last_s_par, a.err_word);
-            if (last_x >= 0) mbar_wait_bounded(&xfull[last_x], last_x_par, a.err_word);
+            for (int b = 0; b < 2; ++b) {
+                if (s_used[b]) mbar_wait_bounded(&sfull[b], s_par[b], a.err_word);
+                if (x_used[b]) mbar_wait_bounded(&xfull[b], x_par[b], a.err_word);
+            }
         }
         return;
     }
@@ -599,6 +596,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
     for (int i = 0; i < kRing - 1; ++i) refill();
     // weights only so far; the bounded waits below start after the gate/up grid is done
     if (P == Proj::Down && has_work) grid_dep_wait();
+    // forced-timeout test: one thread of CTA 0 waits a short time on a barrier that nothing
+    // completes, then takes the timeout path (error word, abort flag) like any other wait
+    if (a.test_wait_ns && blockIdx.x == 0 && warp == 0) {
+        if (lane == 0) {
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait_sleep(never, 0u)) {
+                if (global_timer_ns() - t0 > a.test_wait_ns) {
+                    atomicOr(a.err_word, DEV_ERR_WAIT_TIMEOUT);
+                    *abort_flag = 1;
+                    break;
+                }
+            }
+        }
+        __syncwarp();
+    }
 
     uint32_t use = 0;
     int p = 0, tn = 0;
@@ -676,9 +688,9 @@ cudaError_t gemv_setup(Layer &L)
     GemvMaps *gm = new (std::nothrow) GemvMaps();
     if (!gm) return cudaErrorMemoryAllocation;
     gm->gu[0].g = geometry(true, H);
-    gm->gu[1].g = geometry_from(TFMOE_GEMV_GU_LONG_KS, H);
+    gm->gu[1].g = geometry_from(kGateUpLongKS, H);
     gm->down[0].g = geometry(false, I);
-    gm->down[1].g = geometry_from(TFMOE_GEMV_DOWN_LONG_KS, I);
+    gm->down[1].g = geometry_from(kDownLongKS, I);
     // scale slabs viewed as [E * RT * KT][128 rows] of u32; a task's box is 16*RG rows x all KT slabs
     const uint64_t slabs_gu = (uint64_t)E * (2 * I / kTileRows) * (H / kTileK);
     const uint64_t slabs_d = (uint64_t)E * (H / kTileRows) * (I / kTileK);
@@ -720,6 +732,7 @@ static GemvArgs common_args(const Layer &L) {
     g.expert_list = L.ws.gemv_list; g.list_size = L.ws.list_sizes;
     g.offsets = L.ws.offsets; g.perm = L.ws.perm; g.top_k = L.desc.top_k;
     g.I = L.desc.intermediate; g.err_word = L.ws.err_word;
+    g.test_wait_ns = 0;
     return g;
 }
 
@@ -736,6 +749,7 @@ cudaError_t launch_gemv_gate_up(Layer &L, const uint16_t *x, int T, cudaStream_t
     g.KS = sh.g.KS; g.RG = sh.g.RG;
     g.src = L.ws.xq; g.src_inv = L.ws.xq_inv;
     g.act_out = L.ws.act; g.aq_out = L.ws.aq; g.aq_inv_out = L.ws.aq_inv;
+    if (L.desc.flags & TFMOE_FLAG_TEST_TIMEOUT) g.test_wait_ns = kTestWaitNs;
     gemv_kernel<Proj::GateUp><<<sh.grid, kThreads, sh.smem, s>>>(sh.map, g);
     *launches += 1;
     return cudaGetLastError();
@@ -760,7 +774,7 @@ cudaError_t launch_gemv_down(Layer &L, int T, cudaStream_t s, int *launches)
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = L.plain_order ? 0 : TFMOE_GEMV_DOWN_EARLY;
+    attr[0].val.programmaticStreamSerializationAllowed = L.plain_order ? 0 : 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_kernel<Proj::Down>, sh.map, d);

@@ -36,7 +36,8 @@
 //                memory into 16-byte row pieces, fp32 store for down.
 // Tensor memory: accumulators at columns [0,176) and [176,352), five A stages of
 // 32 columns from 352. Every wait is bounded; on a timeout the CTA records
-// the error, stops issuing work, lets issued copies land, frees tensor memory.
+// the error and stops issuing work; before it exits its issued copies land and
+// its issued MMAs complete (a final commit), and only then is tensor memory freed.
 #include <cuda.h>
 
 #include <new>
@@ -82,6 +83,7 @@ struct MmaSmem {
     uint64_t full[C::kStages], empty[C::kStages], aready[C::kStages];
     uint64_t cfull[C::kCStages], cempty[C::kCStages];
     uint64_t dfull[2], dempty[2];
+    uint64_t mma_done;                        // the issuer's last commit: every MMA of the CTA complete
     uint32_t tmem_base;
     int32_t abort_flag;
 };
@@ -105,21 +107,6 @@ struct MmaArgs {
     int I;
     int32_t *err_word;
 };
-
-#ifdef TFMOE_MMA_STATS
-// Instrumented build only: cycles each role spends in barrier waits, per CTA.
-constexpr int kStatSlots = 12;
-__device__ unsigned long long g_mma_stats[160][kStatSlots];
-#define STAT_WAIT(slot, expr)                                                              \
-    ([&]() {                                                                               \
-        const long long _t0 = clock64();                                                   \
-        const bool _r = (expr);                                                            \
-        atomicAdd(&g_mma_stats[blockIdx.x % 160][slot], (unsigned long long)(clock64() - _t0)); \
-        return _r;                                                                         \
-    }())
-#else
-#define STAT_WAIT(slot, expr) (expr)
-#endif
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, int32_t *abort_flag, int32_t *err) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -236,6 +223,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
             mbar_init(&sm.dfull[b], 1);
             mbar_init(&sm.dempty[b], 128 * C::kEpiGroups);
         }
+        mbar_init(&sm.mma_done, 1);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
@@ -248,9 +236,6 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-#ifdef TFMOE_MMA_STATS
-    const long long t_kernel0 = clock64();
-#endif
 
     if (warp == 0 || warp == 2) {
         // warp 0: token tiles into the 8-stage ring (freed by the MMA commit);
@@ -269,11 +254,11 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
                     const int s = g % nst;
                     const uint32_t ph = (g / nst) & 1u;
                     if (tokens) {
-                        if (!STAT_WAIT(0, wait_or_abort(&sm.empty[s], ph ^ 1u, &sm.abort_flag, a.err_word))) break;
+                        if (!wait_or_abort(&sm.empty[s], ph ^ 1u, &sm.abort_flag, a.err_word)) break;
                         mbar_arrive_expect_tx(&sm.full[s], b_bytes);
                         tma_load_2d(sm.b[s], &maps.box[bi], kt * kTileK, row0, &sm.full[s]);
                     } else {
-                        if (!STAT_WAIT(1, wait_or_abort(&sm.cempty[s], ph ^ 1u, &sm.abort_flag, a.err_word))) break;
+                        if (!wait_or_abort(&sm.cempty[s], ph ^ 1u, &sm.abort_flag, a.err_word)) break;
                         mbar_arrive_expect_tx(&sm.cfull[s], kTileCodeBytes + kTileScaleBytes);
                         bulk_g2s(sm.codes[s], a.codes + (rti * KT + kt) * kTileCodeBytes, kTileCodeBytes, &sm.cfull[s]);
                         bulk_g2s(sm.scales[s], a.scales + scale_offset(rti, KT, kt), kTileScaleBytes, &sm.cfull[s]);
@@ -301,17 +286,14 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
                 const int rows = __ldg(a.entries + 4 * (t / RT) + 2);
                 const uint32_t idesc = instr_desc_16bit(box_rows<C>(box_index<C>(rows)), kType);
                 const int buf = tile_i & 1;
-                if (!STAT_WAIT(2, wait_or_abort(&sm.dempty[buf], ((tile_i >> 1) & 1u) ^ 1u, &sm.abort_flag, a.err_word))) break;
+                if (!wait_or_abort(&sm.dempty[buf], ((tile_i >> 1) & 1u) ^ 1u, &sm.abort_flag, a.err_word)) break;
                 tc_fence_after();
                 const uint32_t dt = tmem + (uint32_t)buf * kMaxN;
                 bool ok = true;
                 for (int kt = 0; kt < KT; ++kt, ++g) {
                     const int s = g % kStages;
                     const uint32_t ph = (g / kStages) & 1u;
-                    if (!STAT_WAIT(4, wait_or_abort(&sm.aready[s], ph, &sm.abort_flag, a.err_word))) { ok = false; break; }
-#ifdef TFMOE_MMA_STATS
-                    const long long tm0 = clock64();
-#endif
+                    if (!wait_or_abort(&sm.aready[s], ph, &sm.abort_flag, a.err_word)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t bd = bdesc0 + (uint64_t)(s * (kBStageBytes >> 4));
                     const uint32_t ad = tmem + kACol + (uint32_t)s * 32u;
@@ -319,19 +301,14 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
                     mma_16bit_ts(dt, ad + 8u, bd + 2u, idesc, 1u);
                     mma_16bit_ts(dt, ad + 16u, bd + 4u, idesc, 1u);
                     mma_16bit_ts(dt, ad + 24u, bd + 6u, idesc, 1u);
-#ifdef TFMOE_MMA_STATS
-                    const long long tm1 = clock64();
-#endif
                     mma_commit(&sm.empty[s]);
-#ifdef TFMOE_MMA_STATS
-                    const long long tm2 = clock64();
-                    g_mma_stats[blockIdx.x % 160][10] += (unsigned long long)(tm1 - tm0);
-                    g_mma_stats[blockIdx.x % 160][11] += (unsigned long long)(tm2 - tm1);
-#endif
                 }
                 if (!ok) break;
                 mma_commit(&sm.dfull[buf]);
             }
+            // on every path, including an abort: tensor memory and the operand stages stay
+            // in use until the MMAs already issued complete, which this commit reports
+            mma_commit(&sm.mma_done);
         }
     } else if (warp >= kDqWarp0 && warp < kEpiWarp0) {
         // decode: warpgroup gq takes the stages g with g % kDqGroups == gq (all 64 columns), so
@@ -346,15 +323,13 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
                 if ((int)(g % C::kDqGroups) != gq) continue;
                 const int s = g % kStages, cs = g % kCStages;
                 const uint32_t ph = (g / kStages) & 1u, pc = (g / kCStages) & 1u;
-                ok = (lane == 0) ? STAT_WAIT(5, wait_or_abort(&sm.cfull[cs], pc, &sm.abort_flag, a.err_word))
-                                 : wait_or_abort(&sm.cfull[cs], pc, &sm.abort_flag, a.err_word);
+                ok = wait_or_abort(&sm.cfull[cs], pc, &sm.abort_flag, a.err_word);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 const uint4 c0 = *reinterpret_cast<const uint4 *>(sm.codes[cs] + q * 16);
                 const uint4 c1 = *reinterpret_cast<const uint4 *>(sm.codes[cs] + 2048 + q * 16);
                 const uint32_t sc4 = *reinterpret_cast<const uint32_t *>(sm.scales[cs] + q * 4);
                 mbar_arrive(&sm.cempty[cs]);                              // code stage consumed
-                ok = (lane == 0) ? STAT_WAIT(6, wait_or_abort(&sm.empty[s], ph ^ 1u, &sm.abort_flag, a.err_word))
-                                 : wait_or_abort(&sm.empty[s], ph ^ 1u, &sm.abort_flag, a.err_word);  // A stage free
+                ok = wait_or_abort(&sm.empty[s], ph ^ 1u, &sm.abort_flag, a.err_word);   // A stage free
                 if (ok) ok = wait_or_abort(&sm.full[s], ph, &sm.abort_flag, a.err_word);             // token tile landed
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 const uint32_t s01 = e4m3x2_to_f16x2(sc4 & 0xFFFFu), s23 = e4m3x2_to_f16x2(sc4 >> 16);
@@ -379,9 +354,6 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
                 tc_wait_st();
                 tc_fence_before();
                 mbar_arrive(&sm.aready[s]);
-#ifdef TFMOE_MMA_STATS
-                if (lane == 0) atomicAdd(&g_mma_stats[blockIdx.x % 160][9], 1ull);
-#endif
             }
         }
     } else if (warp >= kEpiWarp0) {
@@ -397,9 +369,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
             const int rt = t % RT;
             const int n = box_rows<C>(box_index<C>(rows));
             const int buf = tile_i & 1;
-            if (!((lane == 0) ? STAT_WAIT(7, wait_or_abort(&sm.dfull[buf], (tile_i >> 1) & 1u, &sm.abort_flag, a.err_word))
-                              : wait_or_abort(&sm.dfull[buf], (tile_i >> 1) & 1u, &sm.abort_flag, a.err_word)))
-                break;
+            if (!wait_or_abort(&sm.dfull[buf], (tile_i >> 1) & 1u, &sm.abort_flag, a.err_word)) break;
             tc_fence_after();
             const int grow = rt * kM + q;
             const float gs = (P == Proj::GateUp) ? ((grow & 1) ? __ldg(a.glob1 + e) : __ldg(a.glob0 + e))
@@ -451,10 +421,8 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
         }
     }
     __syncthreads();
-#ifdef TFMOE_MMA_STATS
-    if (threadIdx.x == 0) atomicAdd(&g_mma_stats[blockIdx.x % 160][8], (unsigned long long)(clock64() - t_kernel0));
-#endif
     if (warp == 1) {
+        if (lane == 0) mbar_wait_bounded(&sm.mma_done, 0, a.err_word);
         __syncwarp();
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
@@ -629,15 +597,3 @@ cudaError_t launch_mma_down(Layer &L, cudaStream_t s, int *launches)
 }
 
 }  // namespace tfmoe
-
-#ifdef TFMOE_MMA_STATS
-extern "C" __attribute__((visibility("default"))) int tfmoe_debug_mma_stats(unsigned long long *out, int clear)
-{
-    if (cudaMemcpyFromSymbol(out, tfmoe::g_mma_stats, sizeof(tfmoe::g_mma_stats)) != cudaSuccess) return 1;
-    if (clear) {
-        static unsigned long long zeros[160][tfmoe::kStatSlots];
-        if (cudaMemcpyToSymbol(tfmoe::g_mma_stats, zeros, sizeof(zeros)) != cudaSuccess) return 1;
-    }
-    return 0;
-}
-#endif

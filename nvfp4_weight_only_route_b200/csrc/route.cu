@@ -721,11 +721,8 @@ __global__ void __launch_bounds__(256) plan_place_kernel(const int32_t *__restri
 // block is the launch-saving shape proposed in TensorFold issue #627 (comment
 // on the fused tf_nemo_route_row experiment).
 constexpr int kFusedMaxT = 16;
-#ifndef TFMOE_ROUTER_DMMA_MIN_TOKENS
-#define TFMOE_ROUTER_DMMA_MIN_TOKENS 128
-#endif
 // Batches of at least this many tokens take the router on the fp64 tensor cores.
-constexpr int kRouterDmmaMinTokens = TFMOE_ROUTER_DMMA_MIN_TOKENS;
+constexpr int kRouterDmmaMinTokens = 128;
 constexpr int kFusedThreads = 256;
 __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(
     const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, const float *__restrict__ bias,

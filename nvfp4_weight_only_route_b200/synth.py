@@ -91,8 +91,10 @@ def _rng(*key: int) -> np.random.Generator:
 
 
 def _random_bytes(rng: np.random.Generator, n: int) -> np.ndarray:
-    words = rng.bit_generator.random_raw((n + 7) // 8)
-    return words.view(np.uint8)[:n].copy()
+    # full-range 64-bit draws are the generator's raw outputs (the same stream as
+    # bit_generator.random_raw), produced without per-call overhead
+    words = rng.integers(0, np.iinfo(np.uint64).max, (n + 7) // 8, dtype=np.uint64, endpoint=True)
+    return words.view(np.uint8)[:n]
 
 
 def _bf16_bits_normal(rng: np.random.Generator, shape, std: float) -> np.ndarray:

@@ -21,6 +21,7 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "OOM", 3: "CUDA", 4: "NOT_LOADED",
 FLAG_FORCE_GEMV = 0x1
 FLAG_FORCE_MMA = 0x2
 FLAG_DEBUG_CHECKS = 0x4
+FLAG_TEST_TIMEOUT = 0x8
 
 BUF_LOGITS, BUF_TOPK_IDS, BUF_TOPK_WEIGHTS, BUF_EXPERT_COUNTS, BUF_EXPERT_OFFSETS, BUF_PERM, BUF_INV, \
     BUF_ACT, BUF_EXPERT_OUT, BUF_REGIME = range(10)

@@ -69,6 +69,9 @@ def lib():
         _lib.oracle_forward.restype = ctypes.c_int
         _lib.oracle_forward.argtypes = [ctypes.POINTER(_Layer), _u16p, ctypes.c_int32,
                                         ctypes.c_int32, ctypes.POINTER(_Outputs)]
+        _lib.oracle_route.restype = ctypes.c_int
+        _lib.oracle_route.argtypes = [ctypes.POINTER(_Layer), _u16p, ctypes.c_int32, ctypes.c_int32,
+                                      _f32p, _i32p, _f64p]
         _lib.oracle_max_threads.restype = ctypes.c_int
     return _lib
 
@@ -143,6 +146,29 @@ def forward(layer: Dict[str, Optional[np.ndarray]], x: np.ndarray, *, top_k: int
     if rc != 0:
         raise RuntimeError(f"oracle_forward failed with code {rc}")
     del keep, P
+    return res
+
+
+def route(layer: Dict[str, Optional[np.ndarray]], x: np.ndarray, *, top_k: int,
+          nthreads: int = 0) -> Dict[str, np.ndarray]:
+    """Routing alone (logits, ids, g) of every token of ``x`` (bf16 bits [T][H]): the
+    oracle's routing step, without the expert projections."""
+    E, H = layer["router_w"].shape
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    T = x.shape[0]
+    assert x.shape == (T, H)
+    rw = np.ascontiguousarray(layer["router_w"], dtype=np.uint16)
+    bias = None if layer.get("router_bias") is None else np.ascontiguousarray(layer["router_bias"], np.float32)
+    null8 = ctypes.cast(None, _u8p)
+    nullf = ctypes.cast(None, _f32p)
+    L = _Layer(H, 16, E, top_k, _ptr(rw, _u16p), _ptr(bias, _f32p), null8, null8, null8, null8, nullf, nullf,
+               null8, null8, nullf)
+    res = {"logits": np.zeros((T, E), np.float32), "ids": np.zeros((T, top_k), np.int32),
+           "g": np.zeros((T, top_k), np.float64)}
+    rc = lib().oracle_route(ctypes.byref(L), _ptr(x, _u16p), T, nthreads, _ptr(res["logits"], _f32p),
+                            _ptr(res["ids"], _i32p), _ptr(res["g"], _f64p))
+    if rc != 0:
+        raise RuntimeError(f"oracle_route failed with code {rc}")
     return res
 
 

@@ -293,4 +293,21 @@ int oracle_forward(const oracle_layer *L, const uint16_t *x, int32_t T, int32_t 
     return 0;
 }
 
+/* Routing alone: the router logits, top-k ids and softmax weights of every
+ * token, exactly as step 1 of oracle_forward computes them (the same
+ * route_token), without the expert projections. For checks of the routing of
+ * batches whose full forward would take the oracle too long. */
+int oracle_route(const oracle_layer *L, const uint16_t *x, int32_t T, int32_t nthreads,
+                 float *logits, int32_t *ids, double *g)
+{
+    if (!L || T < 0 || !logits || !ids || !g) return 1;
+    const int H = L->hidden, E = L->num_experts, k = L->top_k;
+    if (H <= 0 || E <= 0 || k <= 0 || k > E) return 1;
+    if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic, 4)
+    for (int t = 0; t < T; ++t)
+        route_token(L, x + (size_t)t * H, logits + (size_t)t * E, ids + (size_t)t * k, g + (size_t)t * k);
+    return 0;
+}
+
 int oracle_max_threads(void) { return omp_get_max_threads(); }
