@@ -1,22 +1,30 @@
 #!/usr/bin/env python
 """Throughput of the NVFP4 W4A16 MoE FFN layer forward (libtfmoe) on B200.
 
-Default workload (N=1): the decode layer shape -- H=2048, I=768, E=128, top-8,
-T=8 tokens per forward -- three seeded layers (seeds 1, 2, 3) rotated so that
-consecutive forwards read different weights (each forward touches ~137 MB; a
-layer is re-read only after two other layers' ~274 MB, which exceeds the
-126 MB L2). A step is one forward of the whole layer (router, top-k, permute,
-gate/up + SwiGLU, down, combine) over one batch; eight distinct seeded
-activation batches rotate per layer. Forwards are replayed from CUDA graphs of
-up to 100 consecutive forwards.
+Headline workload (N=1, the default): the large sparse-MoE layer -- H=4096,
+I=2688, E=256, top-8 (4.76 GB of NVFP4 expert weights per layer) -- at T=7234
+tokens per forward (the length of the 7,234-token prompt in the numbers table
+of the DGX Spark GB10 bandwidth-budget page). Five seeded layers (seeds 6..10)
+rotate, one forward each in turn; `value` is the median over the seeds of each
+seed's tokens/s. A step is one forward of the whole layer (router, top-k,
+permute, gate/up + SwiGLU, down, combine) over one batch. Every forward reads
+4.76 GB of weights, far more than the 126 MB L2.
+
+The same JSON line carries `per_config`: tokens/s, the layer's fraction of the
+HBM roofline (8 TB/s and the measured copy bandwidth) or of the bf16 tensor
+peak, the dominant kernel's roofline and the parity result for the tiny layer,
+decode T=1 and T=8, batched decode with Zipf load (T=256), prefill (T=8192) and
+the large sweep at T = 1, 32, 256, 2048 (N=1 only).
 
 Printed JSON line (rank 0): value = tokens/s over all ranks, e2e = the same
 metric through tfmoe_forward_host with pinned host buffers (copies inside the
 timed region), roofline of the dominant kernel measured live with CUDA events,
-cpu_baseline = the fp64 oracle on a bounded sample on this host's cores.
+cpu_baseline = the fp64 oracle on a bounded token sample of the same workload
+on this host's cores.
 
 --impl reference times the fp64 CPU oracle (the only reference this layer has)
-on the same workload, one token per step.
+on the same workload and the same kind of sample as cpu_baseline: each step is
+one oracle call on a fixed number of the workload's tokens.
 
 Multi-GPU (torchrun): replicas only -- every rank runs its own layers on its
 own GPU with no data-path collective (weak scaling); the timed region is
@@ -42,20 +50,43 @@ METRIC = "NVFP4 MoE layer tok/s; decode HBM GB/s, prefill TFLOP/s vs B200 peak"
 NVFP4_BYTES_PER_WEIGHT = 0.5625        # 4-bit code + one E4M3 byte per 16 weights
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+NOMINAL_HBM_GBS = 8000.0               # the ~8 TB/s the decode target is stated against
 
+SWEEP_SEEDS = (6, 7, 8, 9, 10)
 WORKLOADS = {
     # name: (layer shape index, tokens per forward, seeds)
-    "decode": (1, 8, (1, 2, 3)),
-    "decode_t1": (1, 1, (1, 2, 3)),
     "tiny": (0, 4, (0,)),
+    "decode_t1": (1, 1, (1, 2, 3)),
+    "decode": (1, 8, (1, 2, 3)),
     "zipf": (2, 256, (4,)),
     "prefill": (3, 8192, (5,)),
-    "sweep_t1": (4, 1, (6,)),
-    "sweep_t32": (4, 32, (6,)),
-    "sweep_t256": (4, 256, (6,)),
-    "sweep_t2048": (4, 2048, (6,)),
-    "sweep_t7234": (4, 7234, (6,)),
+    "sweep_t1": (4, 1, SWEEP_SEEDS),
+    "sweep_t32": (4, 32, SWEEP_SEEDS),
+    "sweep_t256": (4, 256, SWEEP_SEEDS),
+    "sweep_t2048": (4, 2048, SWEEP_SEEDS),
+    "sweep_t7234": (4, 7234, SWEEP_SEEDS),
 }
+HEADLINE = "sweep_t7234"
+PER_CONFIG = ["tiny", "decode_t1", "decode", "zipf", "prefill", "sweep_t1", "sweep_t32", "sweep_t256",
+              "sweep_t2048"]
+# Tokens of the workload per oracle call, for the CPU baseline and the reference arm.
+ORACLE_SAMPLE_TOKENS = {"tiny": 4, "decode_t1": 1, "decode": 8, "zipf": 16, "prefill": 8}
+
+
+def oracle_tokens_per_call(name: str) -> int:
+    return ORACLE_SAMPLE_TOKENS.get(name, 8)
+
+
+def regime_of(name: str) -> str:
+    """Which roofline a workload is held to: decode-shaped layers stream their active
+    weights (HBM), prefill-shaped ones are one large contraction (tensor); the
+    large sweep at T=2048 sits at the crossover and is reported against both."""
+    T = WORKLOADS[name][1]
+    if name == "prefill" or (name.startswith("sweep") and T >= 7234):
+        return "tensor"
+    if name.startswith("sweep") and T == 2048:
+        return "both"
+    return "hbm"
 
 
 def load_peaks():
@@ -205,23 +236,40 @@ def roofline_for(kernel: str, us: float, H: int, I: int, gemv_experts: float, mm
             "traffic": traffic, "avg_launch_us": us}
 
 
-def oracle_cpu_sample(shape, layers, xs, seconds: float):
-    """Time the fp64 oracle on whole decode batches (or single tokens for big shapes)."""
+def oracle_rate(layer_np, x_np, k: int, tokens_per_call: int, *, seconds: float = 0.0, calls: int = 0,
+                nthreads: int = 0, start: int = 0):
+    """Time the fp64 oracle on consecutive `tokens_per_call`-token slices of x_np (wrapping),
+    for at least `seconds` or exactly `calls` calls. Returns (tokens/s, calls, tokens, seconds)."""
     from oracle import oracle
     oracle.build()
-    tokens, n, t0 = 0, 0, time.perf_counter()
+    T = x_np.shape[0]
+    n = min(tokens_per_call, T)
+    done, tokens = 0, 0
+    t0 = time.perf_counter()
     while True:
-        L = layers[n % len(layers)]
-        x = xs[n % len(xs)]
-        if shape.H * shape.I * shape.k * x.shape[0] > 2 ** 27:
-            x = x[n % x.shape[0]: n % x.shape[0] + 1]
-        oracle.forward(L, x, top_k=shape.k)
-        tokens += x.shape[0]
-        n += 1
+        j = ((start + done) * n) % T
+        sl = x_np[j:j + n] if j + n <= T else np.concatenate([x_np[j:], x_np[:j + n - T]])
+        oracle.forward(layer_np, sl, top_k=k, nthreads=nthreads)
+        done += 1
+        tokens += n
         el = time.perf_counter() - t0
-        if el >= seconds:
+        if (calls and done >= calls) or (not calls and el >= seconds):
             break
-    return tokens / el, oracle.max_threads(), f"{n} oracle forwards, {tokens} tokens, {el:.1f} s"
+    return tokens / el, done, tokens, el
+
+
+def log(msg: str):
+    print(f"[bench {time.strftime('%H:%M:%S')}] {msg}", file=sys.stderr, flush=True)
+
+
+def cpu_description() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def dist_setup(n_gpus, backend: str = "nccl"):
@@ -266,21 +314,23 @@ def weak_value(world: int, tokens_per_step: int, steps: int, ms: float) -> float
 
 
 def run_reference(args):
+    """The reference arm: the fp64 CPU oracle on the same workload, rank 0 only."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     from nvfp4_weight_only_route_b200 import synth
     from oracle import oracle
     oracle.build()
-    shape_idx, T, seeds = WORKLOADS[args.workload]
+    name = args.workload or HEADLINE
+    shape_idx, T, seeds = WORKLOADS[name]
     shape = synth.SHAPES[shape_idx]
+    n = oracle_tokens_per_call(name)
     layers = [synth.make_layer(shape, s) for s in seeds]
-    xs = [synth.make_x(shape, s, T, stream=r) for s in seeds for r in range(2)]
+    xs = [synth.make_x(shape, s, T) for s in seeds]
 
     def step(i):
-        x = xs[i % len(xs)]
-        j = (i // len(xs)) % x.shape[0]
-        oracle.forward(layers[i % len(layers)], x[j:j + 1], top_k=shape.k)
+        li = i % len(layers)
+        oracle_rate(layers[li], xs[li], shape.k, n, calls=1, start=i // len(layers))
 
     for i in range(args.warmup):
         step(i)
@@ -288,292 +338,427 @@ def run_reference(args):
     for i in range(args.steps):
         step(args.warmup + i)
     el = time.perf_counter() - t0
-    value = args.steps / el
+    value = args.steps * min(n, T) / el
+    sample = (f"{args.steps} steps, each one oracle call on {min(n, T)} consecutive tokens of a T={T} batch, "
+              f"layers of seeds {list(seeds)} in turn")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_label(args.workload, shape.H, shape.I, shape.E, shape.k, T, seeds),
+        "config": {"workload": workload_label(name, shape.H, shape.I, shape.E, shape.k, T, seeds),
                    "global_batch": T, "parallelism": "single GPU",
-                   "reference": "fp64 CPU oracle on the host cores, one token of the workload per step"},
+                   "reference": "fp64 CPU oracle on the host cores"},
         "cpu_baseline": {"value": value, "unit": "tok/s", "cores": oracle.max_threads(), "kind": "oracle",
-                         "sample": f"{args.steps} steps of one token each"},
+                         "sample": sample, "cpu": cpu_description()},
         "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
 
 
+class Bench:
+    """Seeded layers on one GPU and the measurements made on them."""
+
+    def __init__(self, args, rank, world, local, pg):
+        import torch
+        from nvfp4_weight_only_route_b200 import synth, tfmoe
+        self.torch, self.synth, self.tfmoe = torch, synth, tfmoe
+        self.args, self.rank, self.world, self.pg = args, rank, world, pg
+        self.dev = torch.device("cuda", local)
+        self.stream = torch.cuda.Stream(device=self.dev)
+        self.hbm_peak, self.bf16_peak, self.bf16_sustained, self.peak_src = load_peaks()
+        self.layers = {}        # (shape index, seed) -> [host layer or None, MoELayer]
+        self.max_tokens = {}    # shape index -> the largest T any workload of this run uses
+        self.gen_s = 0.0
+
+    def plan(self, names):
+        for n in names:
+            si, T, _ = WORKLOADS[n]
+            self.max_tokens[si] = max(self.max_tokens.get(si, 0), T)
+
+    def layer(self, si, seed):
+        key = (si, seed)
+        if key not in self.layers:
+            shape = self.synth.SHAPES[si]
+            t0 = time.perf_counter()
+            lnp = self.synth.make_layer(shape, replica_seed(seed, self.rank))
+            L = self.tfmoe.MoELayer(shape.H, shape.I, shape.E, shape.k, self.max_tokens[si],
+                                    has_router_bias=lnp["router_bias"] is not None, flags=self.args.flags,
+                                    gemv_max_tokens=self.args.gemv_max_tokens)
+            L.load_weights(self.tfmoe.layer_to_device(lnp, self.dev))
+            self.torch.cuda.synchronize()
+            self.gen_s += time.perf_counter() - t0
+            self.layers[key] = [lnp, L]
+        return self.layers[key]
+
+    def slim(self, si, seed):
+        """Keep only the router of a host layer whose expert weights no check reads again."""
+        lnp = self.layers[(si, seed)][0]
+        for k in list(lnp):
+            if k not in ("router_w", "router_bias"):
+                lnp[k] = None
+
+    def inputs(self, name, n_x):
+        si, T, seeds = WORKLOADS[name]
+        shape = self.synth.SHAPES[si]
+        return [[self.torch.from_numpy(self.synth.make_x(shape, s, T, stream=r + 100 * self.rank).view(np.int16))
+                 .to(self.dev) for r in range(n_x)] for s in seeds]
+
+    def parity(self, name, Ls, lnps, xs, n_sample, sample_layers):
+        """Routing of every token against the oracle's routing step (bit-exact ids and
+        logits), the output on sampled tokens within the tolerance."""
+        from oracle import oracle
+        torch, tfmoe = self.torch, self.tfmoe
+        si, T, _ = WORKLOADS[name]
+        k, E = self.synth.SHAPES[si].k, self.synth.SHAPES[si].E
+        out = torch.empty((T, self.synth.SHAPES[si].H), dtype=torch.int16, device=self.dev)
+        worst = 0.0
+        for li, L in enumerate(Ls):
+            with torch.cuda.stream(self.stream):
+                tfmoe.check(L.forward_raw(xs[li][0].data_ptr(), T, out.data_ptr(), self.stream.cuda_stream))
+            self.stream.synchronize()
+            tfmoe.check(L.sync_status(self.stream))
+            x_np = xs[li][0].cpu().numpy().view(np.uint16)
+            ids_g = L.buffer_tensor(tfmoe.BUF_TOPK_IDS, torch.int32, (T, k)).cpu().numpy()
+            log_g = L.buffer_tensor(tfmoe.BUF_LOGITS, torch.float32, (T, E)).cpu().numpy()
+            r = oracle.route(lnps[li], x_np, top_k=k)
+            if not (np.array_equal(ids_g, r["ids"]) and np.array_equal(log_g, r["logits"])):
+                raise SystemExit(f"parity gate ({name}): routing differs from the oracle")
+            if li >= sample_layers:
+                continue
+            got = out.cpu().numpy().view(np.uint16)
+            idx = np.arange(T) if T <= n_sample else np.unique(np.linspace(0, T - 1, n_sample).astype(int))
+            ref = oracle.forward(lnps[li], x_np[idx], top_k=k, intermediates=False)
+            g64 = (got[idx].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            half_ulp = 0.5 * 2.0 ** (np.floor(np.log2(np.maximum(np.maximum(np.abs(g64), np.abs(ref["out64"])),
+                                                                 2.0 ** -126))) - 7)
+            tol = 4e-3 * ref["S"] + 1e-3 + half_ulp
+            err = np.abs(g64 - ref["out64"])
+            if not np.all(err <= tol):
+                raise SystemExit(f"parity gate ({name}): output outside tolerance (worst {float(np.max(err / tol)):.3f})")
+            worst = max(worst, float(np.max(err / tol)))
+        return (f"ok: ids and logits bit-exact for all {T} tokens x {len(Ls)} layer(s); output within "
+                f"4e-3*S+1e-3 on {min(T, n_sample)} sampled tokens x {min(len(Ls), sample_layers)} layer(s), "
+                f"worst |err|/tol {worst:.3f}")
+
+    def routing_stats(self, name, Ls, xs):
+        torch, tfmoe = self.torch, self.tfmoe
+        si, T, _ = WORKLOADS[name]
+        E = self.synth.SHAPES[si].E
+        out = torch.empty((T, self.synth.SHAPES[si].H), dtype=torch.int16, device=self.dev)
+        st = {"active": [], "gemv": [], "mma_pairs": [], "mma": []}
+        launches = 0
+        for li, L in enumerate(Ls):
+            for xb in xs[li]:
+                with torch.cuda.stream(self.stream):
+                    tfmoe.check(L.forward_raw(xb.data_ptr(), T, out.data_ptr(), self.stream.cuda_stream))
+                self.stream.synchronize()
+                launches = L.last_launch_count()
+                cnt = L.buffer_tensor(tfmoe.BUF_EXPERT_COUNTS, torch.int32, (E,)).cpu().numpy()
+                reg = L.buffer_tensor(tfmoe.BUF_REGIME, torch.int32, (E,)).cpu().numpy()
+                st["active"].append(int(np.sum(cnt > 0)))
+                st["gemv"].append(int(np.sum(reg == 1)))
+                st["mma_pairs"].append(int(np.sum(cnt[reg == 2])))
+                st["mma"].append(int(np.sum(reg == 2)))
+        return {k: float(np.mean(v)) for k, v in st.items()}, launches
+
+    def kernel_times(self, name, Ls, xs):
+        """Average launch time of each expert-path kernel: a CUDA graph of back-to-back
+        single-stage replays (tfmoe_forward_stage) rotating the layers, median of 5 replays."""
+        torch, tfmoe = self.torch, self.tfmoe
+        si, T, _ = WORKLOADS[name]
+        out = torch.empty((T, self.synth.SHAPES[si].H), dtype=torch.int16, device=self.dev)
+        s = self.stream
+        for li, L in enumerate(Ls):       # leave every layer's workspace holding input 0's routing
+            with torch.cuda.stream(s):
+                tfmoe.check(L.forward_raw(xs[li][0].data_ptr(), T, out.data_ptr(), s.cuda_stream))
+        s.synchronize()
+        kernel_us = {}
+        for stage in ("gemv_gate_up", "gemv_down", "gather", "mma_gate_up", "mma_down", "combine"):
+            sid = tfmoe.STAGE_ID[stage]
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            launched = 0
+            with torch.cuda.stream(s):
+                e0.record(s)
+                for li, L in enumerate(Ls):
+                    tfmoe.check(L.forward_stage_raw(sid, xs[li][0].data_ptr(), T, out.data_ptr(), s.cuda_stream))
+                    launched += L.last_launch_count()
+                e1.record(s)
+            s.synchronize()
+            if launched == 0:
+                continue
+            est_us = max(1.0, e0.elapsed_time(e1) * 1e3 / len(Ls))
+            reps = int(max(2, min(50, 5000.0 / est_us / len(Ls))))
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                for _ in range(reps):
+                    for li, L in enumerate(Ls):
+                        tfmoe.check(L.forward_stage_raw(sid, xs[li][0].data_ptr(), T, out.data_ptr(), s.cuda_stream))
+            for _ in range(3):      # the first replays of a new graph run slow; keep them out of the timing
+                g.replay()
+            s.synchronize()
+            samples = []
+            for _ in range(5):
+                with torch.cuda.stream(s):
+                    e0.record(s)
+                    g.replay()
+                    e1.record(s)
+                s.synchronize()
+                samples.append(e0.elapsed_time(e1) * 1e3 / (reps * len(Ls)))
+            kernel_us[stage] = float(np.median(samples))
+            del g
+        return kernel_us
+
+    def timed(self, name, Ls, xs, steps, warmup, graph, per_forward, clocks=False):
+        """Device time of `steps` forwards rotating layers (then inputs). With per_forward,
+        an event pair brackets every forward (large batches only) and per-layer mean times
+        come back too. Bracketed by barriers; the max over ranks is taken."""
+        torch, tfmoe = self.torch, self.tfmoe
+        si, T, _ = WORKLOADS[name]
+        s = self.stream
+        out = torch.empty((T, self.synth.SHAPES[si].H), dtype=torch.int16, device=self.dev)
+        n_x = len(xs[0])
+
+        def fwd(i):
+            L = Ls[i % len(Ls)]
+            x = xs[i % len(Ls)][(i // len(Ls)) % n_x]
+            tfmoe.check(L.forward_raw(x.data_ptr(), T, out.data_ptr(), s.cuda_stream))
+
+        cycle = len(Ls) * n_x
+        G = 0
+        if graph > 0 and not per_forward:
+            G = max(cycle, (graph // cycle) * cycle) if steps >= cycle else steps
+            G = min(G, steps)
+        graphs = {}
+
+        def make_graph(n):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                for j in range(n):
+                    fwd(j)
+            return g
+
+        def run(n, start, evs=None):
+            if G == 0:
+                with torch.cuda.stream(s):
+                    for j in range(n):
+                        if evs is not None:
+                            evs[j].record(s)
+                        fwd(start + j)
+                    if evs is not None:
+                        evs[n].record(s)
+                return
+            done = 0
+            while done < n:
+                m = min(G, n - done)
+                graphs[m].replay()
+                done += m
+
+        if G:
+            sizes = {G} if steps >= G else set()
+            if steps % G:
+                sizes.add(steps % G)
+            if warmup % G:
+                sizes.add(warmup % G)
+            for m in sorted(sizes):
+                graphs[m] = make_graph(m)
+                graphs[m].replay()          # the first replay of every graph happens before timing
+            s.synchronize()
+        run(warmup, 0)
+        s.synchronize()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)] if per_forward else None
+        sampler = ClockSampler(self.dev.index) if (clocks and self.rank == 0) else None
+        barrier(self.pg, torch)
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s):
+            ev0.record(s)
+            run(steps, warmup, evs)
+            ev1.record(s)
+        s.synchronize()
+        barrier(self.pg, torch)
+        clk = sampler.stop() if sampler else None
+        ms = max_over_ranks(self.pg, torch, ev0.elapsed_time(ev1))
+        per_layer = None
+        if per_forward:
+            per_layer = []
+            for li in range(len(Ls)):
+                ts = [evs[j].elapsed_time(evs[j + 1]) for j in range(steps) if (warmup + j) % len(Ls) == li]
+                per_layer.append(max_over_ranks(self.pg, torch, float(np.mean(ts))) if ts else None)
+        for g in graphs.values():
+            del g
+        graphs.clear()
+        return ms, per_layer, clk, G
+
+    def fractions(self, name, ms_per_fwd, stats):
+        si, T, _ = WORKLOADS[name]
+        sh = self.synth.SHAPES[si]
+        nbytes, flops = work_per_forward(stats["active"], T, sh.H, sh.I, sh.E, sh.k)
+        t = ms_per_fwd * 1e-3
+        gbs, tfl = nbytes / t / 1e9, flops / t / 1e12
+        d = {"algorithmic_bytes_per_forward": nbytes, "hbm_gbs": gbs, "hbm_frac_of_8tbs": gbs / NOMINAL_HBM_GBS,
+             "hbm_frac_of_measured": gbs / self.hbm_peak, "flops_per_forward": flops, "tflops": tfl,
+             "tensor_frac_of_measured": tfl / self.bf16_peak, "active_experts_mean": stats["active"],
+             "regime": regime_of(name)}
+        reg = regime_of(name)
+        if reg == "hbm":
+            d["target"], d["target_frac"] = "HBM roofline (8 TB/s) >= 0.70", d["hbm_frac_of_8tbs"]
+        elif reg == "tensor":
+            d["target"], d["target_frac"] = "bf16 tensor peak (measured) >= 0.50", d["tensor_frac_of_measured"]
+        else:
+            bind = max(d["hbm_frac_of_8tbs"], d["tensor_frac_of_measured"])
+            d["target"], d["target_frac"] = "the higher of the two (crossover)", bind
+        return d
+
+    def roofline(self, name, kernel_us, stats):
+        si, T, _ = WORKLOADS[name]
+        sh = self.synth.SHAPES[si]
+        dominant = max(kernel_us, key=kernel_us.get)
+        how = ("median of 5 replays of a CUDA graph of back-to-back single-stage launches rotating the workload's "
+               "layers, CUDA events on the launch stream")
+        return roofline_for(dominant, kernel_us[dominant], sh.H, sh.I, stats["gemv"], stats["mma_pairs"],
+                            stats["mma"], self.hbm_peak, self.bf16_peak, self.peak_src == "measured",
+                            ncu_traffic(name, dominant), how)
+
+    def measure(self, name, steps, warmup, graph, n_sample, sample_layers, clocks=False, target_s=None):
+        si, T, seeds = WORKLOADS[name]
+        entries = [self.layer(si, sd) for sd in seeds]
+        lnps, Ls = [e[0] for e in entries], [e[1] for e in entries]
+        n_x = 8 if T <= 256 else 2
+        xs = self.inputs(name, n_x)
+        parity = self.parity(name, Ls, lnps, xs, n_sample, sample_layers) if self.rank == 0 else "rank 0 only"
+        for sd in seeds[max(1, sample_layers):]:
+            self.slim(si, sd)
+        log(f"{name}: parity {parity}")
+        stats, launches = self.routing_stats(name, Ls, xs)
+        per_forward = T >= 1024
+        if target_s:        # size the timed run to about target_s of device time
+            ms1, _, _, _ = self.timed(name, Ls, xs, len(Ls) * n_x, 1, 0, False)
+            est = ms1 / (len(Ls) * n_x)
+            steps = int(max(len(Ls), min(4000, target_s * 1e3 / max(est, 1e-3))))
+        ms, per_layer, clk, G = self.timed(name, Ls, xs, steps, warmup, graph, per_forward, clocks)
+        if per_layer:
+            t_med = float(np.median([v for v in per_layer if v is not None]))
+            value = self.world * T / (t_med * 1e-3)
+        else:
+            t_med = ms / steps
+            value = weak_value(self.world, T, steps, ms)
+        kernel_us = self.kernel_times(name, Ls, xs)
+        res = {"workload": workload_label(name, self.synth.SHAPES[si].H, self.synth.SHAPES[si].I,
+                                          self.synth.SHAPES[si].E, self.synth.SHAPES[si].k, T, seeds),
+               "tok_s": value, "ms_per_forward": t_med, "forwards_timed": steps, "graph_forwards": G,
+               "layer": self.fractions(name, t_med, stats), "roofline": self.roofline(name, kernel_us, stats),
+               "kernel_us": kernel_us, "parity": parity, "launches_per_forward": launches,
+               "mma_pairs_mean": stats["mma_pairs"], "gemv_experts_mean": stats["gemv"]}
+        if per_layer:
+            res["per_seed_ms_per_forward"] = dict(zip([str(x) for x in seeds], per_layer))
+            res["value_is"] = "median over seeds of each seed's tokens/s"
+        return res, ms, clk, Ls, xs
+
+    def e2e(self, name, Ls, xs, steps):
+        torch = self.torch
+        si, T, _ = WORKLOADS[name]
+        H = self.synth.SHAPES[si].H
+        x_host = [xs[li][r].cpu().pin_memory() for li in range(len(Ls)) for r in range(min(len(xs[li]), 2))]
+        out_host = torch.empty((T, H), dtype=torch.int16).pin_memory()
+        barrier(self.pg, torch)
+        t0 = time.perf_counter()
+        for i in range(steps):
+            Ls[i % len(Ls)].forward_host(x_host[i % len(x_host)], out_host, T=T, stream=self.stream)
+        el = max_over_ranks(self.pg, torch, time.perf_counter() - t0)
+        return {"value": self.world * T * steps / el, "unit": "tok/s", "h2d_bytes_per_step": T * H * 2,
+                "d2h_bytes_per_step": T * H * 2, "steps": steps,
+                "how": "tfmoe_forward_host: pinned host x in, pinned host out, returns after the copy out"}
+
+    def cpu_baseline(self, name, seconds, one_thread: bool = False):
+        si, T, _ = WORKLOADS[name]
+        lnp = self.layers[(si, WORKLOADS[name][2][0])][0]
+        x_np = self.synth.make_x(self.synth.SHAPES[si], WORKLOADS[name][2][0], T)
+        n = oracle_tokens_per_call(name)
+        from oracle import oracle
+        v, calls, tokens, el = oracle_rate(lnp, x_np, self.synth.SHAPES[si].k, n, seconds=seconds)
+        d = {"value": v, "unit": "tok/s", "cores": oracle.max_threads(), "kind": "oracle", "cpu": cpu_description(),
+             "sample": f"{calls} oracle calls of {min(n, T)} consecutive tokens of the T={T} batch ({tokens} tokens, "
+                       f"{el:.1f} s)" + ("; tokens/s extrapolates to the full batch" if n < T else "")}
+        if one_thread:
+            v1, c1, t1, e1 = oracle_rate(lnp, x_np, self.synth.SHAPES[si].k, min(n, T), calls=1, nthreads=1)
+            d["one_thread"] = {"value": v1, "unit": "tok/s", "cores": 1,
+                               "sample": f"one oracle call of {min(n, T)} tokens ({e1:.1f} s)"}
+        return d
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tfmoe", "reference"], default="tfmoe")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=None,
+                    help=f"the timed workload (default {HEADLINE})")
     ap.add_argument("--flags", type=int, default=0, help="descriptor flags (1 = force GEMV, 2 = force MMA)")
     ap.add_argument("--gemv-max-tokens", type=int, default=0,
                     help="per-expert token count up to which the GEMV regime is used (0 = library default)")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--graph", type=int, default=100, help="forwards per CUDA graph (0 = no graphs)")
+    ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--graph", type=int, default=100, help="forwards per CUDA graph for small batches (0 = none)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
 
     import torch
-
-    from nvfp4_weight_only_route_b200 import synth, tfmoe
     rank, world, local, pg = dist_setup(args.gpus)
     torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    hbm_peak, bf16_peak, bf16_sustained, peak_src = load_peaks()
+    b = Bench(args, rank, world, local, pg)
+    name = args.workload or HEADLINE
+    per_config = (not args.no_per_config) and world == 1 and args.workload is None
+    b.plan([name] + (PER_CONFIG if per_config else []))
 
-    shape_idx, T, seeds = WORKLOADS[args.workload]
-    shape = synth.SHAPES[shape_idx]
-    H, I, E, k = shape.H, shape.I, shape.E, shape.k
-    n_x = 8 if T <= 256 else 2
-    layers_np, layers, xs = [], [], []
-    for s in seeds:
-        lnp = synth.make_layer(shape, replica_seed(s, rank))
-        layers_np.append(lnp)
-        L = tfmoe.MoELayer(H, I, E, k, T, has_router_bias=lnp["router_bias"] is not None, flags=args.flags,
-                           gemv_max_tokens=args.gemv_max_tokens)
-        L.load_weights(tfmoe.layer_to_device(lnp, dev))
-        layers.append(L)
-        xs.append([torch.from_numpy(synth.make_x(shape, s, T, stream=r + 100 * rank).view(np.int16)).to(dev)
-                   for r in range(n_x)])
-    torch.cuda.synchronize()
-    out = torch.empty((T, H), dtype=torch.int16, device=dev)
-    stream = torch.cuda.Stream(device=dev)
-
-    def fwd(i):
-        L = layers[i % len(layers)]
-        x = xs[i % len(layers)][(i // len(layers)) % n_x]
-        tfmoe.check(L.forward_raw(x.data_ptr(), T, out.data_ptr(), stream.cuda_stream))
-        return L
-
-    # ---- parity gate against the oracle (rank 0), sampled tokens for large T
-    parity = "skipped"
-    if rank == 0:
-        from oracle import oracle
-        worst = 0.0
-        for li, L in enumerate(layers):
-            with torch.cuda.stream(stream):
-                fwd(li)
-            stream.synchronize()
-            tfmoe.check(L.sync_status(stream))
-            got = out.cpu().numpy().view(np.uint16)
-            ids_g = L.buffer_tensor(tfmoe.BUF_TOPK_IDS, torch.int32, (T, k)).cpu().numpy()
-            x_np = xs[li][0].cpu().numpy().view(np.uint16)
-            idx = np.arange(T) if T <= 64 else np.unique(np.linspace(0, T - 1, 16).astype(int))
-            ref = oracle.forward(layers_np[li], x_np[idx], top_k=k, intermediates=True)
-            if not np.array_equal(ids_g[idx], ref["ids"]):
-                raise SystemExit("parity gate: routing differs from the oracle")
-            g64 = (got[idx].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-            half_ulp = 0.5 * 2.0 ** (np.floor(np.log2(np.maximum(np.maximum(np.abs(g64), np.abs(ref["out64"])), 2.0 ** -126))) - 7)
-            tol = 4e-3 * ref["S"] + 1e-3 + half_ulp
-            err = np.abs(g64 - ref["out64"])
-            if not np.all(err <= tol):
-                raise SystemExit(f"parity gate: output outside tolerance (worst {float(np.max(err / tol)):.3f})")
-            worst = max(worst, float(np.max(err / tol)))
-        parity = f"ok: ids bit-exact, worst |err|/tol {worst:.3f} on {len(layers)} layer(s)"
-
-    # ---- routing statistics for the algorithmic byte / flop counts
-    active, gemv_experts, launches_per_fwd = [], [], 0
-    n_inputs = len(layers) * n_x
-    for i in range(n_inputs):
-        with torch.cuda.stream(stream):
-            L = fwd(i)
-        stream.synchronize()
-        launches_per_fwd = L.last_launch_count()
-        cnt = L.buffer_tensor(tfmoe.BUF_EXPERT_COUNTS, torch.int32, (E,)).cpu().numpy()
-        reg = L.buffer_tensor(tfmoe.BUF_REGIME, torch.int32, (E,)).cpu().numpy()
-        active.append(int(np.sum(cnt > 0)))
-        gemv_experts.append(int(np.sum(reg == 1)))
-    mean_active = float(np.mean(active))
-    mean_gemv = float(np.mean(gemv_experts))
-    bytes_per_fwd, flops_per_fwd = work_per_forward(mean_active, T, H, I, E, k)
-
-    # ---- CUDA graphs of consecutive forwards, all captured before timing. Each graph
-    # starts at input index 0 and holds a whole number of input cycles when it can.
-    cycle = len(layers) * n_x
-    G = 0
-    if args.graph > 0:
-        G = max(cycle, (args.graph // cycle) * cycle) if args.steps >= cycle else args.steps
-        G = min(G, args.steps)
-    graphs = {}
-
-    def make_graph(n):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for j in range(n):
-                fwd(j)
-        return g
-
-    def run_steps(n, start):
-        if G == 0:
-            with torch.cuda.stream(stream):
-                for j in range(n):
-                    fwd(start + j)
-            return
-        done = 0
-        while done < n:
-            m = min(G, n - done)
-            graphs[m].replay()
-            done += m
-
-    if G:
-        sizes = {G} if args.steps >= G else set()
-        if args.steps % G:
-            sizes.add(args.steps % G)
-        w_full, w_rem = divmod(args.warmup, G)
-        if w_rem:
-            sizes.add(w_rem)
-        for m in sorted(sizes):
-            graphs[m] = make_graph(m)
-            graphs[m].replay()          # first replay of every graph happens before timing
-        stream.synchronize()
-    run_steps(args.warmup, 0)
-    stream.synchronize()
-
-    # ---- timed region
-    sampler = ClockSampler(local) if rank == 0 else None
-    barrier(pg, torch)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        ev0.record(stream)
-        run_steps(args.steps, args.warmup)
-        ev1.record(stream)
-    stream.synchronize()
-    barrier(pg, torch)
-    clocks = sampler.stop() if sampler else None
-    ms_local = ev0.elapsed_time(ev1)
-    ms = max_over_ranks(pg, torch, ms_local)
-    value = weak_value(world, T, args.steps, ms)
-
-    # ---- per-kernel timing for the roofline: one forward per layer on a known batch, then
-    # a CUDA graph that re-enqueues one stage of those forwards, rotating over the layers
-    # (so consecutive launches read different weights), timed with events on its stream.
-    gemv_units, mma_pairs, mma_units = [], [], []
-    for li, L in enumerate(layers):
-        with torch.cuda.stream(stream):
-            tfmoe.check(L.forward_raw(xs[li][0].data_ptr(), T, out.data_ptr(), stream.cuda_stream))
-        stream.synchronize()
-        reg = L.buffer_tensor(tfmoe.BUF_REGIME, torch.int32, (E,)).cpu().numpy()
-        cnt = L.buffer_tensor(tfmoe.BUF_EXPERT_COUNTS, torch.int32, (E,)).cpu().numpy()
-        gemv_units.append(int(np.sum(reg == 1)))
-        mma_pairs.append(int(np.sum(cnt[reg == 2])))
-        mma_units.append(int(np.sum(reg == 2)))
-    kernel_us = {}
-    for stage in ("gemv_gate_up", "gemv_down", "gather", "mma_gate_up", "mma_down", "combine"):
-        sid = tfmoe.STAGE_ID[stage]
-        # one launch per layer, timed once, sizes the graph to ~5 ms of work
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        launched = 0
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for li, L in enumerate(layers):
-                tfmoe.check(L.forward_stage_raw(sid, xs[li][0].data_ptr(), T, out.data_ptr(), stream.cuda_stream))
-                launched += L.last_launch_count()
-            e1.record(stream)
-        stream.synchronize()
-        if launched == 0:
-            continue
-        est_us = max(1.0, e0.elapsed_time(e1) * 1e3 / len(layers))
-        reps = int(max(2, min(50, 5000.0 / est_us / len(layers))))
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for r in range(reps):
-                for li, L in enumerate(layers):
-                    tfmoe.check(L.forward_stage_raw(sid, xs[li][0].data_ptr(), T, out.data_ptr(), stream.cuda_stream))
-        for _ in range(3):      # the first replays of a new graph run slow; keep them out of the timing
-            g.replay()
-        stream.synchronize()
-        samples = []
-        for _ in range(5):
-            with torch.cuda.stream(stream):
-                e0.record(stream)
-                g.replay()
-                e1.record(stream)
-            stream.synchronize()
-            samples.append(e0.elapsed_time(e1) * 1e3 / (reps * len(layers)))
-        kernel_us[stage] = float(np.median(samples))
-        del g
-    dominant = max(kernel_us, key=kernel_us.get)
-    how = (f"median of 5 replays of a graph of back-to-back launches rotating {len(layers)} layer(s), "
-           "CUDA events on the launch stream")
-    roofline = roofline_for(dominant, kernel_us[dominant], H, I, float(np.mean(gemv_units)),
-                            float(np.mean(mma_pairs)), float(np.mean(mma_units)), hbm_peak, bf16_peak,
-                            peak_src == "measured", ncu_traffic(args.workload, dominant), how)
-
-    # ---- per-stage times of ordinary (profiled, host-synchronised) forwards; these include
-    # host launch gaps and are reported for orientation only
-    prof_steps = min(args.steps, 100)
-    for L in layers:
-        L.profile(True)
-        L.profile_read(reset=True)
-    for i in range(prof_steps):
-        with torch.cuda.stream(stream):
-            fwd(i)
-    stage_ms = {}
-    for L in layers:
-        for name, (ms_tot, calls) in L.profile_read(reset=True).items():
-            a_, c_ = stage_ms.get(name, (0.0, 0))
-            stage_ms[name] = (a_ + ms_tot, c_ + calls)
-        L.profile(False)
-    stage_avg_us = {n: (v[0] / v[1] * 1e3 if v[1] else 0.0) for n, v in stage_ms.items()}
-    layer_gbs = bytes_per_fwd / (ms / args.steps * 1e-3) / 1e9
-    layer_tflops = flops_per_fwd / (ms / args.steps * 1e-3) / 1e12
-
-    # ---- end to end through the host-buffer entry point (pinned memory)
-    x_host = [xs[li][r].cpu().pin_memory() for li in range(len(layers)) for r in range(min(n_x, 2))]
-    out_host = torch.empty((T, H), dtype=torch.int16).pin_memory()
-    e2e_steps = min(args.steps, 500)
-    barrier(pg, torch)
-    t0 = time.perf_counter()
-    for i in range(e2e_steps):
-        L = layers[i % len(layers)]
-        L.forward_host(x_host[i % len(x_host)], out_host, T=T, stream=stream)
-    el = time.perf_counter() - t0
-    el = max_over_ranks(pg, torch, el)
-    e2e = {"value": world * T * e2e_steps / el, "unit": "tok/s", "h2d_bytes_per_step": T * H * 2,
-           "d2h_bytes_per_step": T * H * 2, "steps": e2e_steps}
+    log(f"headline {name}")
+    head, ms, clocks, Ls, xs = b.measure(name, args.steps, args.warmup, args.graph, n_sample=12, sample_layers=len(
+        WORKLOADS[name][2]), clocks=True)
+    e2e = b.e2e(name, Ls, xs, min(args.steps, 20 if WORKLOADS[name][1] > 256 else 500))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = oracle_cpu_sample(shape, layers_np, [x.cpu().numpy().view(np.uint16) for x in xs[0]],
-                                             args.cpu_seconds)
-        cpu = {"value": v, "unit": "tok/s", "cores": cores, "kind": "oracle", "sample": sample}
+        cpu = b.cpu_baseline(name, args.cpu_seconds)
+
+    pcs = None
+    if per_config and rank == 0:
+        pcs = {}
+        for pc in PER_CONFIG:
+            big = WORKLOADS[pc][1] > 256
+            r, _, _, _, _ = b.measure(pc, 0, 3, args.graph, n_sample=8 if big else 64, sample_layers=1,
+                                      target_s=0.3)
+            log(f"{pc}: {r['tok_s']:.0f} tok/s, {r['ms_per_forward'] * 1e3:.1f} us per forward")
+            if not args.no_cpu_baseline:
+                r["cpu_baseline"] = b.cpu_baseline(pc, 2.0, one_thread=pc in ("tiny", "decode_t1", "decode", "zipf"))
+            pcs[pc] = r
 
     if rank == 0:
+        si, T, seeds = WORKLOADS[name]
         line = {
-            "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+            "metric": METRIC, "value": head["tok_s"], "unit": "tok/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16 activations, nvfp4 weights, fp32 accumulate", "data": "synthetic",
-            "config": {"workload": workload_label(args.workload, H, I, E, k, T, seeds), "global_batch": T * world,
+            "config": {"workload": head["workload"], "global_batch": T * world,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "inputs larger than L2: rotating seeded layers / full weight sets exceed 126 MB",
-                       "flags": args.flags, "gemv_max_tokens": args.gemv_max_tokens or "default",
-                       "graph_forwards": G},
-            "roofline": roofline,
-            "layer": {"algorithmic_bytes_per_forward": bytes_per_fwd, "hbm_gbs": layer_gbs,
-                      "hbm_frac": layer_gbs / hbm_peak, "hbm_frac_of_8tbs": layer_gbs / 8000.0,
-                      "flops_per_forward": flops_per_fwd, "tflops": layer_tflops,
-                      "tensor_frac": layer_tflops / bf16_peak, "active_experts_mean": mean_active,
-                      "mma_pairs_mean": float(np.mean(mma_pairs)), "gemv_experts_mean": float(np.mean(gemv_units)),
-                      "kernel_us_graph": kernel_us, "stage_avg_us_profiled": stage_avg_us},
+                       "l2": "inputs larger than L2: every forward reads its layer's active weights "
+                             "(4.76 GB for the headline), and seeded layers rotate",
+                       "value": head.get("value_is", "tokens over the timed device time"),
+                       "flags": args.flags, "gemv_max_tokens": args.gemv_max_tokens or "default"},
+            "roofline": head["roofline"],
+            "layer": dict(head["layer"], kernel_us_graph=head["kernel_us"],
+                          per_seed_ms_per_forward=head.get("per_seed_ms_per_forward")),
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": launches_per_fwd * args.steps,
+            "gpu_launches": head["launches_per_forward"] * args.steps,
             "clocks": clocks,
-            "parity": parity,
+            "parity": head["parity"],
+            "per_config": pcs,
+            "setup_s": {"layers_generated_and_loaded": b.gen_s},
         }
         print(json.dumps(line), flush=True)
-    for g in graphs.values():
-        del g
-    graphs.clear()
-    for L in layers:
+    for _, L in b.layers.values():
         L.close()
     if pg is not None:
         pg.destroy_process_group()

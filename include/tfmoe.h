@@ -246,8 +246,11 @@ TFMOE_API tfmoe_status tfmoe_profile_read(tfmoe_layer *layer, float *ms_total, i
  * calls whose work overlaps on the GPU (two streams, or two host threads)
  * race on it and must be serialised by the caller. Each call overwrites every
  * logit it reads, so nothing needs clearing between calls.
- * The first call on each device looks up the array's device address with
- * that device current; make that first call before any stream capture.
+ * Each call made outside a stream capture looks up the array's device address
+ * in the current CUDA context (so a device reset, which may move the array,
+ * or another context on the device is followed); a call made during a capture
+ * uses the address found by the last uncaptured call in the same context and
+ * returns TFMOE_ERR_CUDA if there is none.
  *
  * Arguments (DEVICE pointers, caller-owned): x bf16 [T][hidden] and router_w
  * bf16 [num_experts][hidden], both 16-byte aligned; router_bias fp32

@@ -887,22 +887,74 @@ namespace {
 
 static __device__ __align__(256) float g_noalloc_logits[TFMOE_ROUTE_NOALLOC_MAX_LOGITS];
 
-// Device address of g_noalloc_logits per device ordinal, looked up once with
-// that device current (the host-side symbol is only a stand-in for it).
-constexpr int kNoAllocMaxDevices = 64;
+// Host code cannot use g_noalloc_logits as a device address: the symbol is a host-side
+// stand-in, and the array's device address belongs to one CUDA context (a device reset
+// reloads the module and may move it; another context on the same device has its own
+// copy). So every call made outside a stream capture looks the address up again with
+// cudaGetSymbolAddress and records it under the current context's unique id; a call
+// made during a capture (where that lookup is not allowed) uses the address recorded
+// for the current context, and fails if there is none.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+constexpr int kNoAllocSlots = 64;
 std::mutex g_noalloc_mutex;
-float *g_noalloc_ptr[kNoAllocMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kNoAllocSlots] = {};   // 0 = empty slot
+float *g_noalloc_ptr[kNoAllocSlots] = {};
+int g_noalloc_next = 0;
 
-cudaError_t noalloc_scratch(int device, float **out) {
+template <class Fn>
+Fn driver_fn(const char *name) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<Fn>(p);
+}
+
+// Unique id of the context current on this thread (0 if it cannot be found).
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id + 1;   // never 0
+}
+
+cudaError_t noalloc_scratch(cudaStream_t s, float **out) {
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[device]) {
-        void *p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_logits);
-        if (e != cudaSuccess) return e;
-        g_noalloc_ptr[device] = static_cast<float *>(p);
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
+        cudaGetLastError();                       // e.g. the legacy stream while another captures
+        cs = cudaStreamCaptureStatusActive;
     }
-    *out = g_noalloc_ptr[device];
-    return cudaSuccess;
+    if (cs == cudaStreamCaptureStatusNone) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_logits);   // also creates the context
+        if (e != cudaSuccess) return e;
+        const unsigned long long id = current_context_id();
+        if (id) {
+            int slot = -1;
+            for (int i = 0; i < kNoAllocSlots; ++i)
+                if (g_noalloc_ctx[i] == id) slot = i;
+            if (slot < 0) {
+                slot = g_noalloc_next;
+                g_noalloc_next = (g_noalloc_next + 1) % kNoAllocSlots;
+            }
+            g_noalloc_ctx[slot] = id;
+            g_noalloc_ptr[slot] = static_cast<float *>(p);
+        }
+        *out = static_cast<float *>(p);
+        return cudaSuccess;
+    }
+    const unsigned long long id = current_context_id();
+    for (int i = 0; id && i < kNoAllocSlots; ++i)
+        if (g_noalloc_ctx[i] == id) {
+            *out = g_noalloc_ptr[i];
+            return cudaSuccess;
+        }
+    return cudaErrorStreamCaptureUnsupported;
 }
 
 }  // namespace
@@ -933,15 +985,14 @@ extern "C" tfmoe_status tfmoe_route_noalloc(const uint16_t *x, int32_t T, int32_
         return record_error(TFMOE_ERR_INVALID_ARG, "tfmoe_route_noalloc: NULL buffer");
     if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(router_w)) & 15u)
         return record_error(TFMOE_ERR_INVALID_ARG, "tfmoe_route_noalloc: x and router_w must be 16-byte aligned");
-    int device = 0;
-    cudaError_t e = cudaGetDevice(&device);
-    if (e == cudaSuccess && (device < 0 || device >= kNoAllocMaxDevices))
-        return record_error(TFMOE_ERR_UNSUPPORTED, "tfmoe_route_noalloc: device ordinal %d too large", device);
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
     float *logits = nullptr;
-    if (e == cudaSuccess) e = noalloc_scratch(device, &logits);
+    cudaError_t e = noalloc_scratch(s, &logits);
+    if (e == cudaErrorStreamCaptureUnsupported)
+        return record_error(TFMOE_ERR_CUDA, "tfmoe_route_noalloc: first call in this context made during a stream "
+                            "capture; make one call outside capture first");
     if (e != cudaSuccess)
         return record_error(TFMOE_ERR_CUDA, "tfmoe_route_noalloc: scratch address: %s", cudaGetErrorString(e));
-    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
     if (T <= 2 * kSmallTokens) {
         const int warps = E * ((T + kSmallTokens - 1) / kSmallTokens);
         router_small_kernel<<<(warps + 3) / 4, 128, 0, s>>>(x, router_w, router_bias, logits, T, H, E, nullptr, 0);

@@ -1,12 +1,14 @@
-"""The allocation-free routing entry point (tfmoe_route_noalloc) matches the
-routing that tfmoe_forward produces (needs a GPU).
+"""The allocation-free routing entry point, tfmoe_route_noalloc (needs a GPU).
 
-It exists for callers that cannot allocate device memory -- a fixed memory
-pool owned by someone else, real-time loops that cannot afford cudaMalloc's
-latency or implicit synchronisation -- so it keeps its logits in a fixed array
-inside the library. This file is collected last on purpose: if it fails, a run
-stopped at the first failure has already run every other test. It must pass
-alone in a fresh process as well.
+Some callers of this library cannot allocate device memory: code running while
+another component owns the whole memory budget through a fixed pool, and
+real-time loops that cannot take cudaMalloc's latency or its implicit device
+synchronisation. For them the entry point keeps its router logits in a fixed
+array compiled into the library. Its ids and weights are checked here against
+the fp64 oracle's routing and against the routing tfmoe_forward computes, on
+two calls in a row. This file is collected last on purpose: if it fails, a run
+stopped at the first failure has already run every other test. It also passes
+alone in a fresh process.
 """
 import numpy as np
 import pytest
@@ -26,7 +28,7 @@ def torch_cuda():
     return torch
 
 
-def _reference_routing(torch, layer_np, shape, x_np):
+def _forward_routing(torch, layer_np, shape, x_np):
     """ids and weights from the regular entry point (tfmoe_forward's workspace)."""
     from nvfp4_weight_only_route_b200 import tfmoe
     T = x_np.shape[0]
@@ -57,18 +59,41 @@ def _noalloc_routing(torch, layer_np, shape, x_np):
     return ids.cpu().numpy(), w.cpu().numpy()
 
 
-def test_noalloc_routing_matches_forward_on_two_calls_in_a_row(torch_cuda):
+# (shape, seed, T): the tiny layer (E=8, top-2, no bias); the decode layer (no bias) at
+# T=1, 8 (the small-batch router kernel), 17 and 63 (partly filled 64-token tiles of the
+# tiled router kernel); the batched-decode layer with its Zipf router bias at T=256.
+CASES = [(0, 0, 4), (1, 1, 1), (1, 1, 8), (1, 2, 17), (1, 3, 63), (2, 4, 256)]
+
+
+@pytest.mark.parametrize("shape_idx,seed,T", CASES)
+def test_noalloc_routing_matches_oracle_and_forward_on_two_calls_in_a_row(torch_cuda, oracle_mod, shape_idx,
+                                                                          seed, T):
     torch = torch_cuda
-    cases = []
-    s2 = synth.SHAPES[2]                       # batched decode with a Zipf router bias, T=256
-    cases.append((synth.make_layer(s2, 4), s2, synth.make_x(s2, 4, 256)))
-    s1 = synth.SHAPES[1]                       # decode, T=8 (the small-T router kernel)
-    cases.append((synth.make_layer(s1, 1), s1, synth.make_x(s1, 1, 8)))
-    for layer_np, shape, x_np in cases:        # two calls in a row, different sizes and kernels
-        ids_ref, w_ref = _reference_routing(torch, layer_np, shape, x_np)
+    shape = synth.SHAPES[shape_idx]
+    layer_np = synth.make_layer(shape, seed)
+    x_np = synth.make_x(shape, seed, T)
+    ref = oracle_mod.route(layer_np, x_np, top_k=shape.k)
+    ids_fwd, w_fwd = _forward_routing(torch, layer_np, shape, x_np)
+    for _ in range(2):                        # the fixed array keeps the previous call's logits
         ids, w = _noalloc_routing(torch, layer_np, shape, x_np)
-        assert np.array_equal(ids, ids_ref)
-        assert np.max(np.abs(w.astype(np.float64) - w_ref)) <= 2e-6
+        assert np.array_equal(ids, ref["ids"]), "ids differ from the oracle's"
+        assert np.max(np.abs(w.astype(np.float64) - ref["g"])) <= 2e-6
+        assert np.array_equal(ids, ids_fwd), "ids differ from tfmoe_forward's"
+        assert np.max(np.abs(w.astype(np.float64) - w_fwd)) <= 2e-6
+
+
+def test_noalloc_ties_go_to_the_lower_expert(torch_cuda, oracle_mod):
+    torch = torch_cuda
+    shape = synth.custom_shape(256, 64, 8, 3, router_std=1.0)
+    layer_np = synth.make_layer(shape, 8)
+    rw = layer_np["router_w"].copy()
+    rw[2] = rw[6] = rw[1]                     # three identical router rows: exact ties
+    layer_np["router_w"] = rw
+    x_np = synth.make_x(shape, 8, 20)
+    ref = oracle_mod.route(layer_np, x_np, top_k=3)
+    assert any(len({1, 2, 6} & set(r.tolist())) >= 2 for r in ref["ids"]), "fixture should produce ties"
+    ids, w = _noalloc_routing(torch, layer_np, shape, x_np)
+    assert np.array_equal(ids, ref["ids"])
 
 
 def test_noalloc_rejects_batches_beyond_the_fixed_scratch(torch_cuda):
