@@ -180,8 +180,14 @@ __device__ __forceinline__ float block16_bf16_to_f16(const uint16_t *src, uint16
     return __int_as_float((127 - sh) << 23);
 }
 
-// z * sigmoid(z); exp and reciprocal on the special-function unit (relative error
-// ~1e-6, far below the bf16 rounding that follows). Large -z gives rcp(inf) = 0.
-__device__ __forceinline__ float silu_f32(float z) { return z * __frcp_rn(1.0f + __expf(-z)); }
+// z * sigmoid(z); exp and reciprocal each one special-function-unit instruction
+// (relative errors of a few ulp of fp32, far below the bf16 rounding that follows).
+// Large -z gives 1 / inf = 0.
+__device__ __forceinline__ float rcp_approx(float v) {
+    float r;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(v));
+    return r;
+}
+__device__ __forceinline__ float silu_f32(float z) { return z * rcp_approx(1.0f + __expf(-z)); }
 
 }  // namespace tfmoe

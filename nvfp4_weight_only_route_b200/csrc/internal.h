@@ -50,7 +50,7 @@ constexpr int kLargePlanPairs = 4096;
 // Tokens per tensor-core tile (the MMA N dimension): up to kMmaTileTokens with one CTA
 // per SM, or up to kMmaSmallTileTokens with two CTAs per SM when a batch averages at most
 // kMmaSmallMaxAvgTokens tokens per expert.
-constexpr int kMmaTileTokens = 176;
+constexpr int kMmaTileTokens = 256;
 constexpr int kMmaSmallTileTokens = 64;
 constexpr int kMmaSmallMaxAvgTokens = 64;
 __host__ __device__ constexpr size_t max_mma_entries(size_t P, size_t E) { return P / kMmaSmallTileTokens + E + 1; }

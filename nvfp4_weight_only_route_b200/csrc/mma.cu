@@ -17,25 +17,24 @@
 //            E2M1 -> f16 is one conversion, the scale one f16x2 multiply.
 //   down   : bf16 x bf16 -> fp32; the SwiGLU output a is a bf16 tensor already.
 //
-// Tile: 128 weight rows (MMA M) x N <= 176 token rows of one expert (MMA N), the
-// reduction in stages of 64. One persistent CTA per SM, 20 warps:
-//   warp 0       producer of the token tiles (TMA, 128-byte swizzle, box 64 x N)
-//                into a 5-stage ring that the MMA commit frees
+// Tile: 128 weight rows (MMA M) x N <= 256 token rows of one expert (MMA N, the
+// tile's tokens rounded up to 16), the reduction in stages of 64. One persistent CTA
+// per SM (big shape), 24 warps:
+//   warp 0       producer of the token tiles (TMA, 128-byte swizzle, box 64 x rows)
+//                into a 4-stage ring that the MMA commit frees
 //   warp 2       producer of the 4 KB code tiles + their 512 B scale slabs (bulk copies)
-//                into a 16-stage ring that the decoders free once they have read it
-//   warp 1       allocates tensor memory; lane 0 issues the MMAs and commits. Each
-//                tcgen05.mma costs the issuing thread ~100 cycles whatever N is, so
-//                tiles are as wide as a double-buffered accumulator allows (N = 176,
-//                ~90 cycles of tensor work per MMA) and the thread does one wait and
-//                one commit per stage.
-//   warps 4-7    decode the even stages, warps 8-11 the odd ones (all 64 columns):
+//                into a 12-stage ring that the decoders free once they have read it
+//   warp 1       allocates tensor memory; lane 0 issues the MMAs and commits: one wait
+//                and one commit per stage, four MMAs of K = 16 in between
+//   warps 4-15   three dequant warpgroups taking every third stage (all 64 columns):
 //                thread q of a warpgroup owns weight row q = tensor-memory lane q
-//   warps 12-19  epilogue, two warpgroups taking alternate 16-column steps of the
-//                accumulator one tile behind the MMAs: SwiGLU for interleaved
-//                gate/up rows (row 2j gate j, 2j+1 up j) staged through shared
-//                memory into 16-byte row pieces, fp32 store for down.
-// Tensor memory: accumulators at columns [0,176) and [176,352), five A stages of
-// 32 columns from 352. Every wait is bounded; on a timeout the CTA records
+//   warps 16-23  epilogue, two warpgroups taking alternate 16-column steps of the
+//                accumulator: SwiGLU for interleaved gate/up rows (row 2j gate j,
+//                2j+1 up j) staged through shared memory into 16-byte row pieces,
+//                fp32 store for down; the accumulator is handed back once read
+// Tensor memory: the accumulator at columns [0,256), four A stages of 32 columns
+// from 256. The small shape (two CTAs per SM, N <= 64) double-buffers its
+// accumulator instead. Every wait is bounded; on a timeout the CTA records
 // the error and stops issuing work; before it exits its issued copies land and
 // its issued MMAs complete (a final commit), and only then is tensor memory freed.
 #include <cuda.h>
@@ -51,28 +50,31 @@ namespace {
 constexpr int kM = 128;
 constexpr int kEpiCols = 16;               // accumulator columns per epilogue step
 
-// Kernel shapes. Big: one CTA per SM, token tiles of up to 176 rows (prefill). Small:
-// two CTAs per SM, token tiles of up to 64 rows (batched decode, tens of tokens per
-// expert). A single thread issues one tcgen05.mma per ~120 cycles whatever N is, and
+// Kernel shapes. Big: one CTA per SM, token tiles of up to 256 rows (prefill): an
+// expert's few hundred tokens take one tile, so its weights are decoded once, and the
+// MMAs are as wide as the instruction allows. The accumulator is single-buffered (256
+// columns; the other 256 hold the decoded weight stages): the epilogue drains it
+// before the next tile's first MMA. Small: two CTAs per SM, token tiles of up to 64
+// rows (batched decode, tens of tokens per expert), double-buffered accumulators.
 // MMAs issued from different CTAs of an SM overlap on the tensor core, so at small N
 // two issuing CTAs per SM nearly double the weight rate.
 //   warps 0, 2: token-tile and code producers; warp 1: TMEM owner and MMA issuer;
 //   warps kDqWarp0..: DqGroups dequant warpgroups; then EpiGroups epilogue warpgroups.
-template <int MaxN, int NumBoxes, int Stages, int CStages, int DqGroups, int EpiGroups, int CtasPerSm>
+template <int MaxN, int NumBoxes, int Stages, int CStages, int DqGroups, int EpiGroups, int CtasPerSm, int DBufs>
 struct MmaCfg {
     static constexpr int kMaxN = MaxN, kNumBoxes = NumBoxes, kStages = Stages, kCStages = CStages;
-    static constexpr int kDqGroups = DqGroups, kEpiGroups = EpiGroups, kCtasPerSm = CtasPerSm;
+    static constexpr int kDqGroups = DqGroups, kEpiGroups = EpiGroups, kCtasPerSm = CtasPerSm, kDBufs = DBufs;
     static constexpr int kDqWarp0 = 4, kEpiWarp0 = 4 + 4 * DqGroups;
     static constexpr int kThreads = 32 * (kEpiWarp0 + 4 * EpiGroups);
-    static constexpr uint32_t kACol = 2 * MaxN;      // accumulators at [0,N), [N,2N); A stages from 2N
+    static constexpr uint32_t kACol = DBufs * MaxN;  // accumulators at [b N, (b+1) N); A stages after them
     static constexpr uint32_t kTmemCols =
         (kACol + Stages * 32 <= 128) ? 128u : (kACol + Stages * 32 <= 256) ? 256u : 512u;
     static constexpr int kBStageBytes = MaxN * 128;  // N rows x 64 16-bit elements
     static_assert(kACol + Stages * 32 <= kTmemCols && kTmemCols * CtasPerSm <= 512, "tensor memory budget");
     static_assert(kBStageBytes % 1024 == 0, "token stages must stay 1 KB aligned");
 };
-using BigCfg = MmaCfg<kMmaTileTokens, 5, 5, 16, 2, 2, 1>;       // 640 threads, 512 TMEM columns
-using SmallCfg = MmaCfg<kMmaSmallTileTokens, 3, 4, 12, 2, 1, 2>; // 512 threads, 256 TMEM columns
+using BigCfg = MmaCfg<kMmaTileTokens, 5, 4, 12, 3, 2, 1, 1>;       // 768 threads, 512 TMEM columns
+using SmallCfg = MmaCfg<kMmaSmallTileTokens, 3, 4, 12, 2, 1, 2, 2>; // 512 threads, 256 TMEM columns
 
 template <class C>
 struct MmaSmem {
@@ -82,7 +84,7 @@ struct MmaSmem {
     uint16_t stage_out[4 * C::kEpiGroups][kEpiCols][16];   // per epilogue warp: 16 tokens x 16 outputs
     uint64_t full[C::kStages], empty[C::kStages], aready[C::kStages];
     uint64_t cfull[C::kCStages], cempty[C::kCStages];
-    uint64_t dfull[2], dempty[2];
+    uint64_t dfull[C::kDBufs], dempty[C::kDBufs];
     uint64_t mma_done;                        // the issuer's last commit: every MMA of the CTA complete
     uint32_t tmem_base;
     int32_t abort_flag;
@@ -192,6 +194,9 @@ __device__ __forceinline__ int box_index(int rows) {
     while (box_rows<C>(i) < rows && i < C::kNumBoxes - 1) ++i;
     return i;
 }
+// MMA N of a token tile of `rows` tokens: the rows rounded up to 16 (the box loaded
+// may be taller; its extra rows are not multiplied).
+__device__ __forceinline__ int mma_n(int rows) { return (rows + 15) & ~15; }
 
 template <class C, Proj P>
 __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const __grid_constant__ TokenMaps<C> maps,
@@ -219,7 +224,7 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
             mbar_init(&sm.cfull[c], 1);
             mbar_init(&sm.cempty[c], 128);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < C::kDBufs; ++b) {
             mbar_init(&sm.dfull[b], 1);
             mbar_init(&sm.dempty[b], 128 * C::kEpiGroups);
         }
@@ -284,9 +289,10 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
             uint32_t g = 0, tile_i = 0;
             for (int t = blockIdx.x; t < n_tiles && !sm.abort_flag; t += gridDim.x, ++tile_i) {
                 const int rows = __ldg(a.entries + 4 * (t / RT) + 2);
-                const uint32_t idesc = instr_desc_16bit(box_rows<C>(box_index<C>(rows)), kType);
-                const int buf = tile_i & 1;
-                if (!wait_or_abort(&sm.dempty[buf], ((tile_i >> 1) & 1u) ^ 1u, &sm.abort_flag, a.err_word)) break;
+                const uint32_t idesc = instr_desc_16bit(mma_n(rows), kType);
+                const int buf = (int)(tile_i % C::kDBufs);
+                const uint32_t use = tile_i / C::kDBufs;
+                if (!wait_or_abort(&sm.dempty[buf], (use & 1u) ^ 1u, &sm.abort_flag, a.err_word)) break;
                 tc_fence_after();
                 const uint32_t dt = tmem + (uint32_t)buf * kMaxN;
                 bool ok = true;
@@ -367,13 +373,13 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
             const int32_t *ent = a.entries + 4 * (t / RT);
             const int e = __ldg(ent), row0 = __ldg(ent + 1), rows = __ldg(ent + 2);
             const int rt = t % RT;
-            const int n = box_rows<C>(box_index<C>(rows));
-            const int buf = tile_i & 1;
-            if (!wait_or_abort(&sm.dfull[buf], (tile_i >> 1) & 1u, &sm.abort_flag, a.err_word)) break;
+            const int n = mma_n(rows);
+            const int buf = (int)(tile_i % C::kDBufs);
+            if (!wait_or_abort(&sm.dfull[buf], (tile_i / C::kDBufs) & 1u, &sm.abort_flag, a.err_word)) break;
             tc_fence_after();
             const int grow = rt * kM + q;
-            const float gs = (P == Proj::GateUp) ? ((grow & 1) ? __ldg(a.glob1 + e) : __ldg(a.glob0 + e))
-                                                 : __ldg(a.glob0 + e);
+            const float gs = __ldg(a.glob0 + e);                               // gate (or down) scale
+            const float gs_up = (P == Proj::GateUp) ? __ldg(a.glob1 + e) : 0.f;
             // this group's steps: group eg takes steps eg, eg + kEpiGroups, ...
             const int steps = n / kEpiCols;
             bool handed_back = false;
@@ -388,14 +394,24 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
                     handed_back = true;
                 }
                 if (P == Proj::GateUp) {
-                    // even lane 2i holds gate j = (grow >> 1), lane 2i+1 the up row of the same j;
-                    // stage a[16 tokens][16 j] in shared memory, then write 16-byte row pieces
-                    const float xi = (lane < kEpiCols && c + lane < rows) ? __ldg(a.row_inv_scale + row0 + c + lane) : 0.f;
+                    // even lane 2i holds gate row j of the step's 16 tokens, lane 2i+1 the up row of
+                    // the same j. The pair splits the work: the even lane takes tokens 0..7 of the
+                    // step, the odd lane tokens 8..15, each receiving its partner's values of those
+                    // tokens (one shuffle per token), so no lane idles through the SwiGLU. The a
+                    // values [16 tokens][16 j] are staged in shared memory, then written as 16-byte
+                    // row pieces.
+                    const float xi_src = (lane < kEpiCols && c + lane < rows) ? __ldg(a.row_inv_scale + row0 + c + lane) : 0.f;
+                    const bool odd = (lane & 1) != 0;
+                    const int half = odd ? 8 : 0;
 #pragma unroll
-                    for (int i = 0; i < kEpiCols; ++i) {
-                        const float v = __uint_as_float(d[i]) * gs * __shfl_sync(0xffffffffu, xi, i);
-                        const float other = __shfl_xor_sync(0xffffffffu, v, 1);
-                        if (!(lane & 1)) sm.stage_out[ew][i][lane >> 1] = float_to_bf16_bits_rn(silu_f32(v) * other);
+                    for (int i = 0; i < 8; ++i) {
+                        const float keep = __uint_as_float(odd ? d[i + 8] : d[i]);
+                        const float give = __uint_as_float(odd ? d[i] : d[i + 8]);
+                        const float got = __shfl_xor_sync(0xffffffffu, give, 1);
+                        const float xi = __shfl_sync(0xffffffffu, xi_src, i + half);
+                        const float gv = (odd ? got : keep) * (gs * xi);       // xi: an exact power of two
+                        const float uv = (odd ? keep : got) * (gs_up * xi);
+                        sm.stage_out[ew][half + i][lane >> 1] = float_to_bf16_bits_rn(silu_f32(gv) * uv);
                     }
                     __syncwarp();
                     // 16 tokens x 32 bytes: lane l writes token l/2, bytes 16*(l&1) .. +16

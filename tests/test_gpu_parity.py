@@ -362,3 +362,25 @@ def test_debug_checks_flag_non_finite_logits(oracle_mod, value):
             check_output(g["out"], o)
     finally:
         run.close()
+
+
+def test_handles_of_different_shapes_coexist(oracle_mod):
+    """Several handles of different layer shapes live in one process: one created later
+    with a smaller layer must not break launches of an earlier, larger one (per-kernel
+    settings such as the shared-memory limit are process-wide)."""
+    big_s = synth.custom_shape(H=512, I=1024, E=8, k=2, global_scale=0.05, router_std=1.0)
+    small_s = synth.custom_shape(H=128, I=64, E=4, k=1, global_scale=0.05, router_std=1.0)
+    big_l, small_l = synth.make_layer(big_s, 41), synth.make_layer(small_s, 42)
+    big = GpuRun(big_l, 512, 1024, 8, 2, 40, flags=REGIMES["gemv"])
+    small = GpuRun(small_l, 128, 64, 4, 1, 40, flags=REGIMES["gemv"])
+    try:
+        for T in (5, 33):
+            for run, layer, s in ((big, big_l, big_s), (small, small_l, small_s)):
+                x = synth.make_x(s, 40 + T, T)
+                g = run.forward(x)
+                o = oracle_mod.forward(layer, x, top_k=s.k, intermediates=True)
+                check_routing(g, o, s.E, s.k)
+                check_output(g["out"], o)
+    finally:
+        small.close()
+        big.close()
