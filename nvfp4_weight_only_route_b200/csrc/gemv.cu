@@ -81,9 +81,6 @@ struct GemvArgs {
     int I;
     int32_t *err_word;
     uint32_t test_wait_ns;      // > 0: CTA 0 first waits this long on a barrier nothing completes
-    const uint8_t *pf_codes;    // GateUp: the down projection's tiled codes, prefetched into L2 (or null)
-    const uint8_t *pf_scales;   //         and its scale slabs
-    uint32_t pf_code_bytes, pf_scale_bytes;   // per expert
 };
 
 struct Geometry {
@@ -174,26 +171,6 @@ __device__ __forceinline__ float2 e4m3_pair_at(uint32_t w, uint32_t sh) {
     uint32_t h2;
     asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}" : "=r"(h2) : "r"(w >> sh));
     return f16x2_to_float2(h2);
-}
-// Prefetch `bytes` (a multiple of 16, 16-byte aligned address) of global memory into L2.
-__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-constexpr uint32_t kPrefetchChunk = 32768;
-// The down projection's weights of the GEMV-list entries li = blockIdx.x, + gridDim.x, ...
-// into L2, in 32 KB pieces spread over the lanes of the calling warp. The decode step's
-// gate/up stream leaves HBM bandwidth unused; reading the down weights meanwhile lets the
-// down launch find them in L2.
-__device__ __forceinline__ void prefetch_down_weights(const GemvArgs &a, const int32_t *tab, int n_list, int lane) {
-    for (int li = blockIdx.x; li < n_list; li += gridDim.x) {
-        const size_t e = (size_t)tab[li];
-        const uint8_t *c = a.pf_codes + e * a.pf_code_bytes;
-        for (uint32_t off = (uint32_t)lane * kPrefetchChunk; off < a.pf_code_bytes; off += 32u * kPrefetchChunk)
-            prefetch_l2(c + off, min(kPrefetchChunk, a.pf_code_bytes - off));
-        const uint8_t *sc = a.pf_scales + e * a.pf_scale_bytes;
-        for (uint32_t off = (uint32_t)lane * kPrefetchChunk; off < a.pf_scale_bytes; off += 32u * kPrefetchChunk)
-            prefetch_l2(sc + off, min(kPrefetchChunk, a.pf_scale_bytes - off));
-    }
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -484,7 +461,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
         if (first_pass(fc)) {
             issue_next(true);
             issue_next(false);
-            if (P == Proj::GateUp && a.pf_codes) prefetch_down_weights(a, tab, n_list, lane);
             int p = 0;
             for (Cursor c = fc; c.id < n_tasks; advance(c)) {
                 int r_begin;
@@ -765,8 +741,6 @@ static GemvArgs common_args(const Layer &L) {
     g.offsets = L.ws.offsets; g.perm = L.ws.perm; g.top_k = L.desc.top_k;
     g.I = L.desc.intermediate; g.err_word = L.ws.err_word;
     g.test_wait_ns = 0;
-    g.pf_codes = nullptr;
-    g.pf_scales = nullptr;
     return g;
 }
 
@@ -784,10 +758,6 @@ cudaError_t launch_gemv_gate_up(Layer &L, const uint16_t *x, int T, cudaStream_t
     g.src = L.ws.xq; g.src_inv = L.ws.xq_inv;
     g.act_out = L.ws.act; g.aq_out = L.ws.aq; g.aq_inv_out = L.ws.aq_inv;
     if (L.desc.flags & TFMOE_FLAG_TEST_TIMEOUT) g.test_wait_ns = kTestWaitNs;
-    g.pf_codes = L.w.d_codes;
-    g.pf_scales = L.w.d_scales;
-    g.pf_code_bytes = (uint32_t)((size_t)L.desc.hidden * L.desc.intermediate / 2);
-    g.pf_scale_bytes = (uint32_t)((size_t)L.desc.hidden * L.desc.intermediate / 16);
     gemv_kernel<Proj::GateUp><<<sh.grid, kThreads, sh.smem, s>>>(sh.map, g);
     *launches += 1;
     return cudaGetLastError();

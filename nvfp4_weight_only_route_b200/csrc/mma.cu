@@ -82,6 +82,7 @@ struct MmaSmem {
     uint8_t codes[C::kCStages][kTileCodeBytes];
     uint8_t scales[C::kCStages][kTileScaleBytes];
     uint16_t stage_out[4 * C::kEpiGroups][kEpiCols][16];   // per epilogue warp: 16 tokens x 16 outputs
+    float xi_s[4 * C::kEpiGroups][C::kMaxN];              // per epilogue warp: the tile's token scales
     uint64_t full[C::kStages], empty[C::kStages], aready[C::kStages];
     uint64_t cfull[C::kCStages], cempty[C::kCStages];
     uint64_t dfull[C::kDBufs], dempty[C::kDBufs];
@@ -143,6 +144,15 @@ __device__ __forceinline__ void mma_16bit_ts(uint32_t d_tmem, uint32_t a_tmem, u
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}"
         ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u));
+}
+
+// True in one lane of a converged warp (the lowest active lane, so the same lane at
+// every call while the warp stays converged).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile("{\n\t.reg .b32 rx;\n\t.reg .pred px;\n\telect.sync rx|px, %1;\n\t@px mov.s32 %0, 1;\n\t}"
+                 : "+r"(pred) : "r"(0xffffffffu));
+    return pred != 0;
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
@@ -282,40 +292,53 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            // one wait per stage (the decoders also wait for the token tile), descriptors
-            // advanced by adds, one commit per stage: the issuing thread does little else
-            const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sm.b[0]));
-            uint32_t g = 0, tile_i = 0;
-            for (int t = blockIdx.x; t < n_tiles && !sm.abort_flag; t += gridDim.x, ++tile_i) {
-                const int rows = __ldg(a.entries + 4 * (t / RT) + 2);
-                const uint32_t idesc = instr_desc_16bit(mma_n(rows), kType);
-                const int buf = (int)(tile_i % C::kDBufs);
-                const uint32_t use = tile_i / C::kDBufs;
-                if (!wait_or_abort(&sm.dempty[buf], (use & 1u) ^ 1u, &sm.abort_flag, a.err_word)) break;
+        // The MMA issue is the kernel's critical path (each tcgen05.mma keeps the issuing
+        // thread busy for tens of cycles). The whole warp runs the loop and waits, and one
+        // elected lane (the same one throughout: the warp is converged at every election)
+        // issues each stage's four MMAs and its commit, so a commit covers every MMA before
+        // it. Per stage: one wait (the decoders also wait for the token tile), four MMAs with
+        // descriptors advanced by adds, one commit; the stage slot and phase advance by
+        // increments.
+        const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sm.b[0]));
+        const uint32_t acol0 = tmem + kACol;
+        int s = 0;
+        uint32_t ph = 0, tile_i = 0;
+        for (int t = blockIdx.x; t < n_tiles && !sm.abort_flag; t += gridDim.x, ++tile_i) {
+            const int rows = __ldg(a.entries + 4 * (t / RT) + 2);
+            const uint32_t idesc = instr_desc_16bit(mma_n(rows), kType);
+            const int buf = (int)(tile_i % C::kDBufs);
+            const uint32_t use = tile_i / C::kDBufs;
+            if (!__all_sync(0xffffffffu, wait_or_abort(&sm.dempty[buf], (use & 1u) ^ 1u, &sm.abort_flag, a.err_word)))
+                break;
+            tc_fence_after();
+            const uint32_t dt = tmem + (uint32_t)buf * kMaxN;
+            bool ok = true;
+            for (int kt = 0; kt < KT; ++kt) {
+                if (!__all_sync(0xffffffffu, wait_or_abort(&sm.aready[s], ph, &sm.abort_flag, a.err_word))) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
-                const uint32_t dt = tmem + (uint32_t)buf * kMaxN;
-                bool ok = true;
-                for (int kt = 0; kt < KT; ++kt, ++g) {
-                    const int s = g % kStages;
-                    const uint32_t ph = (g / kStages) & 1u;
-                    if (!wait_or_abort(&sm.aready[s], ph, &sm.abort_flag, a.err_word)) { ok = false; break; }
-                    tc_fence_after();
+                if (elect_one()) {
                     const uint64_t bd = bdesc0 + (uint64_t)(s * (kBStageBytes >> 4));
-                    const uint32_t ad = tmem + kACol + (uint32_t)s * 32u;
+                    const uint32_t ad = acol0 + (uint32_t)s * 32u;
                     mma_16bit_ts(dt, ad, bd, idesc, kt != 0);
                     mma_16bit_ts(dt, ad + 8u, bd + 2u, idesc, 1u);
                     mma_16bit_ts(dt, ad + 16u, bd + 4u, idesc, 1u);
                     mma_16bit_ts(dt, ad + 24u, bd + 6u, idesc, 1u);
                     mma_commit(&sm.empty[s]);
                 }
-                if (!ok) break;
-                mma_commit(&sm.dfull[buf]);
+                __syncwarp();
+                if (++s == kStages) { s = 0; ph ^= 1u; }
             }
-            // on every path, including an abort: tensor memory and the operand stages stay
-            // in use until the MMAs already issued complete, which this commit reports
-            mma_commit(&sm.mma_done);
+            if (!ok) break;
+            if (elect_one()) mma_commit(&sm.dfull[buf]);
+            __syncwarp();
         }
+        // on every path, including an abort: tensor memory and the operand stages stay
+        // in use until the MMAs already issued complete, which this commit reports
+        if (elect_one()) mma_commit(&sm.mma_done);
+        __syncwarp();
     } else if (warp >= kDqWarp0 && warp < kEpiWarp0) {
         // decode: warpgroup gq takes the stages g with g % kDqGroups == gq (all 64 columns), so
         // stages are decoded concurrently; thread q owns weight row q = TMEM lane q
@@ -335,17 +358,16 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
                 const uint4 c1 = *reinterpret_cast<const uint4 *>(sm.codes[cs] + 2048 + q * 16);
                 const uint32_t sc4 = *reinterpret_cast<const uint32_t *>(sm.scales[cs] + q * 4);
                 mbar_arrive(&sm.cempty[cs]);                              // code stage consumed
-                ok = wait_or_abort(&sm.empty[s], ph ^ 1u, &sm.abort_flag, a.err_word);   // A stage free
-                if (ok) ok = wait_or_abort(&sm.full[s], ph, &sm.abort_flag, a.err_word);             // token tile landed
-                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                // decode the whole stage into registers first; then wait for the A stage to be
+                // free and for the token tile (so that the MMA issuer needs one wait per stage)
                 const uint32_t s01 = e4m3x2_to_f16x2(sc4 & 0xFFFFu), s23 = e4m3x2_to_f16x2(sc4 >> 16);
                 const __half2 h01 = *reinterpret_cast<const __half2 *>(&s01);
                 const __half2 h23 = *reinterpret_cast<const __half2 *>(&s23);
                 const __half2 sb[4] = {__low2half2(h01), __high2half2(h01), __low2half2(h23), __high2half2(h23)};
                 const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                uint32_t r[2][16];
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {      // columns 0..31, then 32..63
-                    uint32_t r[16];
 #pragma unroll
                     for (int w4 = 0; w4 < 4; ++w4) {  // word holds elements 8*w4 .. 8*w4 + 7 of the half
                         uint32_t h4[4];
@@ -353,17 +375,23 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
                         const __half2 sc = sb[2 * hh + (w4 >> 1)];
 #pragma unroll
                         for (int b = 0; b < 4; ++b)
-                            r[4 * w4 + b] = (kType == 0u) ? scale_pair_f16(h4[b], sc) : scale_pair_bf16(h4[b], sc);
+                            r[hh][4 * w4 + b] = (kType == 0u) ? scale_pair_f16(h4[b], sc) : scale_pair_bf16(h4[b], sc);
                     }
-                    tmem_st16(tmem + lane_base + kACol + (uint32_t)s * 32u + (uint32_t)hh * 16u, r);
                 }
+                ok = wait_or_abort(&sm.empty[s], ph ^ 1u, &sm.abort_flag, a.err_word);   // A stage free
+                if (ok) ok = wait_or_abort(&sm.full[s], ph, &sm.abort_flag, a.err_word); // token tile landed
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tmem_st16(tmem + lane_base + kACol + (uint32_t)s * 32u, r[0]);
+                tmem_st16(tmem + lane_base + kACol + (uint32_t)s * 32u + 16u, r[1]);
                 tc_wait_st();
                 tc_fence_before();
                 mbar_arrive(&sm.aready[s]);
             }
         }
     } else if (warp >= kEpiWarp0) {
-        // two warpgroups split the accumulator columns in steps of 16; one buffer behind the MMAs
+        // epilogue warpgroups take alternate 16-column steps of the accumulator. Each warp
+        // has the next step's tensor-memory load in flight while it processes the current
+        // one, and stages the tile's per-token activation scales in shared memory once.
         const int eg = (warp - kEpiWarp0) >> 2;
         const int ew = warp - kEpiWarp0;                           // staging slot
         const int q = (warp & 3) * 32 + lane;                      // weight row = TMEM lane
@@ -375,24 +403,22 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
             const int rt = t % RT;
             const int n = mma_n(rows);
             const int buf = (int)(tile_i % C::kDBufs);
+            const float gs = __ldg(a.glob0 + e);                               // gate (or down) scale
+            const float gs_up = (P == Proj::GateUp) ? __ldg(a.glob1 + e) : 0.f;
+            if (P == Proj::GateUp) {
+                __syncwarp();
+                for (int c = lane; c < n; c += 32)
+                    sm.xi_s[ew][c] = (c < rows) ? __ldg(a.row_inv_scale + row0 + c) : 0.f;
+                __syncwarp();
+            }
             if (!wait_or_abort(&sm.dfull[buf], (tile_i / C::kDBufs) & 1u, &sm.abort_flag, a.err_word)) break;
             tc_fence_after();
             const int grow = rt * kM + q;
-            const float gs = __ldg(a.glob0 + e);                               // gate (or down) scale
-            const float gs_up = (P == Proj::GateUp) ? __ldg(a.glob1 + e) : 0.f;
-            // this group's steps: group eg takes steps eg, eg + kEpiGroups, ...
+            const uint32_t dcol = tmem + lane_base + (uint32_t)buf * kMaxN;
+            // this group's steps: eg, eg + kEpiGroups, ...
             const int steps = n / kEpiCols;
-            bool handed_back = false;
-            for (int st = eg; st < steps; st += C::kEpiGroups) {
+            auto process = [&](const uint32_t (&d)[16], int st) {
                 const int c = st * kEpiCols;
-                uint32_t d[16];
-                tmem_ld16(tmem + lane_base + (uint32_t)buf * kMaxN + (uint32_t)c, d);
-                tc_wait_ld();
-                if (st + C::kEpiGroups >= steps) {   // last read of this group: hand the buffer back
-                    tc_fence_before();
-                    mbar_arrive(&sm.dempty[buf]);
-                    handed_back = true;
-                }
                 if (P == Proj::GateUp) {
                     // even lane 2i holds gate row j of the step's 16 tokens, lane 2i+1 the up row of
                     // the same j. The pair splits the work: the even lane takes tokens 0..7 of the
@@ -400,7 +426,6 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
                     // tokens (one shuffle per token), so no lane idles through the SwiGLU. The a
                     // values [16 tokens][16 j] are staged in shared memory, then written as 16-byte
                     // row pieces.
-                    const float xi_src = (lane < kEpiCols && c + lane < rows) ? __ldg(a.row_inv_scale + row0 + c + lane) : 0.f;
                     const bool odd = (lane & 1) != 0;
                     const int half = odd ? 8 : 0;
 #pragma unroll
@@ -408,8 +433,8 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
                         const float keep = __uint_as_float(odd ? d[i + 8] : d[i]);
                         const float give = __uint_as_float(odd ? d[i] : d[i + 8]);
                         const float got = __shfl_xor_sync(0xffffffffu, give, 1);
-                        const float xi = __shfl_sync(0xffffffffu, xi_src, i + half);
-                        const float gv = (odd ? got : keep) * (gs * xi);       // xi: an exact power of two
+                        const float xi = sm.xi_s[ew][c + half + i];            // an exact power of two
+                        const float gv = (odd ? got : keep) * (gs * xi);
                         const float uv = (odd ? keep : got) * (gs_up * xi);
                         sm.stage_out[ew][half + i][lane >> 1] = float_to_bf16_bits_rn(silu_f32(gv) * uv);
                     }
@@ -429,8 +454,28 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
                         if (tok < rows) a.y_out[(size_t)(row0 + tok) * a.R + grow] = __uint_as_float(d[i]) * gs;
                     }
                 }
+            };
+            uint32_t d0[16], d1[16];
+            int st = eg;
+            if (st < steps) tmem_ld16(dcol + (uint32_t)(st * kEpiCols), d0);
+            // two steps per iteration, alternating the register buffers: load step st+G while
+            // processing step st. After the last load lands the accumulator is handed back.
+            while (st < steps) {
+                tc_wait_ld();
+                int nst = st + C::kEpiGroups;
+                if (nst < steps) tmem_ld16(dcol + (uint32_t)(nst * kEpiCols), d1);
+                else { tc_fence_before(); mbar_arrive(&sm.dempty[buf]); }
+                process(d0, st);
+                st = nst;
+                if (st >= steps) break;
+                tc_wait_ld();
+                nst = st + C::kEpiGroups;
+                if (nst < steps) tmem_ld16(dcol + (uint32_t)(nst * kEpiCols), d0);
+                else { tc_fence_before(); mbar_arrive(&sm.dempty[buf]); }
+                process(d1, st);
+                st = nst;
             }
-            if (!handed_back) {                  // no step for this group in this tile
+            if (eg >= steps) {                   // no step for this group in this tile
                 tc_fence_before();
                 mbar_arrive(&sm.dempty[buf]);
             }
