@@ -228,15 +228,15 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
-            mbar_init(&sm.aready[s], 128);
+            mbar_init(&sm.aready[s], 4);               // one arrival per decoder warp
         }
         for (int c = 0; c < kCStages; ++c) {
             mbar_init(&sm.cfull[c], 1);
-            mbar_init(&sm.cempty[c], 128);
+            mbar_init(&sm.cempty[c], 4);
         }
         for (int b = 0; b < C::kDBufs; ++b) {
             mbar_init(&sm.dfull[b], 1);
-            mbar_init(&sm.dempty[b], 128 * C::kEpiGroups);
+            mbar_init(&sm.dempty[b], 4 * C::kEpiGroups);   // one arrival per epilogue warp
         }
         mbar_init(&sm.mma_done, 1);
         sm.abort_flag = 0;
@@ -357,7 +357,8 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
                 const uint4 c0 = *reinterpret_cast<const uint4 *>(sm.codes[cs] + q * 16);
                 const uint4 c1 = *reinterpret_cast<const uint4 *>(sm.codes[cs] + 2048 + q * 16);
                 const uint32_t sc4 = *reinterpret_cast<const uint32_t *>(sm.scales[cs] + q * 4);
-                mbar_arrive(&sm.cempty[cs]);                              // code stage consumed
+                __syncwarp();                                              // every lane has read its codes
+                if (lane == 0) mbar_arrive(&sm.cempty[cs]);                // code stage consumed
                 // decode the whole stage into registers first; then wait for the A stage to be
                 // free and for the token tile (so that the MMA issuer needs one wait per stage)
                 const uint32_t s01 = e4m3x2_to_f16x2(sc4 & 0xFFFFu), s23 = e4m3x2_to_f16x2(sc4 >> 16);
@@ -385,7 +386,8 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
                 tmem_st16(tmem + lane_base + kACol + (uint32_t)s * 32u + 16u, r[1]);
                 tc_wait_st();
                 tc_fence_before();
-                mbar_arrive(&sm.aready[s]);
+                __syncwarp();                        // the warp's stores precede its one arrival
+                if (lane == 0) mbar_arrive(&sm.aready[s]);
             }
         }
     } else if (warp >= kEpiWarp0) {
@@ -417,6 +419,11 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
             const uint32_t dcol = tmem + lane_base + (uint32_t)buf * kMaxN;
             // this group's steps: eg, eg + kEpiGroups, ...
             const int steps = n / kEpiCols;
+            auto hand_back = [&]() {             // the warp's reads precede its one arrival
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.dempty[buf]);
+            };
             auto process = [&](const uint32_t (&d)[16], int st) {
                 const int c = st * kEpiCols;
                 if (P == Proj::GateUp) {
@@ -464,21 +471,18 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
                 tc_wait_ld();
                 int nst = st + C::kEpiGroups;
                 if (nst < steps) tmem_ld16(dcol + (uint32_t)(nst * kEpiCols), d1);
-                else { tc_fence_before(); mbar_arrive(&sm.dempty[buf]); }
+                else hand_back();
                 process(d0, st);
                 st = nst;
                 if (st >= steps) break;
                 tc_wait_ld();
                 nst = st + C::kEpiGroups;
                 if (nst < steps) tmem_ld16(dcol + (uint32_t)(nst * kEpiCols), d0);
-                else { tc_fence_before(); mbar_arrive(&sm.dempty[buf]); }
+                else hand_back();
                 process(d1, st);
                 st = nst;
             }
-            if (eg >= steps) {                   // no step for this group in this tile
-                tc_fence_before();
-                mbar_arrive(&sm.dempty[buf]);
-            }
+            if (eg >= steps) hand_back();        // no step for this group in this tile
         }
     }
     __syncthreads();
