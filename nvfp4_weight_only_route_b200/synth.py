@@ -36,6 +36,15 @@ Workload recipe (sizes and distributions of the five layer shapes):
     beta = sigma_l * sqrt(6) / pi, sigma_l = router_std * x_std * sqrt(H) the
     analytic std of the unbiased logits (the Gumbel scale that turns the
     bias into top-1 Zipf load).
+  * Shared expert (optional): one SwiGLU FFN of width Is = m * I in the same
+    formats and distributions as a routed expert (codes uniform, scales
+    2**U[-4, 2], per-tensor scale as the routed experts').
+  * Residual: N(0, 1) bf16 [T][H]. RMS-norm weight gamma: U[0.5, 1.5] bf16 [H].
+
+Shared-expert layout (canonical, row-major): shared_gate_codes / shared_up_codes
+uint8 [Is][H/2], shared_gate_scales / shared_up_scales [Is][H/16],
+shared_down_codes [H][Is/2], shared_down_scales [H][Is/16], and the three
+per-tensor multipliers as fp32 arrays of one element.
 """
 from __future__ import annotations
 
@@ -135,6 +144,30 @@ def make_layer(shape: LayerShape, seed: int) -> Dict[str, Optional[np.ndarray]]:
     else:
         layer["router_bias"] = None
     return layer
+
+
+def make_shared(shape: LayerShape, seed: int, Is: int) -> Dict[str, np.ndarray]:
+    """Seeded shared expert of width Is (canonical layout, host numpy arrays)."""
+    H = shape.H
+    assert Is % 16 == 0 and Is > 0
+    r = _rng(seed, 0x5EED, Is)
+    out: Dict[str, np.ndarray] = {}
+    for name, rows, K in (("gate", Is, H), ("up", Is, H), ("down", H, Is)):
+        out[f"shared_{name}_codes"] = _random_bytes(r, rows * (K // 2)).reshape(rows, K // 2)
+        out[f"shared_{name}_scales"] = _e4m3_bits_loguniform(r, rows * (K // 16)).reshape(rows, K // 16)
+        out[f"shared_{name}_global"] = np.full(1, shape.global_scale, dtype=np.float32)
+    return out
+
+
+def make_residual(shape: LayerShape, seed: int, T: int) -> np.ndarray:
+    """Seeded residual stream, bf16 bits [T][H]."""
+    return _bf16_bits_normal(_rng(seed, 0x2E5, T), (T, shape.H), 1.0)
+
+
+def make_norm_weight(shape: LayerShape, seed: int) -> np.ndarray:
+    """Seeded RMS-norm gamma, bf16 bits [H], uniform on [0.5, 1.5]."""
+    f = _rng(seed, 0x4042).random(shape.H, dtype=np.float32) + np.float32(0.5)
+    return torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
 
 
 def make_x(shape: LayerShape, seed: int, T: int, stream: int = 0) -> np.ndarray:

@@ -32,13 +32,28 @@ class _Layer(ctypes.Structure):
                 ("gate_codes", _u8p), ("up_codes", _u8p),
                 ("gate_scales", _u8p), ("up_scales", _u8p),
                 ("gate_global", _f32p), ("up_global", _f32p),
-                ("down_codes", _u8p), ("down_scales", _u8p), ("down_global", _f32p)]
+                ("down_codes", _u8p), ("down_scales", _u8p), ("down_global", _f32p),
+                ("shared_intermediate", ctypes.c_int32),
+                ("sh_gate_codes", _u8p), ("sh_up_codes", _u8p),
+                ("sh_gate_scales", _u8p), ("sh_up_scales", _u8p),
+                ("sh_gate_global", ctypes.c_float), ("sh_up_global", ctypes.c_float),
+                ("sh_down_codes", _u8p), ("sh_down_scales", _u8p), ("sh_down_global", ctypes.c_float)]
+
+
+class _Epilogue(ctypes.Structure):
+    _fields_ = [("residual", _u16p), ("norm_w", _u16p), ("eps", ctypes.c_double)]
 
 
 class _Outputs(ctypes.Structure):
     _fields_ = [("out", _u16p), ("out64", _f64p), ("S", _f64p), ("logits", _f32p),
                 ("ids", _i32p), ("g", _f64p), ("G", _f32p), ("U", _f32p),
-                ("a", _u16p), ("y", _f64p), ("yabs", _f64p)]
+                ("a", _u16p), ("y", _f64p), ("yabs", _f64p),
+                ("out_norm", _u16p), ("a_sh", _u16p), ("y_sh", _f64p)]
+
+# Keys of the optional shared expert in a layer dict (canonical layout, see forward()).
+SHARED_KEYS = ("shared_gate_codes", "shared_up_codes", "shared_gate_scales", "shared_up_scales",
+               "shared_gate_global", "shared_up_global", "shared_down_codes", "shared_down_scales",
+               "shared_down_global")
 
 
 def build(force: bool = False) -> str:
@@ -68,7 +83,9 @@ def lib():
         _lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
         _lib.oracle_forward.restype = ctypes.c_int
         _lib.oracle_forward.argtypes = [ctypes.POINTER(_Layer), _u16p, ctypes.c_int32,
-                                        ctypes.c_int32, ctypes.POINTER(_Outputs)]
+                                        ctypes.c_int32, ctypes.POINTER(_Epilogue), ctypes.POINTER(_Outputs)]
+        _lib.oracle_rms_norm.restype = ctypes.c_int
+        _lib.oracle_rms_norm.argtypes = [_u16p, _u16p, ctypes.c_int32, ctypes.c_int32, ctypes.c_double, _u16p]
         _lib.oracle_route.restype = ctypes.c_int
         _lib.oracle_route.argtypes = [ctypes.POINTER(_Layer), _u16p, ctypes.c_int32, ctypes.c_int32,
                                       _f32p, _i32p, _f64p]
@@ -103,12 +120,29 @@ def _ptr(a: Optional[np.ndarray], t):
     return a.ctypes.data_as(t)
 
 
+def rms_norm(v: np.ndarray, gamma: np.ndarray, eps: float) -> np.ndarray:
+    """The oracle's RMS norm of bf16 rows v [T][H] with bf16 gamma [H] (bf16 bits out)."""
+    v = np.ascontiguousarray(v, dtype=np.uint16)
+    gamma = np.ascontiguousarray(gamma, dtype=np.uint16)
+    T, H = v.shape
+    out = np.zeros((T, H), np.uint16)
+    rc = lib().oracle_rms_norm(_ptr(v, _u16p), _ptr(gamma, _u16p), T, H, eps, _ptr(out, _u16p))
+    if rc != 0:
+        raise RuntimeError(f"oracle_rms_norm failed with code {rc}")
+    return out
+
+
 def forward(layer: Dict[str, Optional[np.ndarray]], x: np.ndarray, *, top_k: int,
-            nthreads: int = 0, intermediates: bool = False) -> Dict[str, np.ndarray]:
+            nthreads: int = 0, intermediates: bool = False, residual: Optional[np.ndarray] = None,
+            norm_w: Optional[np.ndarray] = None, eps: float = 1e-6) -> Dict[str, np.ndarray]:
     """Run the oracle on host arrays in the canonical layout.
 
     ``x`` is bf16 bits [T][H]. Returns out (bf16 bits), out64, S, and with
     ``intermediates`` also logits, ids, g, G, U, a and y.
+    A layer dict holding the SHARED_KEYS (codes/scales [Is][H/2], [Is][H/16], down
+    [H][Is/2], [H][Is/16], globals as one-element fp32 arrays) adds the shared expert
+    (``a_sh``, ``y_sh`` with ``intermediates``). ``residual`` (bf16 bits [T][H]) is added
+    to the output; ``norm_w`` (bf16 bits [H]) adds ``out_norm``, the RMS norm of ``out``.
     """
     E, H = layer["router_w"].shape
     I = layer["gate_codes"].shape[1]
@@ -130,9 +164,36 @@ def forward(layer: Dict[str, Optional[np.ndarray]], x: np.ndarray, *, top_k: int
                _ptr(arr("gate_global", np.float32), _f32p), _ptr(arr("up_global", np.float32), _f32p),
                _ptr(arr("down_codes", np.uint8), _u8p), _ptr(arr("down_scales", np.uint8), _u8p),
                _ptr(arr("down_global", np.float32), _f32p))
+    Is = 0
+    if layer.get("shared_gate_codes") is not None:
+        Is = layer["shared_gate_codes"].shape[0]
+        assert layer["shared_down_codes"].shape == (H, Is // 2)
+        L.shared_intermediate = Is
+        L.sh_gate_codes = _ptr(arr("shared_gate_codes", np.uint8), _u8p)
+        L.sh_up_codes = _ptr(arr("shared_up_codes", np.uint8), _u8p)
+        L.sh_gate_scales = _ptr(arr("shared_gate_scales", np.uint8), _u8p)
+        L.sh_up_scales = _ptr(arr("shared_up_scales", np.uint8), _u8p)
+        L.sh_gate_global = float(np.float32(layer["shared_gate_global"].reshape(-1)[0]))
+        L.sh_up_global = float(np.float32(layer["shared_up_global"].reshape(-1)[0]))
+        L.sh_down_codes = _ptr(arr("shared_down_codes", np.uint8), _u8p)
+        L.sh_down_scales = _ptr(arr("shared_down_scales", np.uint8), _u8p)
+        L.sh_down_global = float(np.float32(layer["shared_down_global"].reshape(-1)[0]))
+    epi = _Epilogue(_ptr(None, _u16p), _ptr(None, _u16p), float(eps))
+    if residual is not None:
+        residual = np.ascontiguousarray(residual, dtype=np.uint16)
+        assert residual.shape == (T, H)
+        epi.residual = _ptr(residual, _u16p)
+    if norm_w is not None:
+        norm_w = np.ascontiguousarray(norm_w, dtype=np.uint16)
+        assert norm_w.shape == (H,)
+        epi.norm_w = _ptr(norm_w, _u16p)
     P = T * top_k
     res = {"out": np.zeros((T, H), np.uint16), "out64": np.zeros((T, H), np.float64),
            "S": np.zeros((T, H), np.float64)}
+    if norm_w is not None:
+        res["out_norm"] = np.zeros((T, H), np.uint16)
+    if intermediates and Is:
+        res.update(a_sh=np.zeros((T, Is), np.uint16), y_sh=np.zeros((T, H), np.float64))
     if intermediates:
         res.update(logits=np.zeros((T, E), np.float32), ids=np.zeros((T, top_k), np.int32),
                    g=np.zeros((T, top_k), np.float64), G=np.zeros((T, top_k, I), np.float32),
@@ -141,11 +202,12 @@ def forward(layer: Dict[str, Optional[np.ndarray]], x: np.ndarray, *, top_k: int
     O = _Outputs(_ptr(res["out"], _u16p), _ptr(res["out64"], _f64p), _ptr(res["S"], _f64p),
                  _ptr(res.get("logits"), _f32p), _ptr(res.get("ids"), _i32p),
                  _ptr(res.get("g"), _f64p), _ptr(res.get("G"), _f32p), _ptr(res.get("U"), _f32p),
-                 _ptr(res.get("a"), _u16p), _ptr(res.get("y"), _f64p), _ptr(res.get("yabs"), _f64p))
-    rc = lib().oracle_forward(ctypes.byref(L), _ptr(x, _u16p), T, nthreads, ctypes.byref(O))
+                 _ptr(res.get("a"), _u16p), _ptr(res.get("y"), _f64p), _ptr(res.get("yabs"), _f64p),
+                 _ptr(res.get("out_norm"), _u16p), _ptr(res.get("a_sh"), _u16p), _ptr(res.get("y_sh"), _f64p))
+    rc = lib().oracle_forward(ctypes.byref(L), _ptr(x, _u16p), T, nthreads, ctypes.byref(epi), ctypes.byref(O))
     if rc != 0:
         raise RuntimeError(f"oracle_forward failed with code {rc}")
-    del keep, P
+    del keep, P, residual, norm_w
     return res
 
 

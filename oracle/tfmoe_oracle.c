@@ -24,13 +24,26 @@
  *    fp32 per-tensor multiplier per (expert, projection).
  *  - The reference is 64-bit, as the error budget of [TensorFold issue #627,
  *    "Description"] is stated against a float64 reference.
+ *  - Optional steps on either side of the routed path, from the same MoE
+ *    chain [TensorFold issue #627, the per-launch kernel table (add_moe_norm)
+ *    and "Where the 0.35 ms per step goes" (the shared expert, run beside the
+ *    routed experts)]: a shared expert -- one SwiGLU FFN of width Is in the
+ *    same NVFP4 formats that every token passes through with weight 1 -- the
+ *    residual add, and an RMS norm of the sum. The pages name these steps but
+ *    not their arithmetic; the readings taken here are: the shared expert's a
+ *    is rounded to bf16 like a routed expert's; the residual (bf16) is added
+ *    in the same fp64 sum as the expert outputs; the layer output (the new
+ *    residual stream) is that sum rounded once to bf16; the norm reads that
+ *    rounded output: out_norm = bf16_RNE( h * gamma / sqrt(mean(h^2) + eps) ).
  *
  * Rounding points (the only places precision is lost on purpose):
  *   router logit      = fp32( fp64 sum of bf16*bf16 products ) (+ fp32 bias)
  *   gate G, up U      = fp32( fp64 sum over K of x * deq(w) )
  *   a = bf16_RNE( silu(G) * U )   evaluated in fp64 from the fp32 G, U
  *   y = fp64 sum over K of a * deq(w)      (not rounded)
- *   out = bf16_RNE( sum over slots s=0..k-1 of g_s * y_s )   in fp64
+ *   out = bf16_RNE( sum over slots s=0..k-1 of g_s * y_s
+ *                   (+ y_shared) (+ residual) )                   in fp64
+ *   out_norm = bf16_RNE( out * gamma / sqrt(mean over h of out^2 + eps) )
  *
  * Parity pins live in the repository's CPU test-suite; every function below
  * is pinned there (format tables, a hand-worked block, closed-form chains,
@@ -125,7 +138,22 @@ typedef struct {
     const uint8_t *down_codes;                /* [E][H][I/2] */
     const uint8_t *down_scales;               /* [E][H][I/16] */
     const float *down_global;                 /* [E] */
+    /* Shared expert: shared_intermediate = Is (0: none). */
+    int32_t shared_intermediate;
+    const uint8_t *sh_gate_codes, *sh_up_codes;     /* [Is][H/2] */
+    const uint8_t *sh_gate_scales, *sh_up_scales;   /* [Is][H/16] */
+    float sh_gate_global, sh_up_global;
+    const uint8_t *sh_down_codes;                   /* [H][Is/2] */
+    const uint8_t *sh_down_scales;                  /* [H][Is/16] */
+    float sh_down_global;
 } oracle_layer;
+
+/* Inputs of the steps after the combine; any pointer may be NULL (step skipped). */
+typedef struct {
+    const uint16_t *residual;   /* bf16 [T][H], added to the layer output */
+    const uint16_t *norm_w;     /* bf16 [H], gamma of the RMS norm of the layer output */
+    double eps;                 /* the norm's epsilon */
+} oracle_epilogue;
 
 /* Outputs. Every pointer except out may be NULL. Per-pair arrays are indexed
  * by pair = t*k + s, s the slot (0 = highest logit). */
@@ -140,6 +168,9 @@ typedef struct {
     uint16_t *a;        /* bf16 [T][k][I] */
     double *y;          /* [T][k][H] */
     double *yabs;       /* [T][k][H] sum_j |a[j] * deq(Wd)[h][j]| */
+    uint16_t *out_norm; /* bf16 [T][H] RMS norm of out (needs epilogue norm_w) */
+    uint16_t *a_sh;     /* bf16 [T][Is] shared expert's SwiGLU output */
+    double *y_sh;       /* [T][H] shared expert's down projection */
 } oracle_outputs;
 
 /* Router logits, top-k (ties to the lower expert index) and the softmax
@@ -169,12 +200,86 @@ static void route_token(const oracle_layer *L, const uint16_t *x, float *logits,
     for (int s = 0; s < k; ++s) g[s] = exp((double)logits[ids[s]] - lmax) / den;
 }
 
+/* The shared expert for every token: a_sh = bf16(silu(G) * U) with G, U the fp32-rounded
+ * fp64 sums over H, then y_sh = the fp64 sum over Is of a_sh * deq(Wd_sh) and its absolute
+ * counterpart. The same arithmetic as a routed expert, without routing. */
+static void shared_expert(const oracle_layer *L, const double *xd, int32_t T, int nthreads, uint16_t *a_sh,
+                          double *y_sh, double *yabs_sh)
+{
+    const int H = L->hidden, Is = L->shared_intermediate;
+#pragma omp parallel num_threads(nthreads)
+    {
+        double *dg = (double *)malloc(sizeof(double) * H);
+        double *du = (double *)malloc(sizeof(double) * H);
+#pragma omp for schedule(static)
+        for (int j = 0; j < Is; ++j) {
+            dequant_row(L->sh_gate_codes + (size_t)j * (H / 2), L->sh_gate_scales + (size_t)j * (H / 16),
+                        L->sh_gate_global, H, dg);
+            dequant_row(L->sh_up_codes + (size_t)j * (H / 2), L->sh_up_scales + (size_t)j * (H / 16),
+                        L->sh_up_global, H, du);
+            for (int t = 0; t < T; ++t) {
+                const double *xr = xd + (size_t)t * H;
+                double sg = 0.0, su = 0.0;
+                for (int h = 0; h < H; ++h) { sg += xr[h] * dg[h]; su += xr[h] * du[h]; }
+                float G = (float)sg, U = (float)su;
+                a_sh[(size_t)t * Is + j] = oracle_round_bf16(silu((double)G) * (double)U);
+            }
+        }
+        free(dg);
+        free(du);
+    }
+#pragma omp parallel num_threads(nthreads)
+    {
+        double *dd = (double *)malloc(sizeof(double) * Is);
+#pragma omp for schedule(static)
+        for (int h = 0; h < H; ++h) {
+            dequant_row(L->sh_down_codes + (size_t)h * (Is / 2), L->sh_down_scales + (size_t)h * (Is / 16),
+                        L->sh_down_global, Is, dd);
+            for (int t = 0; t < T; ++t) {
+                const uint16_t *ar = a_sh + (size_t)t * Is;
+                double s = 0.0, sa = 0.0;
+                for (int j = 0; j < Is; ++j) {
+                    double term = oracle_bf16_to_double(ar[j]) * dd[j];
+                    s += term;
+                    sa += fabs(term);
+                }
+                y_sh[(size_t)t * H + h] = s;
+                yabs_sh[(size_t)t * H + h] = sa;
+            }
+        }
+        free(dd);
+    }
+}
+
+/* RMS norm of one bf16 row: bf16_RNE( v[h] * gamma[h] / sqrt(mean(v^2) + eps) ), in fp64. */
+static void rms_norm_row(const uint16_t *v, const uint16_t *gamma, int H, double eps, uint16_t *out)
+{
+    double ss = 0.0;
+    for (int h = 0; h < H; ++h) {
+        double f = oracle_bf16_to_double(v[h]);
+        ss += f * f;
+    }
+    double r = 1.0 / sqrt(ss / (double)H + eps);
+    for (int h = 0; h < H; ++h)
+        out[h] = oracle_round_bf16(oracle_bf16_to_double(v[h]) * r * oracle_bf16_to_double(gamma[h]));
+}
+
+int oracle_rms_norm(const uint16_t *v, const uint16_t *gamma, int32_t T, int32_t H, double eps, uint16_t *out)
+{
+    if (!v || !gamma || !out || T < 0 || H <= 0) return 1;
+    for (int t = 0; t < T; ++t) rms_norm_row(v + (size_t)t * H, gamma, H, eps, out + (size_t)t * H);
+    return 0;
+}
+
 int oracle_forward(const oracle_layer *L, const uint16_t *x, int32_t T, int32_t nthreads,
-                   const oracle_outputs *O)
+                   const oracle_epilogue *epi, const oracle_outputs *O)
 {
     if (!L || !O || T < 0) return 1;
     const int H = L->hidden, I = L->intermediate, E = L->num_experts, k = L->top_k;
     if (H <= 0 || I <= 0 || E <= 0 || k <= 0 || k > E || H % 16 || I % 16) return 1;
+    const int Is = L->shared_intermediate;
+    if (Is < 0 || Is % 16) return 1;
+    if (O->out_norm && !(epi && epi->norm_w && O->out)) return 1;
     if (T == 0) return 0;
     if (nthreads <= 0) nthreads = omp_get_max_threads();
     const size_t P = (size_t)T * k;
@@ -190,6 +295,14 @@ int oracle_forward(const oracle_layer *L, const uint16_t *x, int32_t T, int32_t 
     int32_t *start = (int32_t *)malloc(sizeof(int32_t) * ((size_t)E + 1));
     int32_t *pairs = (int32_t *)malloc(sizeof(int32_t) * P);
     if (!logits || !ids || !g || !a || !y || !yabs || !xd || !count || !start || !pairs) return 2;
+    uint16_t *a_sh = NULL;
+    double *y_sh = NULL, *yabs_sh = NULL;
+    if (Is > 0) {
+        a_sh = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)T * Is);
+        y_sh = (double *)malloc(sizeof(double) * (size_t)T * H);
+        yabs_sh = (double *)malloc(sizeof(double) * (size_t)T * H);
+        if (!a_sh || !y_sh || !yabs_sh) return 2;
+    }
 
     /* Step 1: routing, token by token. */
 #pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1)
@@ -264,7 +377,12 @@ int oracle_forward(const oracle_layer *L, const uint16_t *x, int32_t T, int32_t 
         }
     }
 
-    /* Step 5: weighted combine in slot order, rounded once to bf16. */
+    /* Step 4b: the shared expert, every token with weight 1. */
+    if (Is > 0) shared_expert(L, xd, T, nthreads, a_sh, y_sh, yabs_sh);
+
+    /* Step 5: weighted combine in slot order, then the shared expert's output and the
+     * residual, in one fp64 sum rounded once to bf16. */
+    const uint16_t *res = epi ? epi->residual : NULL;
 #pragma omp parallel for num_threads(nthreads) schedule(static)
     for (int t = 0; t < T; ++t) {
         for (int h = 0; h < H; ++h) {
@@ -275,10 +393,23 @@ int oracle_forward(const oracle_layer *L, const uint16_t *x, int32_t T, int32_t 
                 bound += g[p] * yabs[p * H + h];
             }
             size_t o = (size_t)t * H + h;
+            if (Is > 0) {
+                acc += y_sh[o];
+                bound += yabs_sh[o];
+            }
+            if (res) acc += oracle_bf16_to_double(res[o]);
             if (O->out) O->out[o] = oracle_round_bf16(acc);
             if (O->out64) O->out64[o] = acc;
             if (O->S) O->S[o] = bound;
         }
+    }
+
+    /* Step 6: RMS norm of the rounded layer output. */
+    if (O->out_norm) oracle_rms_norm(O->out, epi->norm_w, T, H, epi->eps, O->out_norm);
+    if (Is > 0) {
+        if (O->a_sh) memcpy(O->a_sh, a_sh, sizeof(uint16_t) * (size_t)T * Is);
+        if (O->y_sh) memcpy(O->y_sh, y_sh, sizeof(double) * (size_t)T * H);
+        free(a_sh); free(y_sh); free(yabs_sh);
     }
 
     if (O->logits) memcpy(O->logits, logits, sizeof(float) * (size_t)T * E);

@@ -15,6 +15,7 @@ from oracle import oracle as oracle_module
 
 import test_oracle_bruteforce as bf
 import test_oracle_closed_form as cf
+import test_oracle_epilogue as ep
 import test_oracle_formats as ff
 
 MUTATIONS = {
@@ -35,6 +36,16 @@ MUTATIONS = {
     "bf16_truncate": ("rint(ldexp(a, -q_exp))", "floor(ldexp(a, -q_exp))"),
     "gate_not_rounded_fp32": ("a[(size_t)p * I + j] = oracle_round_bf16(silu((double)G) * (double)U);",
                               "a[(size_t)p * I + j] = oracle_round_bf16(silu(sg) * su);"),
+    "shared_down_uses_up_global": ("L->sh_down_global, Is, dd", "L->sh_up_global, Is, dd"),
+    "shared_output_dropped": ("acc += y_sh[o];", ";"),
+    "shared_gate_up_swapped": ("oracle_round_bf16(silu((double)G) * (double)U);\n            }\n        }\n        free(dg);\n        free(du);\n    }\n#pragma omp parallel num_threads(nthreads)\n    {\n        double *dd = (double *)malloc(sizeof(double) * Is);",
+                               "oracle_round_bf16(silu((double)U) * (double)G);\n            }\n        }\n        free(dg);\n        free(du);\n    }\n#pragma omp parallel num_threads(nthreads)\n    {\n        double *dd = (double *)malloc(sizeof(double) * Is);"),
+    "shared_down_row_stride": ("L->sh_down_codes + (size_t)h * (Is / 2)", "L->sh_down_codes + (size_t)h * (H / 2)"),
+    "residual_dropped": ("if (res) acc += oracle_bf16_to_double(res[o]);", ""),
+    "norm_sum_not_mean": ("sqrt(ss / (double)H + eps)", "sqrt(ss + eps)"),
+    "norm_eps_outside_root": ("1.0 / sqrt(ss / (double)H + eps)", "1.0 / (sqrt(ss / (double)H) + eps)"),
+    "norm_gamma_column_0": ("oracle_bf16_to_double(gamma[h])", "oracle_bf16_to_double(gamma[0])"),
+    "norm_mean_off_by_one": ("sqrt(ss / (double)H + eps)", "sqrt(ss / (double)(H - 1) + eps)"),
 }
 
 
@@ -54,6 +65,12 @@ def _all_pins(mod):
     cases.append(lambda: bf.test_oracle_matches_brute_force_tiny(mod, 64, 32, 4, 2, 4, 12))
     cases.append(lambda: bf.test_oracle_matches_brute_force_with_bias(mod))
     cases.append(lambda: bf.test_oracle_matches_brute_force_tiny_layer_shape(mod))
+    for name in dir(ep):
+        if name.startswith("test_") and name not in ("test_shared_expert_residual_and_norm_match_dense",
+                                                     "test_norm_of_constant_row_is_sign_when_eps_is_zero"):
+            cases.append(lambda n=name: getattr(ep, n)(mod))
+    cases.append(lambda: ep.test_shared_expert_residual_and_norm_match_dense(mod, 64, 32, 4, 2, 32, 3, 21))
+    cases.append(lambda: ep.test_norm_of_constant_row_is_sign_when_eps_is_zero(mod, 0.75))
     for c in cases:
         try:
             c()
