@@ -406,7 +406,8 @@ class Bench:
 
     def parity(self, name, Ls, lnps, xs, n_sample, sample_layers):
         """Routing of every token against the oracle's routing step (bit-exact ids and
-        logits), the output on sampled tokens within the tolerance."""
+        selected logits; every other logit exact or within the library's stated bound of the
+        tensor-core approximation), the output on sampled tokens within the tolerance."""
         from oracle import oracle
         torch, tfmoe = self.torch, self.tfmoe
         si, T, _ = WORKLOADS[name]
@@ -422,8 +423,16 @@ class Bench:
             ids_g = L.buffer_tensor(tfmoe.BUF_TOPK_IDS, torch.int32, (T, k)).cpu().numpy()
             log_g = L.buffer_tensor(tfmoe.BUF_LOGITS, torch.float32, (T, E)).cpu().numpy()
             r = oracle.route(lnps[li], x_np, top_k=k)
-            if not (np.array_equal(ids_g, r["ids"]) and np.array_equal(log_g, r["logits"])):
+            if not (np.array_equal(ids_g, r["ids"]) and
+                    np.array_equal(np.take_along_axis(log_g, r["ids"], 1), np.take_along_axis(r["logits"], r["ids"], 1))):
                 raise SystemExit(f"parity gate ({name}): routing differs from the oracle")
+            xf = (x_np.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            wf = (lnps[li]["router_w"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            bound = (xf.shape[1] + 34) * 2.0 ** -22 * np.outer(np.linalg.norm(xf, axis=1), np.linalg.norm(wf, axis=1))
+            if lnps[li].get("router_bias") is not None:
+                bound = bound + 2.0 ** -21 * np.abs(lnps[li]["router_bias"].astype(np.float64))[None, :]
+            if not np.all(np.abs(log_g.astype(np.float64) - r["logits"]) <= bound * 1.01 + 1e-6):
+                raise SystemExit(f"parity gate ({name}): router logits outside the stated bound")
             if li >= sample_layers:
                 continue
             got = out.cpu().numpy().view(np.uint16)
@@ -437,7 +446,7 @@ class Bench:
             if not np.all(err <= tol):
                 raise SystemExit(f"parity gate ({name}): output outside tolerance (worst {float(np.max(err / tol)):.3f})")
             worst = max(worst, float(np.max(err / tol)))
-        return (f"ok: ids and logits bit-exact for all {T} tokens x {len(Ls)} layer(s); output within "
+        return (f"ok: ids and selected logits bit-exact (others within the stated bound) for all {T} tokens x {len(Ls)} layer(s); output within "
                 f"4e-3*S+1e-3 on {min(T, n_sample)} sampled tokens x {min(len(Ls), sample_layers)} layer(s), "
                 f"worst |err|/tol {worst:.3f}")
 

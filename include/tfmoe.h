@@ -13,6 +13,12 @@
  *   y = a . deq(Wdown_e)^T                                            down projection
  *   out[t,h] = bf16( sum_s g[t,s] * y_s[h] )                          weighted combine
  *
+ * Optional steps on either side of the routed path (tfmoe_forward_add_norm):
+ *   y_sh = the shared expert, an FFN of the same form and formats with width Is,
+ *          that every token passes through with weight 1, added into the combine;
+ *   out  = bf16( sum_s g[t,s] * y_s + y_sh + residual )               residual add
+ *   out_norm = bf16( out * gamma / sqrt(mean_h(out^2) + eps) )         RMS norm
+ *
  *   deq(W)[r,c] = E2M1(code[r,c]) * E4M3(scale[r, c/16]) * global
  *
  * Passages this follows:
@@ -27,6 +33,10 @@
  *  - The chain router -> top-k -> plan -> routed experts -> weighted combine:
  *    TensorFold issue #627, comment "Where the 0.35 ms per step goes" and
  *    the per-launch kernel table (router, topk, add_moe_norm).
+ *  - The shared expert beside the routed ones, and the combine fused with the
+ *    residual add and the norm (add_moe_norm): the same comment and table.
+ *    The pages do not spell out their arithmetic; this library takes the
+ *    readings stated at tfmoe_forward_add_norm.
  *  - E2M1 and E4M3 bit layouts: OCP Microscaling (MX) format definitions.
  *
  * Threading: handles are not thread-safe; use one handle per host thread or
@@ -77,6 +87,10 @@ typedef struct tfmoe_layer tfmoe_layer;   /* opaque */
  *   max_tokens >= 1.
  * This build additionally needs H % 128 == 0, I % 64 == 0 and num_experts <= 256
  * (else TFMOE_ERR_UNSUPPORTED).
+ * shared_intermediate: 0, or the shared expert's width Is, a multiple of I; the
+ * library runs it as m = Is / I extra expert slots that every token takes with
+ * weight 1 (needs num_experts + m <= 256 and top_k + m <= 32).
+ * norm_eps: the RMS norm's epsilon (>= 0), used by tfmoe_forward_add_norm.
  */
 typedef struct {
     int32_t hidden;            /* H */
@@ -90,6 +104,8 @@ typedef struct {
                                   regime, the others the tcgen05 tensor-core regime;
                                   <= 0 selects the built-in crossover: every expert in the
                                   GEMV regime while T <= 16, else 2 tokens */
+    int32_t shared_intermediate; /* Is: width of the shared expert, 0 = none */
+    float norm_eps;            /* epsilon of the RMS norm */
 } tfmoe_layer_desc;
 
 /*
@@ -111,6 +127,16 @@ typedef struct {
     const uint8_t  *down_codes;     /* [E][H][I/2] */
     const uint8_t  *down_scales;    /* e4m3 [E][H][I/16] */
     const float    *down_global;    /* [E] */
+    /* The shared expert, read only when shared_intermediate > 0 (same formats): */
+    const uint8_t  *shared_gate_codes;   /* [Is][H/2] */
+    const uint8_t  *shared_up_codes;     /* [Is][H/2] */
+    const uint8_t  *shared_gate_scales;  /* e4m3 [Is][H/16] */
+    const uint8_t  *shared_up_scales;    /* e4m3 [Is][H/16] */
+    const float    *shared_gate_global;  /* [1] */
+    const float    *shared_up_global;    /* [1] */
+    const uint8_t  *shared_down_codes;   /* [H][Is/2] */
+    const uint8_t  *shared_down_scales;  /* e4m3 [H][Is/16] */
+    const float    *shared_down_global;  /* [1] */
 } tfmoe_weights;
 
 /* Create a layer handle on the current CUDA device and allocate its
@@ -142,6 +168,25 @@ TFMOE_API tfmoe_status tfmoe_forward(tfmoe_layer *layer, const uint16_t *x, int3
                            uint16_t *out, void *cuda_stream);
 
 /*
+ * The layer followed by the residual add and the RMS norm, fused into the
+ * combine (the add_moe_norm step of TensorFold issue #627's per-launch table):
+ *   out[t,h]      = bf16( sum_s g[t,s] y_s[t,h] + y_sh[t,h] + residual[t,h] )
+ *   out_norm[t,h] = bf16( out[t,h] * norm_w[h] / sqrt(mean_h out[t,h]^2 + eps) )
+ * with y_sh the shared expert (when the descriptor has one) and eps the
+ * descriptor's norm_eps. Readings of the pages: the shared expert rounds its
+ * SwiGLU output to bf16 like a routed expert; the residual joins the same sum,
+ * rounded once; the norm reads the rounded out (the new residual stream).
+ * DEVICE pointers, bf16 bits, 16-byte aligned, caller-owned: residual [T][H] or
+ * NULL (no add); norm_w [H] or NULL (no norm: out_norm is not written and may
+ * be NULL); out [T][H]; out_norm [T][H]. residual may be the same array as out
+ * (the residual stream updated in place); otherwise none of x, residual, out
+ * and out_norm may overlap. Everything else as tfmoe_forward.
+ */
+TFMOE_API tfmoe_status tfmoe_forward_add_norm(tfmoe_layer *layer, const uint16_t *x, int32_t T,
+                                              const uint16_t *residual, const uint16_t *norm_w,
+                                              uint16_t *out, uint16_t *out_norm, void *cuda_stream);
+
+/*
  * Same computation with HOST buffers: x_host[T][H] is copied to the
  * device, the layer runs, and the result is copied into out_host[T][H];
  * all on `cuda_stream`, and the call returns after the result has arrived
@@ -165,20 +210,29 @@ TFMOE_API const char *tfmoe_last_error(void);
  * Intermediate buffers of the last forward, for inspection (tests, tools).
  * Returns a DEVICE pointer into the handle's workspace and its size in
  * bytes; contents are valid after the forward has completed on its stream.
- * Layouts (P = T*k pairs, rows of the permuted order r = 0..P-1, grouped by
- * expert in ascending (expert, token, slot) order):
+ * Layouts (P = T*(k+m) pairs, m the shared expert's slots (0 without one), rows
+ * of the permuted order r = 0..P-1, grouped by expert slot in ascending
+ * (slot, token, token's slot) order):
  */
 typedef enum {
-    TFMOE_BUF_LOGITS = 0,     /* fp32 [T][E] router logits (bias included) */
-    TFMOE_BUF_TOPK_IDS = 1,   /* int32 [T][k] selected experts, slot 0 = largest logit */
-    TFMOE_BUF_TOPK_WEIGHTS = 2, /* fp32 [T][k] softmax weights over the selected logits */
-    TFMOE_BUF_EXPERT_COUNTS = 3, /* int32 [E] tokens routed to each expert */
-    TFMOE_BUF_EXPERT_OFFSETS = 4, /* int32 [E+1] exclusive prefix sum of the counts */
+    TFMOE_BUF_LOGITS = 0,     /* fp32 [T][E] router logits (bias included). For T <= 16 every
+                                 entry is the exact logit. For T > 16 the entries of every
+                                 expert that could be in the token's top k -- the k selected
+                                 ones included -- are exact; the others hold the tensor-core
+                                 approximation, within (H + 34) 2^-22 ||x_t|| ||w_e|| +
+                                 2^-21 |bias_e| of the exact value. */
+    TFMOE_BUF_TOPK_IDS = 1,   /* int32 [T][k+m] selected experts, slot 0 = largest logit; with a
+                                 shared expert of m = Is/I slots, slots k..k+m-1 hold the
+                                 shared slots E..E+m-1 */
+    TFMOE_BUF_TOPK_WEIGHTS = 2, /* fp32 [T][k+m] softmax weights over the selected logits
+                                   (1 in the shared slots) */
+    TFMOE_BUF_EXPERT_COUNTS = 3, /* int32 [E+m] tokens routed to each expert slot */
+    TFMOE_BUF_EXPERT_OFFSETS = 4, /* int32 [E+m+1] exclusive prefix sum of the counts */
     TFMOE_BUF_PERM = 5,       /* int32 [P] pair index t*k+s held by permuted row r */
     TFMOE_BUF_INV = 6,        /* int32 [P] permuted row of pair t*k+s */
     TFMOE_BUF_ACT = 7,        /* bf16 [P][I] SwiGLU output a, permuted rows */
     TFMOE_BUF_EXPERT_OUT = 8, /* fp32 [P][H] down-projection output y, permuted rows */
-    TFMOE_BUF_REGIME = 9      /* int32 [E] 0 = not routed, 1 = GEMV regime, 2 = MMA regime */
+    TFMOE_BUF_REGIME = 9      /* int32 [E+m] 0 = not routed, 1 = GEMV regime, 2 = MMA regime */
 } tfmoe_buffer;
 
 TFMOE_API tfmoe_status tfmoe_get_buffer(tfmoe_layer *layer, tfmoe_buffer which, void **dev_ptr, size_t *bytes);
@@ -202,7 +256,7 @@ typedef enum {
     TFMOE_STAGE_GEMV_DOWN = 4,    /* GEMV regime: down projection */
     TFMOE_STAGE_MMA_GATE_UP = 5,  /* tensor-core regime: gate/up projections + SwiGLU */
     TFMOE_STAGE_MMA_DOWN = 6,     /* tensor-core regime: down projection */
-    TFMOE_STAGE_COMBINE = 7,      /* weighted combine */
+    TFMOE_STAGE_COMBINE = 7,      /* weighted combine (+ residual add and norm in tfmoe_forward_add_norm) */
     TFMOE_STAGE_GATHER = 8,       /* tensor-core regime: activation row gather */
     TFMOE_STAGE_COUNT = 9
 } tfmoe_stage;

@@ -58,13 +58,15 @@ struct Carver {
 };
 
 void carve_workspace(Layer &L, uint8_t *base, size_t *total) {
-    const size_t T = L.desc.max_tokens, E = L.desc.num_experts, k = L.desc.top_k;
+    // E: expert slots (routed + shared), k: slots per token; the logits cover the routed experts
+    const size_t T = L.desc.max_tokens, E = expert_slots(L), k = token_slots(L);
     const size_t H = L.desc.hidden, I = L.desc.intermediate, P = T * k;
     Workspace &w = L.ws;
     Carver c;
-    c.take(&w.logits, T * E, base);
-    L.router_partial_cap = std::min(kRouterPartialMax, (size_t)kRouterMaxSlices * T * E);
-    c.take(&w.router_partial, L.router_partial_cap, base);
+    c.take(&w.logits, T * L.desc.num_experts, base);
+    c.take(&w.xnorm, T, base);
+    c.take(&w.cand_cnt, T, base);
+    c.take(&w.cand, T * kRouterMaxCand, base);
     c.take(&w.ids, P, base);
     c.take(&w.topk_w, P, base);
     c.take(&w.counts, E, base);
@@ -96,11 +98,12 @@ void carve_workspace(Layer &L, uint8_t *base, size_t *total) {
 }
 
 void carve_weights(Layer &L, uint8_t *base, size_t *total) {
-    const size_t E = L.desc.num_experts, H = L.desc.hidden, I = L.desc.intermediate;
+    const size_t E = expert_slots(L), ER = L.desc.num_experts, H = L.desc.hidden, I = L.desc.intermediate;
     Weights &w = L.w;
     Carver c;
-    c.take(&w.router_w, E * H, base);
-    c.take(&w.router_bias, E, base);
+    c.take(&w.router_w, ER * H, base);
+    c.take(&w.router_cst, ER, base);
+    c.take(&w.router_bias, ER, base);
     c.take(&w.gu_codes, E * 2 * I * H / 2, base);
     c.take(&w.gu_scales, E * 2 * I * H / 16, base);
     c.take(&w.d_codes, E * H * I / 2, base);
@@ -161,12 +164,20 @@ tfmoe_status tfmoe_create(const tfmoe_layer_desc *desc, tfmoe_layer **out)
     if (d.hidden > kMaxReduction || d.intermediate > kMaxReduction)
         return fail(TFMOE_ERR_UNSUPPORTED, "this build supports hidden and intermediate up to %d (got %d, %d)",
                     kMaxReduction, d.hidden, d.intermediate);
-    if (d.num_experts > 256 || d.top_k > 32)
-        return fail(TFMOE_ERR_UNSUPPORTED, "this build supports num_experts <= 256 and top_k <= 32");
-    if ((long long)d.max_tokens * d.top_k > (1LL << 30))
-        return fail(TFMOE_ERR_UNSUPPORTED, "max_tokens * top_k too large");
-    if ((long long)d.max_tokens * d.top_k * (d.hidden > d.intermediate ? d.hidden : d.intermediate) >= (1LL << 32))
-        return fail(TFMOE_ERR_UNSUPPORTED, "max_tokens * top_k * max(hidden, intermediate) must stay below 2^32");
+    if (d.shared_intermediate < 0 || d.shared_intermediate % d.intermediate)
+        return fail(TFMOE_ERR_INVALID_ARG, "shared_intermediate (%d) must be 0 or a multiple of intermediate (%d)",
+                    d.shared_intermediate, d.intermediate);
+    if (!(d.norm_eps >= 0.f) || d.norm_eps == __builtin_inff())
+        return fail(TFMOE_ERR_INVALID_ARG, "norm_eps must be finite and >= 0");
+    const long long m = d.shared_intermediate / d.intermediate;
+    if (d.num_experts + m > 256 || d.top_k + m > 32)
+        return fail(TFMOE_ERR_UNSUPPORTED, "this build supports num_experts + m <= 256 and top_k + m <= 32 "
+                    "(m = shared_intermediate / intermediate = %lld)", m);
+    const long long kx = d.top_k + m;
+    if ((long long)d.max_tokens * kx > (1LL << 30))
+        return fail(TFMOE_ERR_UNSUPPORTED, "max_tokens * (top_k + m) too large");
+    if ((long long)d.max_tokens * kx * (d.hidden > d.intermediate ? d.hidden : d.intermediate) >= (1LL << 32))
+        return fail(TFMOE_ERR_UNSUPPORTED, "max_tokens * (top_k + m) * max(hidden, intermediate) must stay below 2^32");
 
     const char *fail_env = getenv("TFMOE_FAIL_ALLOC");
     if (fail_env && atoi(fail_env) != 0)
@@ -198,7 +209,9 @@ tfmoe_status tfmoe_create(const tfmoe_layer_desc *desc, tfmoe_layer **out)
     if (e == cudaSuccess) e = cudaMemset(L.ws.plan_counter, 0, sizeof(int32_t));
     if (e == cudaSuccess) e = gemv_setup(L);
     if (e == cudaSuccess) e = mma_setup(L);
+    if (e == cudaSuccess) e = router_setup(L);
     if (e != cudaSuccess) {
+        router_teardown(L);
         mma_teardown(L);
         gemv_teardown(L);
         cudaFree(L.ws_block);
@@ -227,6 +240,22 @@ tfmoe_status tfmoe_load_weights(tfmoe_layer *layer, const tfmoe_weights *w)
     for (const void *p : sc)
         if (reinterpret_cast<uintptr_t>(p) & 3u)
             return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_load_weights: scales must be 4-byte aligned");
+    const int m = shared_slots(L);
+    if (m > 0) {
+        const void *sh[] = {w->shared_gate_codes, w->shared_up_codes, w->shared_gate_scales, w->shared_up_scales,
+                            w->shared_gate_global, w->shared_up_global, w->shared_down_codes,
+                            w->shared_down_scales, w->shared_down_global};
+        for (const void *p : sh)
+            if (!p) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_load_weights: a shared-expert weight pointer is NULL");
+        const void *shv[] = {w->shared_gate_codes, w->shared_up_codes, w->shared_down_codes};
+        for (const void *p : shv)
+            if (!aligned16(p))
+                return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_load_weights: shared codes must be 16-byte aligned");
+        const void *shs[] = {w->shared_gate_scales, w->shared_up_scales, w->shared_down_scales};
+        for (const void *p : shs)
+            if (reinterpret_cast<uintptr_t>(p) & 3u)
+                return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_load_weights: shared scales must be 4-byte aligned");
+    }
 
     DeviceGuard dg(L.device);
     const size_t E = L.desc.num_experts, H = L.desc.hidden;
@@ -239,7 +268,16 @@ tfmoe_status tfmoe_load_weights(tfmoe_layer *layer, const tfmoe_weights *w)
     if (e == cudaSuccess) e = cudaMemcpyAsync(L.w.gate_global, w->gate_global, E * 4, cudaMemcpyDeviceToDevice, s);
     if (e == cudaSuccess) e = cudaMemcpyAsync(L.w.up_global, w->up_global, E * 4, cudaMemcpyDeviceToDevice, s);
     if (e == cudaSuccess) e = cudaMemcpyAsync(L.w.down_global, w->down_global, E * 4, cudaMemcpyDeviceToDevice, s);
+    // every shared slot carries the shared expert's per-tensor multipliers
+    for (int j = 0; j < m && e == cudaSuccess; ++j) {
+        e = cudaMemcpyAsync(L.w.gate_global + E + j, w->shared_gate_global, 4, cudaMemcpyDeviceToDevice, s);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(L.w.up_global + E + j, w->shared_up_global, 4, cudaMemcpyDeviceToDevice, s);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(L.w.down_global + E + j, w->shared_down_global, 4, cudaMemcpyDeviceToDevice, s);
+    }
     if (e == cudaSuccess) e = launch_repack(L, *w, s);
+    if (e == cudaSuccess) e = launch_router_norms(L, s);
     cudaError_t e2 = cudaStreamSynchronize(s);
     cudaStreamDestroy(s);
     if (e == cudaSuccess) e = e2;
@@ -248,21 +286,40 @@ tfmoe_status tfmoe_load_weights(tfmoe_layer *layer, const tfmoe_weights *w)
     return ok();
 }
 
-tfmoe_status tfmoe_forward(tfmoe_layer *layer, const uint16_t *x, int32_t T, uint16_t *out, void *cuda_stream)
+}  // extern "C"
+
+namespace {
+
+bool overlap(const void *a, const void *b, size_t bytes) {
+    if (!a || !b) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + bytes && y < x + bytes;
+}
+
+// The forward chain; residual, norm_w and out_norm are the optional epilogue (see
+// tfmoe_forward_add_norm), all NULL for tfmoe_forward.
+tfmoe_status forward_impl(tfmoe_layer *layer, const char *who, const uint16_t *x, int32_t T,
+                          const uint16_t *residual, const uint16_t *norm_w, uint16_t *out, uint16_t *out_norm,
+                          void *cuda_stream)
 {
-    if (!layer) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward: layer is NULL");
+    if (!layer) return fail(TFMOE_ERR_INVALID_ARG, "%s: layer is NULL", who);
     Layer &L = layer->impl;
     L.last_launches = 0;
-    if (!L.loaded) return fail(TFMOE_ERR_NOT_LOADED, "tfmoe_forward: weights not loaded");
+    if (!L.loaded) return fail(TFMOE_ERR_NOT_LOADED, "%s: weights not loaded", who);
     if (T < 0 || T > L.desc.max_tokens)
-        return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward: T=%d outside [0, max_tokens=%d]", T, L.desc.max_tokens);
+        return fail(TFMOE_ERR_INVALID_ARG, "%s: T=%d outside [0, max_tokens=%d]", who, T, L.desc.max_tokens);
     if (T == 0) return ok();
-    if (!x || !out) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward: x or out is NULL");
-    if (!aligned16(x) || !aligned16(out))
-        return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward: x and out must be 16-byte aligned");
+    if (!x || !out) return fail(TFMOE_ERR_INVALID_ARG, "%s: x or out is NULL", who);
+    if (norm_w && !out_norm) return fail(TFMOE_ERR_INVALID_ARG, "%s: norm_w given but out_norm is NULL", who);
+    if (!norm_w) out_norm = nullptr;
+    if (!aligned16(x) || !aligned16(out) || !aligned16(residual) || !aligned16(norm_w) || !aligned16(out_norm))
+        return fail(TFMOE_ERR_INVALID_ARG, "%s: x, out, residual, norm_w and out_norm must be 16-byte aligned", who);
     const size_t bytes = (size_t)T * L.desc.hidden * 2;
-    const uintptr_t xa = reinterpret_cast<uintptr_t>(x), oa = reinterpret_cast<uintptr_t>(out);
-    if (xa < oa + bytes && oa < xa + bytes) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_forward: out overlaps x");
+    if (overlap(x, out, bytes) || overlap(x, out_norm, bytes) || overlap(out, out_norm, bytes) ||
+        overlap(residual, out_norm, bytes) || overlap(residual, x, bytes) ||
+        (residual != out && overlap(residual, out, bytes)))
+        return fail(TFMOE_ERR_INVALID_ARG, "%s: overlapping x / residual / out / out_norm (only residual == out "
+                    "is allowed)", who);
 
     DeviceGuard dg(L.device);
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
@@ -280,11 +337,11 @@ tfmoe_status tfmoe_forward(tfmoe_layer *layer, const uint16_t *x, int32_t T, uin
     if (e == cudaSuccess && use_gemv) e = launch_gemv_gate_up(L, x, T, s, &n);
     if (e == cudaSuccess && use_mma) e = launch_mma_down(L, s, &n);
     if (e == cudaSuccess && use_gemv) e = launch_gemv_down(L, T, s, &n);
-    if (e == cudaSuccess) e = launch_combine(L, T, out, s, &n);
+    if (e == cudaSuccess) e = launch_combine(L, T, out, s, &n, residual, norm_w, out_norm);
     L.last_use_mma = use_mma;
     L.last_use_gemv = use_gemv;
     L.last_launches = n;
-    if (e != cudaSuccess) return cuda_fail(e, "tfmoe_forward: launch");
+    if (e != cudaSuccess) return cuda_fail(e, who);
     L.last_T = T;
     if (L.profiling) {
         e = cudaStreamSynchronize(s);
@@ -296,9 +353,24 @@ tfmoe_status tfmoe_forward(tfmoe_layer *layer, const uint16_t *x, int32_t T, uin
             L.prof_calls[st] += 1;
             L.prof_used[st] = false;
         }
-        if (e != cudaSuccess) return cuda_fail(e, "tfmoe_forward: profiling events");
+        if (e != cudaSuccess) return cuda_fail(e, "profiling events");
     }
     return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+tfmoe_status tfmoe_forward(tfmoe_layer *layer, const uint16_t *x, int32_t T, uint16_t *out, void *cuda_stream)
+{
+    return forward_impl(layer, "tfmoe_forward", x, T, nullptr, nullptr, out, nullptr, cuda_stream);
+}
+
+tfmoe_status tfmoe_forward_add_norm(tfmoe_layer *layer, const uint16_t *x, int32_t T, const uint16_t *residual,
+                                    const uint16_t *norm_w, uint16_t *out, uint16_t *out_norm, void *cuda_stream)
+{
+    return forward_impl(layer, "tfmoe_forward_add_norm", x, T, residual, norm_w, out, out_norm, cuda_stream);
 }
 
 tfmoe_status tfmoe_forward_host(tfmoe_layer *layer, const uint16_t *x_host, int32_t T, uint16_t *out_host,
@@ -352,6 +424,7 @@ void tfmoe_destroy(tfmoe_layer *layer)
                 if (ev) cudaEventDestroy(ev);
         if (L.ws_block) cudaFree(L.ws_block);
         if (L.w_block) cudaFree(L.w_block);
+        router_teardown(L);
         mma_teardown(L);
         gemv_teardown(L);
     }
@@ -362,10 +435,10 @@ tfmoe_status tfmoe_get_buffer(tfmoe_layer *layer, tfmoe_buffer which, void **dev
 {
     if (!layer || !dev_ptr || !bytes) return fail(TFMOE_ERR_INVALID_ARG, "tfmoe_get_buffer: NULL argument");
     Layer &L = layer->impl;
-    const size_t T = L.desc.max_tokens, E = L.desc.num_experts, k = L.desc.top_k;
+    const size_t T = L.desc.max_tokens, E = expert_slots(L), k = token_slots(L);
     const size_t H = L.desc.hidden, I = L.desc.intermediate, P = T * k;
     switch (which) {
-    case TFMOE_BUF_LOGITS: *dev_ptr = L.ws.logits; *bytes = T * E * 4; break;
+    case TFMOE_BUF_LOGITS: *dev_ptr = L.ws.logits; *bytes = T * L.desc.num_experts * 4; break;
     case TFMOE_BUF_TOPK_IDS: *dev_ptr = L.ws.ids; *bytes = P * 4; break;
     case TFMOE_BUF_TOPK_WEIGHTS: *dev_ptr = L.ws.topk_w; *bytes = P * 4; break;
     case TFMOE_BUF_EXPERT_COUNTS: *dev_ptr = L.ws.counts; *bytes = E * 4; break;

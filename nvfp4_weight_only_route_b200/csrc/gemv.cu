@@ -307,6 +307,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_kernel(const __grid
                                                                     const GemvArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
+    // gate/up is launched as a programmatic dependent of the kernel before it (the routing
+    // kernel at decode sizes): everything it reads comes from that grid, so it waits first,
+    // before it lets the down projection launch
+    if (P == Proj::GateUp) grid_dep_wait();
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     const int K = a.K, KT = K / kTileK, KS = a.KS, RG = a.RG;
     const int rows_task = 16 * RG, KTW = KT / KS;
@@ -675,7 +679,7 @@ struct GemvMaps {
 // The shape for a batch of T tokens: long when the GEMV list (at most min(E, T k)
 // experts) gives each CTA kLongTasksPerCta long tasks.
 const GemvShape &pick_shape(const Layer &L, const GemvShape (&sh)[2], int R, int T) {
-    const int experts = min(L.desc.num_experts, T * L.desc.top_k);
+    const int experts = min(expert_slots(L), T * token_slots(L));
     const long long tasks = (long long)experts * (R / (16 * sh[1].g.RG));
     return (sh[1].g.KS != sh[0].g.KS && tasks >= (long long)kLongTasksPerCta * sh[1].grid) ? sh[1] : sh[0];
 }
@@ -684,7 +688,7 @@ const GemvShape &pick_shape(const Layer &L, const GemvShape (&sh)[2], int R, int
 
 cudaError_t gemv_setup(Layer &L)
 {
-    const int H = L.desc.hidden, I = L.desc.intermediate, E = L.desc.num_experts;
+    const int H = L.desc.hidden, I = L.desc.intermediate, E = expert_slots(L);
     GemvMaps *gm = new (std::nothrow) GemvMaps();
     if (!gm) return cudaErrorMemoryAllocation;
     gm->gu[0].g = geometry(true, H);
@@ -738,7 +742,7 @@ void gemv_teardown(Layer &L)
 static GemvArgs common_args(const Layer &L) {
     GemvArgs g{};
     g.expert_list = L.ws.gemv_list; g.list_size = L.ws.list_sizes;
-    g.offsets = L.ws.offsets; g.perm = L.ws.perm; g.top_k = L.desc.top_k;
+    g.offsets = L.ws.offsets; g.perm = L.ws.perm; g.top_k = token_slots(L);
     g.I = L.desc.intermediate; g.err_word = L.ws.err_word;
     g.test_wait_ns = 0;
     return g;
@@ -758,9 +762,19 @@ cudaError_t launch_gemv_gate_up(Layer &L, const uint16_t *x, int T, cudaStream_t
     g.src = L.ws.xq; g.src_inv = L.ws.xq_inv;
     g.act_out = L.ws.act; g.aq_out = L.ws.aq; g.aq_inv_out = L.ws.aq_inv;
     if (L.desc.flags & TFMOE_FLAG_TEST_TIMEOUT) g.test_wait_ns = kTestWaitNs;
-    gemv_kernel<Proj::GateUp><<<sh.grid, kThreads, sh.smem, s>>>(sh.map, g);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(sh.grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = sh.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = L.plain_order ? 0 : 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_kernel<Proj::GateUp>, sh.map, g);
     *launches += 1;
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_gemv_down(Layer &L, int T, cudaStream_t s, int *launches)

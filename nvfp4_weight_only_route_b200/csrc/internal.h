@@ -38,14 +38,18 @@ constexpr int kMaxReduction = 256 * kTileK;
 constexpr int kSmallBatchTokens = 16;
 constexpr int kDefaultGemvMaxTokens = 2;
 
-// Router for T > 16: at most this many hidden-dimension slices, and at most
-// kRouterPartialMax fp64 partial logits held at once.
-constexpr int kRouterMaxSlices = 16;
-constexpr size_t kRouterPartialMax = size_t(1) << 22;
+// Router for T > 16 (tensor-core approximation + exact candidates): the largest top_k,
+// and the candidate experts one token's list holds (beyond it the token takes every expert
+// exactly).
+constexpr int kRouterMaxK = 32;
+constexpr int kRouterMaxCand = 64;
 
 // Batches with more than this many (token, expert) pairs build the plan with a
 // multi-CTA scan instead of one CTA.
 constexpr int kLargePlanPairs = 4096;
+// Tokens per segment of the multi-CTA plan: the router's last kernel writes each segment's
+// expert histogram (one CTA of warps per segment, one warp per token).
+constexpr int kPlanSegTokens = 8;
 
 // Tokens per tensor-core tile (the MMA N dimension): up to kMmaTileTokens with one CTA
 // per SM, or up to kMmaSmallTileTokens with two CTAs per SM when a batch averages at most
@@ -57,7 +61,9 @@ __host__ __device__ constexpr size_t max_mma_entries(size_t P, size_t E) { retur
 
 struct Workspace {
     float *logits = nullptr;        // [maxT][E]
-    double *router_partial = nullptr; // [router_partial_cap] fp64 partial logits of hidden-dimension slices
+    float *xnorm = nullptr;         // [maxT] upper bound of ||x_t||_2 (router, T > 16)
+    int32_t *cand_cnt = nullptr;    // [maxT] router candidates per token, -1 = every expert
+    uint16_t *cand = nullptr;       // [maxT][kRouterMaxCand] router candidate experts
     int32_t *ids = nullptr;         // [maxT][k]
     float *topk_w = nullptr;        // [maxT][k]
     int32_t *counts = nullptr;      // [E]
@@ -89,14 +95,16 @@ struct Workspace {
 
 struct Weights {
     uint16_t *router_w = nullptr;   // [E][H] bf16
+    float4 *router_cst = nullptr;   // [E] router bound constants {bias, C_e, B_e, 0} (router_tc.cu)
     float *router_bias = nullptr;   // [E]
-    uint8_t *gu_codes = nullptr;    // [E][2I/128][H/64] tiles (gate row j -> 2j, up row j -> 2j+1)
+    // Expert-slot arrays hold the E routed experts, then the shared expert's m = Is/I slots.
+    uint8_t *gu_codes = nullptr;    // [E+m][2I/128][H/64] tiles (gate row j -> 2j, up row j -> 2j+1)
     uint8_t *gu_scales = nullptr;
-    uint8_t *d_codes = nullptr;     // [E][H/128][I/64] tiles
+    uint8_t *d_codes = nullptr;     // [E+m][H/128][I/64] tiles
     uint8_t *d_scales = nullptr;
-    float *gate_global = nullptr;   // [E]
-    float *up_global = nullptr;     // [E]
-    float *down_global = nullptr;   // [E]
+    float *gate_global = nullptr;   // [E+m]
+    float *up_global = nullptr;     // [E+m]
+    float *down_global = nullptr;   // [E+m]
 };
 
 struct Layer {
@@ -115,7 +123,7 @@ struct Layer {
     int32_t last_T = -1;            // T of the last successful forward (stage replays need it)
     bool last_use_mma = false, last_use_gemv = false;
     bool mma_small = false;         // the tensor-core regime of the current forward uses small tiles
-    size_t router_partial_cap = 0;  // doubles in ws.router_partial
+    void *router_maps = nullptr;    // tensor map of the router weights (router_tc.cu)
     void *gemv_maps = nullptr;      // tensor maps of the GEMV regime's scale slabs
     void *mma_maps = nullptr;       // tensor maps of the MMA regime's token operands
     // per-stage profiling (tfmoe_profile_enable)
@@ -140,6 +148,15 @@ struct StageTimer {
     }
 };
 
+// The shared expert runs as m = Is / I extra expert slots E..E+m-1 that every token takes
+// with weight 1: the plan, the expert kernels and the combine see E+m slots and k+m slots
+// per token; the router and top-k see the E routed experts and k.
+inline int shared_slots(const Layer &L) {
+    return L.desc.shared_intermediate > 0 ? L.desc.shared_intermediate / L.desc.intermediate : 0;
+}
+inline int expert_slots(const Layer &L) { return L.desc.num_experts + shared_slots(L); }
+inline int token_slots(const Layer &L) { return L.desc.top_k + shared_slots(L); }
+
 // Per-expert token count up to which the GEMV regime is used, for a batch of T tokens.
 inline int gemv_threshold(const Layer &L, int T) {
     if (L.gemv_max_tokens > 0) return L.gemv_max_tokens;
@@ -149,11 +166,20 @@ inline int gemv_threshold(const Layer &L, int T) {
 // Launchers. Each returns cudaGetLastError() after its launches and adds
 // the number of kernels it enqueued to *launches.
 cudaError_t launch_router(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches);
+cudaError_t launch_router_tc(Layer &L, const uint16_t *x, int T, bool gemv, int32_t *seg_cnt, cudaStream_t s,
+                             int *launches);
+cudaError_t launch_router_norms(const Layer &L, cudaStream_t s);
+cudaError_t router_setup(Layer &L);
+void router_teardown(Layer &L);
 cudaError_t launch_permute(Layer &L, int T, cudaStream_t s, int *launches);
 cudaError_t launch_gemv(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches);
 cudaError_t launch_gemv_gate_up(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches);
 cudaError_t launch_gemv_down(Layer &L, int T, cudaStream_t s, int *launches);
-cudaError_t launch_combine(Layer &L, int T, uint16_t *out, cudaStream_t s, int *launches);
+// Weighted combine into out; with residual, added before the rounding; with norm_w, also
+// the RMS norm of out into out_norm (one CTA per token).
+cudaError_t launch_combine(Layer &L, int T, uint16_t *out, cudaStream_t s, int *launches,
+                           const uint16_t *residual = nullptr, const uint16_t *norm_w = nullptr,
+                           uint16_t *out_norm = nullptr);
 cudaError_t launch_repack(const Layer &L, const tfmoe_weights &src, cudaStream_t s);
 cudaError_t gemv_setup(Layer &L);
 void gemv_teardown(Layer &L);

@@ -413,7 +413,9 @@ __global__ void __launch_bounds__(C::kThreads, C::kCtasPerSm) mma_kernel(const _
                     sm.xi_s[ew][c] = (c < rows) ? __ldg(a.row_inv_scale + row0 + c) : 0.f;
                 __syncwarp();
             }
-            if (!wait_or_abort(&sm.dfull[buf], (tile_i / C::kDBufs) & 1u, &sm.abort_flag, a.err_word)) break;
+            if (!__all_sync(0xffffffffu, wait_or_abort(&sm.dfull[buf], (tile_i / C::kDBufs) & 1u, &sm.abort_flag,
+                                                       a.err_word)))
+                break;                           // warp-uniform: the loads below are warp-collective
             tc_fence_after();
             const int grow = rt * kM + q;
             const uint32_t dcol = tmem + lane_base + (uint32_t)buf * kMaxN;
@@ -576,12 +578,12 @@ struct MmaMaps {
 };
 
 bool mma_use_small_tiles(const Layer &L, int T) {
-    return (long long)T * L.desc.top_k <= (long long)kMmaSmallMaxAvgTokens * L.desc.num_experts;
+    return (long long)T * token_slots(L) <= (long long)kMmaSmallMaxAvgTokens * expert_slots(L);
 }
 
 cudaError_t mma_setup(Layer &L)
 {
-    const int maxP = L.desc.max_tokens * L.desc.top_k;
+    const int maxP = L.desc.max_tokens * token_slots(L);
     const int H = L.desc.hidden, I = L.desc.intermediate;
     MmaMaps *mm = new (std::nothrow) MmaMaps();
     if (!mm) return cudaErrorMemoryAllocation;
@@ -607,10 +609,10 @@ void mma_teardown(Layer &L)
 cudaError_t launch_gather(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches)
 {
     StageTimer timer(L, TFMOE_STAGE_GATHER, s);
-    const int P = T * L.desc.top_k;
-    dim3 grid((unsigned)max_mma_entries(P, L.desc.num_experts), 16);
+    const int P = T * token_slots(L);
+    dim3 grid((unsigned)max_mma_entries(P, expert_slots(L)), 16);
     gather_kernel<<<grid, 256, 0, s>>>(x, L.ws.perm, L.ws.mma_entries, L.ws.list_sizes, L.desc.hidden,
-                                       L.desc.top_k, L.ws.x_perm, L.ws.row_inv);
+                                       token_slots(L), L.ws.x_perm, L.ws.row_inv);
     *launches += 1;
     return cudaGetLastError();
 }

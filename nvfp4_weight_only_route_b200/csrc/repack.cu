@@ -15,9 +15,13 @@ namespace tfmoe {
 namespace {
 
 // One thread per (expert, tiled row, column tile): copies 2 x 16 code bytes and 4 scale bytes.
+// Source row r of expert e starts at element (e * rows + r) * K; with split_ld > 0 the source
+// is one matrix of rows of split_ld elements whose column block [e*K, (e+1)*K) is expert e
+// (the shared expert's down projection, cut along its reduction dimension into slots).
 __global__ void repack_kernel(const uint8_t *__restrict__ codes_a, const uint8_t *__restrict__ scales_a,
                               const uint8_t *__restrict__ codes_b, const uint8_t *__restrict__ scales_b,
-                              int E, int R, int K, uint8_t *__restrict__ out_codes, uint8_t *__restrict__ out_scales)
+                              int E, int R, int K, uint8_t *__restrict__ out_codes, uint8_t *__restrict__ out_scales,
+                              int split_ld = 0)
 {
     // interleaved (codes_b != nullptr): tiled row r -> source (r & 1 ? b : a) row r >> 1
     const int KT = K / kTileK, RT = R / kTileRows;
@@ -39,9 +43,10 @@ __global__ void repack_kernel(const uint8_t *__restrict__ codes_a, const uint8_t
             sc = codes_a;
             sr = scales_a;
         }
-        const size_t row_off = (size_t)e * src_rows + src_row;
-        const uint8_t *crow = sc + row_off * (K / 2) + (size_t)kt * 32;
-        const uint8_t *srow = sr + row_off * (K / 16) + (size_t)kt * 4;
+        const size_t elem = split_ld > 0 ? (size_t)src_row * split_ld + (size_t)e * K
+                                         : ((size_t)e * src_rows + src_row) * K;
+        const uint8_t *crow = sc + elem / 2 + (size_t)kt * 32;
+        const uint8_t *srow = sr + elem / 16 + (size_t)kt * 4;
         const size_t tile = ((size_t)e * RT + r / kTileRows) * KT + kt;
         uint8_t *ct = out_codes + tile * kTileCodeBytes + (r % kTileRows) * 16;
         *reinterpret_cast<uint4 *>(ct) = *reinterpret_cast<const uint4 *>(crow);
@@ -61,6 +66,20 @@ cudaError_t launch_repack(const Layer &L, const tfmoe_weights &src, cudaStream_t
                                                  E, 2 * I, H, L.w.gu_codes, L.w.gu_scales);
     repack_kernel<<<4 * L.num_sms, 256, 0, s>>>(src.down_codes, src.down_scales, nullptr, nullptr,
                                                  E, H, I, L.w.d_codes, L.w.d_scales);
+    const int m = shared_slots(L);
+    if (m > 0) {
+        // the shared expert's m slots follow the routed experts: gate/up rows [m][I] as m
+        // experts, the down projection's columns cut into m blocks of I
+        const size_t gu_tiles = (size_t)E * (2 * I / kTileRows) * (H / kTileK);
+        const size_t d_tiles = (size_t)E * (H / kTileRows) * (I / kTileK);
+        repack_kernel<<<4 * L.num_sms, 256, 0, s>>>(src.shared_gate_codes, src.shared_gate_scales,
+                                                     src.shared_up_codes, src.shared_up_scales, m, 2 * I, H,
+                                                     L.w.gu_codes + gu_tiles * kTileCodeBytes,
+                                                     L.w.gu_scales + gu_tiles * kTileScaleBytes);
+        repack_kernel<<<4 * L.num_sms, 256, 0, s>>>(src.shared_down_codes, src.shared_down_scales, nullptr, nullptr,
+                                                     m, H, I, L.w.d_codes + d_tiles * kTileCodeBytes,
+                                                     L.w.d_scales + d_tiles * kTileScaleBytes, m * I);
+    }
     return cudaGetLastError();
 }
 

@@ -143,180 +143,6 @@ __global__ void __launch_bounds__(256) router_tiled_kernel(
     }
 }
 
-// Layer path for T > 16: (16M tokens x 16M experts) tiles, M = 2 or 4, over a z-range of
-// the hidden dimension each. With one z-slice the CTA rounds its fp64 sums to fp32 and
-// adds the bias; with several it writes fp64 partial sums [z][T][E] that the top-k
-// kernel adds in z order. Small batches get small tiles and many slices, so the grid
-// still covers the GPU.
-template <int M>
-__global__ void __launch_bounds__(256) router_split_kernel(
-    const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, const float *__restrict__ bias,
-    float *__restrict__ logits, double *__restrict__ partial, int T, int H, int E, int k_len, int32_t *err_word,
-    int debug, uint16_t *xq, float *xq_inv)
-{
-    constexpr int TT = 16 * M, TE = 16 * M, KC = 32;
-    __shared__ double xs[KC][TT + 1];
-    __shared__ double ws[KC][TE + 1];
-    const int t_base = blockIdx.x * TT, e_base = blockIdx.y * TE, k_begin = blockIdx.z * k_len;
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    double acc[M][M];
-#pragma unroll
-    for (int i = 0; i < M; ++i)
-#pragma unroll
-        for (int j = 0; j < M; ++j) acc[i][j] = 0.0;
-    for (int k0 = k_begin; k0 < k_begin + k_len; k0 += KC) {
-        // TT rows x 32 columns of x and of wr: 8 elements per item
-        for (int i = threadIdx.x; i < TT * KC / 8; i += 256) {
-            const int row = i / (KC / 8), col = (i % (KC / 8)) * 8;
-            const int t = t_base + row, e = e_base + row;
-            uint4 xv = make_uint4(0, 0, 0, 0), wv = make_uint4(0, 0, 0, 0);
-            if (t < T) xv = *reinterpret_cast<const uint4 *>(x + (size_t)t * H + k0 + col);
-            if (e < E) wv = *reinterpret_cast<const uint4 *>(wr + (size_t)e * H + k0 + col);
-            const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w}, wu[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                xs[col + 2 * j][row] = (double)bf16_bits_to_float(xu[j] & 0xFFFFu);
-                xs[col + 2 * j + 1][row] = (double)bf16_bits_to_float(xu[j] >> 16);
-                ws[col + 2 * j][row] = (double)bf16_bits_to_float(wu[j] & 0xFFFFu);
-                ws[col + 2 * j + 1][row] = (double)bf16_bits_to_float(wu[j] >> 16);
-            }
-        }
-        __syncthreads();
-#pragma unroll 4
-        for (int kk = 0; kk < KC; ++kk) {
-            double xv[M], wv[M];
-#pragma unroll
-            for (int i = 0; i < M; ++i) xv[i] = xs[kk][ty + 16 * i];
-#pragma unroll
-            for (int j = 0; j < M; ++j) wv[j] = ws[kk][tx + 16 * j];
-#pragma unroll
-            for (int i = 0; i < M; ++i)
-#pragma unroll
-                for (int j = 0; j < M; ++j) acc[i][j] = fma(xv[i], wv[j], acc[i][j]);
-        }
-        __syncthreads();
-    }
-#pragma unroll
-    for (int i = 0; i < M; ++i) {
-        const int t = t_base + ty + 16 * i;
-        if (t >= T) continue;
-#pragma unroll
-        for (int j = 0; j < M; ++j) {
-            const int e = e_base + tx + 16 * j;
-            if (e >= E) continue;
-            if (partial) {
-                partial[((size_t)blockIdx.z * T + t) * E + e] = acc[i][j];
-            } else {
-                float l = (float)acc[i][j];
-                if (bias) l = l + bias[e];
-                if (debug && !isfinite(l)) atomicOr(err_word, DEV_ERR_NONFINITE);
-                logits[(size_t)t * E + e] = l;
-            }
-        }
-    }
-    // the CTAs of the first expert tile also write the GEMV regime's x operand for their
-    // tokens and hidden-dimension slice (16-element blocks, see block16_bf16_to_f16)
-    if (xq && blockIdx.y == 0) {
-        const int rows = min(TT, T - t_base), blocks = k_len / 16;
-        for (int i = threadIdx.x; i < rows * blocks; i += blockDim.x) {
-            const int t = t_base + i / blocks;
-            const size_t off = (size_t)t * H + k_begin + (size_t)(i % blocks) * 16;
-            xq_inv[off / 16] = block16_bf16_to_f16(x + off, xq + off);
-        }
-    }
-}
-
-// Layer path for larger batches on the fp64 tensor cores: mma.sync m8n8k4 f64 (each
-// product of two bf16 values is exact in fp64, sums accumulate in fp64 as in the scalar
-// kernel). CTA tile 64 tokens x 64 experts over a z-slice of the hidden dimension, staged
-// 32 columns at a time as fp64 in shared memory; warp (wm, wn) of 2 x 4 owns 32 tokens x
-// 16 experts = 4 x 2 tiles of 8 x 8. Output as router_split_kernel (fp32 logits + bias, or
-// fp64 partials [z][T][E]) and the same x conversion by the first expert-tile column.
-__device__ __forceinline__ void dmma_8x8x4(double &d0, double &d1, double a, double b) {
-    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
-                 : "+d"(d0), "+d"(d1) : "d"(a), "d"(b));
-}
-
-__global__ void __launch_bounds__(256) router_dmma_kernel(
-    const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, const float *__restrict__ bias,
-    float *__restrict__ logits, double *__restrict__ partial, int T, int H, int E, int k_len, int32_t *err_word,
-    int debug, uint16_t *xq, float *xq_inv)
-{
-    constexpr int TT = 64, TE = 64, KC = 32, LD = KC + 2;   // row stride in doubles
-    __shared__ double xs[TT * LD];
-    __shared__ double ws[TE * LD];
-    const int t_base = blockIdx.x * TT, e_base = blockIdx.y * TE, k_begin = blockIdx.z * k_len;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int wm = warp >> 2, wn = warp & 3;                 // 2 x 4 warps
-    const int g = lane >> 2, q = lane & 3;                   // fragment row group / thread in group
-    double acc[4][2][2];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 2; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
-    for (int k0 = k_begin; k0 < k_begin + k_len; k0 += KC) {
-        // 64 rows x 32 columns of x and of wr, 8 bf16 per item, converted to fp64
-        for (int i = threadIdx.x; i < TT * KC / 8; i += 256) {
-            const int row = i / (KC / 8), col = (i % (KC / 8)) * 8;
-            const int t = t_base + row, e = e_base + row;
-            uint4 xv = make_uint4(0, 0, 0, 0), wv = make_uint4(0, 0, 0, 0);
-            if (t < T) xv = *reinterpret_cast<const uint4 *>(x + (size_t)t * H + k0 + col);
-            if (e < E) wv = *reinterpret_cast<const uint4 *>(wr + (size_t)e * H + k0 + col);
-            const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w}, wu[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                xs[row * LD + col + 2 * j] = (double)bf16_bits_to_float(xu[j] & 0xFFFFu);
-                xs[row * LD + col + 2 * j + 1] = (double)bf16_bits_to_float(xu[j] >> 16);
-                ws[row * LD + col + 2 * j] = (double)bf16_bits_to_float(wu[j] & 0xFFFFu);
-                ws[row * LD + col + 2 * j + 1] = (double)bf16_bits_to_float(wu[j] >> 16);
-            }
-        }
-        __syncthreads();
-#pragma unroll
-        for (int kk = 0; kk < KC; kk += 4) {
-            double a[4], b[2];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = xs[(wm * 32 + i * 8 + g) * LD + kk + q];      // A[token g][k q]
-#pragma unroll
-            for (int j = 0; j < 2; ++j) b[j] = ws[(wn * 16 + j * 8 + g) * LD + kk + q];      // B[k q][expert g]
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 2; ++j) dmma_8x8x4(acc[i][j][0], acc[i][j][1], a[i], b[j]);
-        }
-        __syncthreads();
-    }
-    // D[row g][col 2q + c] of each 8 x 8 tile
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int t = t_base + wm * 32 + i * 8 + g;
-        if (t >= T) continue;
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                const int e = e_base + wn * 16 + j * 8 + 2 * q + c;
-                if (e >= E) continue;
-                if (partial) {
-                    partial[((size_t)blockIdx.z * T + t) * E + e] = acc[i][j][c];
-                } else {
-                    float l = (float)acc[i][j][c];
-                    if (bias) l = l + bias[e];
-                    if (debug && !isfinite(l)) atomicOr(err_word, DEV_ERR_NONFINITE);
-                    logits[(size_t)t * E + e] = l;
-                }
-            }
-    }
-    if (xq && blockIdx.y == 0) {
-        const int rows = min(TT, T - t_base), blocks = k_len / 16;
-        for (int i = threadIdx.x; i < rows * blocks; i += blockDim.x) {
-            const int t = t_base + i / blocks;
-            const size_t off = (size_t)t * H + k_begin + (size_t)(i % blocks) * 16;
-            xq_inv[off / 16] = block16_bf16_to_f16(x + off, xq + off);
-        }
-    }
-}
-
 // One warp per token: k rounds of a warp arg-max over (logit desc, index asc),
 // then softmax over the selected logits (max-subtracted, fp32).
 constexpr int kMaxEPerLane = 8;   // E <= 256
@@ -331,9 +157,10 @@ __device__ __forceinline__ uint32_t logit_key(float v) {
 
 // One warp selects a token's top k experts: k rounds, each a lane-local best (largest key,
 // lowest expert on ties) followed by a warp-wide max of the keys and a min of the expert ids
-// that hold it (two redux.sync), so ties go to the lower expert index.
+// that hold it (two redux.sync), so ties go to the lower expert index. With m shared slots the
+// row continues with slots k..k+m-1 = experts E..E+m-1 at weight 1 (the shared expert).
 __device__ __forceinline__ void topk_warp(const float *row, int E, int k, int32_t *ids_row, float *w_row,
-                                          int32_t *ids_copy = nullptr)
+                                          int32_t *ids_copy = nullptr, int m = 0)
 {
     const int lane = threadIdx.x & 31;
     float v[kMaxEPerLane];
@@ -377,6 +204,10 @@ __device__ __forceinline__ void topk_warp(const float *row, int E, int k, int32_
         ids_row[lane] = my_id;
         w_row[lane] = ex / den;
         if (ids_copy) ids_copy[lane] = my_id;
+    } else if (lane < k + m) {
+        ids_row[lane] = E + lane - k;
+        w_row[lane] = 1.f;
+        if (ids_copy) ids_copy[lane] = E + lane - k;
     }
 }
 
@@ -391,47 +222,13 @@ __device__ __forceinline__ void convert_x_blocks(const uint16_t *__restrict__ x,
     }
 }
 
-// One warp per token; with xq given, the grid also writes the GEMV regime's x operand.
-// With S > 1 fp64 partial sums [S][T][E], the warp first adds them in slice order,
-// rounds once to fp32, adds the bias and stores the token's logits.
-// Tokens per top-k CTA (one warp each); a CTA's pairs form one segment of the plan.
-constexpr int kTopkTokens = 8;
-
-__global__ void __launch_bounds__(256) topk_kernel(
-    float *__restrict__ logits, int32_t *__restrict__ ids, float *__restrict__ wts, int T, int E, int k,
-    const uint16_t *__restrict__ x, int H, uint16_t *xq, float *xq_inv, const double *__restrict__ partial, int S,
-    const float *__restrict__ bias, int32_t *err_word, int debug, int32_t *seg_cnt)
+// One warp per token of full logits: top k and softmax weights (the allocation-free routing).
+__global__ void __launch_bounds__(256) topk_kernel(const float *__restrict__ logits, int32_t *__restrict__ ids,
+                                                   float *__restrict__ wts, int T, int E, int k)
 {
-    __shared__ int32_t ids_s[kTopkTokens * 32];
-    __shared__ int32_t cnt_s[256];
-    if (xq) convert_x_blocks(x, T, H, xq, xq_inv);
-    if (seg_cnt)
-        for (int e = threadIdx.x; e < E; e += blockDim.x) cnt_s[e] = 0;
-    const int warp = threadIdx.x >> 5;
-    const int t = blockIdx.x * kTopkTokens + warp;
-    if (t < T) {
-        if (partial) {
-            for (int e = threadIdx.x & 31; e < E; e += 32) {
-                double v = 0.0;
-                for (int z = 0; z < S; ++z) v += partial[((size_t)z * T + t) * E + e];
-                float l = (float)v;
-                if (bias) l = l + bias[e];
-                if (debug && !isfinite(l)) atomicOr(err_word, DEV_ERR_NONFINITE);
-                logits[(size_t)t * E + e] = l;
-            }
-            __syncwarp();
-        }
-        topk_warp(logits + (size_t)t * E, E, k, ids + (size_t)t * k, wts + (size_t)t * k, ids_s + warp * k);
-    }
-    if (!seg_cnt) return;
-    // this segment's expert histogram, for the multi-CTA plan
-    __syncthreads();
-    const int n = min(kTopkTokens, T - (int)blockIdx.x * kTopkTokens) * k;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) atomicAdd(&cnt_s[ids_s[i]], 1);
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) seg_cnt[(size_t)blockIdx.x * E + e] = cnt_s[e];
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t < T) topk_warp(logits + (size_t)t * E, E, k, ids + (size_t)t * k, wts + (size_t)t * k);
 }
-
 
 // The expert plan, computed by one CTA of W warps. Pairs p = t*k + s are split
 // into W contiguous segments, one per warp. Pass 1 counts per (segment,
@@ -696,9 +493,9 @@ __global__ void __launch_bounds__(256) plan_place_kernel(const int32_t *__restri
                                                          const int32_t *__restrict__ offsets, int E,
                                                          int32_t *__restrict__ perm, int32_t *__restrict__ inv)
 {
-    __shared__ int32_t ids_s[kTopkTokens * 32];
-    const int p0 = blockIdx.x * kTopkTokens * k;
-    const int n = min(kTopkTokens * k, P - p0);
+    __shared__ int32_t ids_s[kPlanSegTokens * 32];
+    const int p0 = blockIdx.x * kPlanSegTokens * k;
+    const int n = min(kPlanSegTokens * k, P - p0);
     for (int i = threadIdx.x; i < n; i += blockDim.x) ids_s[i] = ids[p0 + i];
     __syncthreads();
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
@@ -721,17 +518,19 @@ __global__ void __launch_bounds__(256) plan_place_kernel(const int32_t *__restri
 // block is the launch-saving shape proposed in TensorFold issue #627 (comment
 // on the fused tf_nemo_route_row experiment).
 constexpr int kFusedMaxT = 16;
-// Batches of at least this many tokens take the router on the fp64 tensor cores.
-constexpr int kRouterDmmaMinTokens = 128;
 constexpr int kFusedThreads = 256;
 __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(
     const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, const float *__restrict__ bias,
     float *__restrict__ logits, int32_t *__restrict__ ids, float *__restrict__ wts, int T, int H, int k,
-    PlanArgs pa, int32_t *counter, uint16_t *xq, float *xq_inv)
+    PlanArgs pa, int32_t *counter, uint16_t *xq, float *xq_inv, int m)
 {
     extern __shared__ int32_t sm[];
     __shared__ int is_last;
-    const int E = pa.E, e = blockIdx.x;
+    // one CTA per routed expert; the plan (pa.E) also covers the m shared slots
+    const int E = (int)gridDim.x, e = blockIdx.x, kx = k + m;
+    // the GEMV gate/up grid may launch now: its CTAs take their places and wait for this
+    // grid to complete before they read anything
+    grid_dep_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // logits of expert e: warp w takes tokens w, w + 8 (T <= 16); lane l covers 8 columns per
     // 256-column step, and the warp adds its lanes in a fixed shuffle order
@@ -777,9 +576,9 @@ __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(
     // the ids stay in shared memory for the plan: no global round trip on the serial tail
     __shared__ int32_t ids_sm[kFusedMaxT * 32];
     for (int t = warp; t < T; t += kFusedThreads / 32)
-        topk_warp(logits + (size_t)t * E, E, k, ids + (size_t)t * k, wts + (size_t)t * k, ids_sm + t * k);
+        topk_warp(logits + (size_t)t * E, E, k, ids + (size_t)t * kx, wts + (size_t)t * kx, ids_sm + t * kx, m);
     __syncthreads();
-    plan_block(ids_sm, T * k, pa, sm);
+    plan_block(ids_sm, T * kx, pa, sm);
     if (threadIdx.x == 0) *counter = 0;
 }
 
@@ -787,7 +586,7 @@ __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(
 
 static PlanArgs plan_args(const Layer &L, int T) {
     PlanArgs pa{};
-    pa.E = L.desc.num_experts;
+    pa.E = expert_slots(L);
     pa.gemv_max_tokens = gemv_threshold(L, T);
     pa.mma_tile = L.mma_small ? kMmaSmallTileTokens : kMmaTileTokens;
     pa.flags = L.desc.flags;
@@ -802,68 +601,38 @@ static PlanArgs plan_args(const Layer &L, int T) {
 bool route_fused_applies(const Layer &, int T) { return T <= kFusedMaxT; }
 
 static bool large_plan(const Layer &L, int T) {
-    return T > kFusedMaxT && (long long)T * L.desc.top_k > kLargePlanPairs;
+    return T > kFusedMaxT && (long long)T * token_slots(L) > kLargePlanPairs;
 }
 
 cudaError_t launch_router(Layer &L, const uint16_t *x, int T, cudaStream_t s, int *launches)
 {
     const int H = L.desc.hidden, E = L.desc.num_experts, k = L.desc.top_k;
-    const int debug = (L.desc.flags & TFMOE_FLAG_DEBUG_CHECKS) ? 1 : 0;
     const float *bias = L.desc.has_router_bias ? L.w.router_bias : nullptr;
     const bool gemv = !(L.desc.flags & TFMOE_FLAG_FORCE_MMA);   // the GEMV regime may run: write its x operand
     if (route_fused_applies(L, T)) {
         // router, top-k and plan in one launch (the permute launcher then does nothing)
         StageTimer timer(L, TFMOE_STAGE_ROUTER, s);
-        const size_t smem = sizeof(int32_t) * plan_smem_ints(kFusedThreads / 32, E);
+        const size_t smem = sizeof(int32_t) * plan_smem_ints(kFusedThreads / 32, expert_slots(L));
         route_fused_kernel<<<E, kFusedThreads, smem, s>>>(x, L.w.router_w, bias, L.ws.logits, L.ws.ids,
                                                           L.ws.topk_w, T, H, k, plan_args(L, T), L.ws.route_counter,
-                                                          gemv ? L.ws.xq : nullptr, L.ws.xq_inv);
+                                                          gemv ? L.ws.xq : nullptr, L.ws.xq_inv, shared_slots(L));
         *launches += 1;
         return cudaGetLastError();
     }
-    // tile size and hidden-dimension slices: enough CTAs for two per SM where possible
-    const bool dmma = T >= kRouterDmmaMinTokens;
-    const int M = (T >= 2048) ? 4 : 2, tile = dmma ? 64 : 16 * M;
-    const int tiles = ((T + tile - 1) / tile) * ((E + tile - 1) / tile);
-    int S = 1;
-    if (tiles < 2 * L.num_sms) {
-        S = std::min(kRouterMaxSlices, (2 * L.num_sms + tiles - 1) / tiles);
-        while (S > 1 && ((H / 32) % S || (size_t)S * T * E > L.router_partial_cap)) --S;
-    }
-    double *partial = (S > 1) ? L.ws.router_partial : nullptr;
-    {
-        StageTimer timer(L, TFMOE_STAGE_ROUTER, s);
-        dim3 grid((T + tile - 1) / tile, (E + tile - 1) / tile, S);
-        if (dmma)
-            router_dmma_kernel<<<grid, 256, 0, s>>>(x, L.w.router_w, bias, L.ws.logits, partial, T, H, E, H / S,
-                                                    L.ws.err_word, debug, gemv ? L.ws.xq : nullptr, L.ws.xq_inv);
-        else if (M == 4)
-            router_split_kernel<4><<<grid, 256, 0, s>>>(x, L.w.router_w, bias, L.ws.logits, partial, T, H, E, H / S,
-                                                        L.ws.err_word, debug, gemv ? L.ws.xq : nullptr, L.ws.xq_inv);
-        else
-            router_split_kernel<2><<<grid, 256, 0, s>>>(x, L.w.router_w, bias, L.ws.logits, partial, T, H, E, H / S,
-                                                        L.ws.err_word, debug, gemv ? L.ws.xq : nullptr, L.ws.xq_inv);
-    }
-    {
-        StageTimer timer(L, TFMOE_STAGE_TOPK, s);
-        topk_kernel<<<(T + kTopkTokens - 1) / kTopkTokens, 256, 0, s>>>(
-            L.ws.logits, L.ws.ids, L.ws.topk_w, T, E, k, x, H, nullptr, nullptr, partial, S, bias, L.ws.err_word, debug,
-            large_plan(L, T) ? L.ws.seg_cnt : nullptr);
-    }
-    *launches += 2;
-    return cudaGetLastError();
+    // larger batches: tensor-core approximate logits, exact candidates, exact top k
+    return launch_router_tc(L, x, T, gemv, large_plan(L, T) ? L.ws.seg_cnt : nullptr, s, launches);
 }
 
 cudaError_t launch_permute(Layer &L, int T, cudaStream_t s, int *launches)
 {
     if (route_fused_applies(L, T)) return cudaSuccess;
     StageTimer timer(L, TFMOE_STAGE_PERMUTE, s);
-    const int E = L.desc.num_experts, P = T * L.desc.top_k;
+    const int E = expert_slots(L), kx = token_slots(L), P = T * kx;
     if (large_plan(L, T)) {
-        const int nseg = (T + kTopkTokens - 1) / kTopkTokens;
+        const int nseg = (T + kPlanSegTokens - 1) / kPlanSegTokens;
         plan_scan_kernel<<<E, 256, 0, s>>>(L.ws.seg_cnt, nseg, L.ws.seg_base, L.ws.plan_tot, L.ws.plan_counter,
                                            plan_args(L, T));
-        plan_place_kernel<<<nseg, 256, 0, s>>>(L.ws.ids, P, L.desc.top_k, L.ws.seg_base, L.ws.offsets, E, L.ws.perm,
+        plan_place_kernel<<<nseg, 256, 0, s>>>(L.ws.ids, P, kx, L.ws.seg_base, L.ws.offsets, E, L.ws.perm,
                                                L.ws.inv);
         *launches += 2;
         return cudaGetLastError();
@@ -1000,8 +769,7 @@ extern "C" tfmoe_status tfmoe_route_noalloc(const uint16_t *x, int32_t T, int32_
         dim3 grid((T + RT_T - 1) / RT_T, (E + RT_E - 1) / RT_E);
         router_tiled_kernel<<<grid, 256, 0, s>>>(x, router_w, router_bias, logits, T, H, E, nullptr, 0);
     }
-    topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(logits, ids_out, weights_out, T, E, k, x, H, nullptr, nullptr, nullptr,
-                                            1, nullptr, nullptr, 0, nullptr);
+    topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(logits, ids_out, weights_out, T, E, k);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return record_error(TFMOE_ERR_CUDA, "tfmoe_route_noalloc: launch: %s", cudaGetErrorString(e));

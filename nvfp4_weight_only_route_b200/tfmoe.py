@@ -28,7 +28,8 @@ BUF_LOGITS, BUF_TOPK_IDS, BUF_TOPK_WEIGHTS, BUF_EXPERT_COUNTS, BUF_EXPERT_OFFSET
 
 EXPORTED = ["tfmoe_create", "tfmoe_load_weights", "tfmoe_forward", "tfmoe_forward_host", "tfmoe_sync_status",
             "tfmoe_destroy", "tfmoe_last_error", "tfmoe_get_buffer", "tfmoe_last_launch_count",
-            "tfmoe_profile_enable", "tfmoe_profile_read", "tfmoe_route_noalloc", "tfmoe_forward_stage"]
+            "tfmoe_profile_enable", "tfmoe_profile_read", "tfmoe_route_noalloc", "tfmoe_forward_stage",
+            "tfmoe_forward_add_norm"]
 
 ROUTE_NOALLOC_MAX_LOGITS = 1 << 20
 
@@ -40,13 +41,17 @@ class LayerDesc(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int32), ("intermediate", ctypes.c_int32),
                 ("num_experts", ctypes.c_int32), ("top_k", ctypes.c_int32),
                 ("max_tokens", ctypes.c_int32), ("has_router_bias", ctypes.c_int32),
-                ("flags", ctypes.c_uint32), ("gemv_max_tokens", ctypes.c_int32)]
+                ("flags", ctypes.c_uint32), ("gemv_max_tokens", ctypes.c_int32),
+                ("shared_intermediate", ctypes.c_int32), ("norm_eps", ctypes.c_float)]
 
 
 class Weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "router_w", "router_bias", "gate_codes", "up_codes", "gate_scales", "up_scales",
-        "gate_global", "up_global", "down_codes", "down_scales", "down_global")]
+        "gate_global", "up_global", "down_codes", "down_scales", "down_global",
+        "shared_gate_codes", "shared_up_codes", "shared_gate_scales", "shared_up_scales",
+        "shared_gate_global", "shared_up_global", "shared_down_codes", "shared_down_scales",
+        "shared_down_global")]
 
 
 class TfmoeError(RuntimeError):
@@ -73,6 +78,8 @@ def load_library(path: str = LIB_PATH):
     lib.tfmoe_load_weights.restype = ctypes.c_int
     lib.tfmoe_forward.argtypes = [vp, vp, i32, vp, vp]
     lib.tfmoe_forward.restype = ctypes.c_int
+    lib.tfmoe_forward_add_norm.argtypes = [vp, vp, i32, vp, vp, vp, vp, vp]
+    lib.tfmoe_forward_add_norm.restype = ctypes.c_int
     lib.tfmoe_forward_host.argtypes = [vp, vp, i32, vp, vp]
     lib.tfmoe_forward_host.restype = ctypes.c_int
     lib.tfmoe_sync_status.argtypes = [vp, vp]
@@ -122,10 +129,11 @@ class MoELayer:
     """One NVFP4 W4A16 MoE FFN layer held by libtfmoe on the current CUDA device."""
 
     def __init__(self, hidden: int, intermediate: int, num_experts: int, top_k: int, max_tokens: int,
-                 has_router_bias: bool = False, flags: int = 0, gemv_max_tokens: int = 0):
+                 has_router_bias: bool = False, flags: int = 0, gemv_max_tokens: int = 0,
+                 shared_intermediate: int = 0, norm_eps: float = 1e-6):
         self.lib = load_library()
         self.desc = LayerDesc(hidden, intermediate, num_experts, top_k, max_tokens,
-                              1 if has_router_bias else 0, flags, gemv_max_tokens)
+                              1 if has_router_bias else 0, flags, gemv_max_tokens, shared_intermediate, norm_eps)
         h = ctypes.c_void_p()
         check(self.lib.tfmoe_create(ctypes.byref(self.desc), ctypes.byref(h)))
         self.handle = h
@@ -144,6 +152,22 @@ class MoELayer:
             out = torch.empty((T, self.desc.hidden), dtype=torch.bfloat16, device=x.device)
         check(self.lib.tfmoe_forward(self.handle, _ptr(x), T, _ptr(out), _stream_handle(stream)))
         return out
+
+    def forward_add_norm(self, x, residual=None, norm_w=None, out=None, out_norm=None, T: Optional[int] = None,
+                         stream=None):
+        """The layer, + residual (may be out itself), and with norm_w the RMS norm of the result
+        (tfmoe_forward_add_norm). Returns (out, out_norm or None)."""
+        import torch
+        if T is None:
+            T = x.shape[0]
+        if out is None:
+            out = torch.empty((T, self.desc.hidden), dtype=torch.bfloat16, device=x.device)
+        if norm_w is not None and out_norm is None:
+            out_norm = torch.empty((T, self.desc.hidden), dtype=torch.bfloat16, device=x.device)
+        check(self.lib.tfmoe_forward_add_norm(self.handle, _ptr(x), T, _ptr(residual), _ptr(norm_w), _ptr(out),
+                                              _ptr(out_norm) if norm_w is not None else None,
+                                              _stream_handle(stream)))
+        return out, (out_norm if norm_w is not None else None)
 
     def forward_raw(self, x_ptr: int, T: int, out_ptr: int, stream_handle: int) -> int:
         return self.lib.tfmoe_forward(self.handle, x_ptr, T, out_ptr, stream_handle)

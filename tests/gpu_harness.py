@@ -56,12 +56,36 @@ class GpuRun:
         self.layer.close()
 
 
-def check_routing(g, o, E, k):
-    """Router logits, ids (bit-exact), weights; then the expert permutation."""
+def logit_bound(x_bits, w_bits, bias=None):
+    """The bound on |approximate - exact| router logit the library states for the experts it
+    does not recompute exactly: (H + 34) 2^-22 ||x_t|| ||w_e|| + 2^-21 |bias_e| (with a 1 %
+    margin)."""
+    xf, wf = bf16_to_f64(x_bits), bf16_to_f64(w_bits)
+    H = xf.shape[1]
+    b = 0.0 if bias is None else 2.0 ** -21 * np.abs(np.asarray(bias, np.float64))[None, :]
+    return ((H + 34) * 2.0 ** -22 * np.outer(np.linalg.norm(xf, axis=1), np.linalg.norm(wf, axis=1)) + b) * 1.01 + 1e-6
+
+
+def check_logits(g_logits, o_logits, ids, bound=None):
+    """The logits of the selected experts are bit-exact. Every other entry is either exact or,
+    for batches routed through the tensor-core approximation, within `bound` of it."""
+    sel_g = np.take_along_axis(g_logits, ids, axis=1)
+    sel_o = np.take_along_axis(o_logits, ids, axis=1)
+    n_bad = int(np.sum(sel_g != sel_o))
+    assert n_bad == 0, f"{n_bad} router logits of selected experts differ from the oracle"
+    diff = np.abs(g_logits.astype(np.float64) - o_logits.astype(np.float64))
+    if bound is None:
+        assert np.all(diff == 0), f"{int(np.sum(diff != 0))} router logits differ from the oracle"
+    else:
+        assert np.all(diff <= bound), f"router logits off by more than the stated bound: {float(np.max(diff / bound)):.3f}"
+
+
+def check_routing(g, o, E, k, bound=None):
+    """Router logits (selected ones bit-exact), ids (bit-exact), weights; then the expert
+    permutation."""
     T = o["ids"].shape[0]
     assert np.array_equal(g["ids"], o["ids"]), "top-k ids differ from the oracle"
-    n_bad_logits = int(np.sum(g["logits"] != o["logits"]))
-    assert n_bad_logits == 0, f"{n_bad_logits} router logits differ from the oracle"
+    check_logits(g["logits"], o["logits"], o["ids"], bound)
     assert np.max(np.abs(g["g"].astype(np.float64) - o["g"])) <= 2e-6
     ids = o["ids"].ravel()
     counts = np.bincount(ids, minlength=E)

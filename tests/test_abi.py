@@ -44,8 +44,9 @@ def test_struct_layout_matches_header(tf):
 #include <stddef.h>
 #include "tfmoe.h"
 int main(void) {
-  printf("%zu %zu %zu %zu\\n", sizeof(tfmoe_layer_desc), offsetof(tfmoe_layer_desc, gemv_max_tokens),
-         sizeof(tfmoe_weights), offsetof(tfmoe_weights, down_global));
+  printf("%zu %zu %zu %zu %zu %zu %zu\\n", sizeof(tfmoe_layer_desc), offsetof(tfmoe_layer_desc, gemv_max_tokens),
+         sizeof(tfmoe_weights), offsetof(tfmoe_weights, down_global), offsetof(tfmoe_layer_desc, shared_intermediate),
+         offsetof(tfmoe_layer_desc, norm_eps), offsetof(tfmoe_weights, shared_down_global));
   return 0;
 }
 """
@@ -56,13 +57,14 @@ int main(void) {
         subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe])
         got = [int(v) for v in subprocess.check_output([exe]).split()]
     want = [ctypes.sizeof(tf.LayerDesc), tf.LayerDesc.gemv_max_tokens.offset,
-            ctypes.sizeof(tf.Weights), tf.Weights.down_global.offset]
+            ctypes.sizeof(tf.Weights), tf.Weights.down_global.offset, tf.LayerDesc.shared_intermediate.offset,
+            tf.LayerDesc.norm_eps.offset, tf.Weights.shared_down_global.offset]
     assert got == want
 
 
 def _create(tf, **kw):
     d = dict(hidden=512, intermediate=256, num_experts=8, top_k=2, max_tokens=4, has_router_bias=0,
-             flags=0, gemv_max_tokens=0)
+             flags=0, gemv_max_tokens=0, shared_intermediate=0, norm_eps=1e-6)
     d.update(kw)
     desc = tf.LayerDesc(**d)
     h = ctypes.c_void_p()
@@ -80,6 +82,11 @@ def _create(tf, **kw):
     (dict(num_experts=64, top_k=33), 5),
     (dict(max_tokens=(1 << 31) // 8, top_k=8, num_experts=8), 5),
     (dict(hidden=4096, max_tokens=131072, top_k=8, num_experts=8), 5),
+    # the shared expert: a multiple of the routed width; its slots count against E and k
+    (dict(shared_intermediate=128), 1), (dict(shared_intermediate=-256), 1),
+    (dict(norm_eps=-1.0), 1), (dict(norm_eps=float("nan")), 1), (dict(norm_eps=float("inf")), 1),
+    (dict(num_experts=255, shared_intermediate=512), 5),
+    (dict(num_experts=64, top_k=31, shared_intermediate=512), 5),
 ])
 def test_create_rejects_bad_descriptors_without_gpu(tf, kw, status):
     st, h = _create(tf, **kw)
@@ -106,6 +113,7 @@ def test_null_handle_calls(tf):
     lib = tf.load_library()
     assert lib.tfmoe_forward(None, None, 1, None, None) == tf.ERR_INVALID_ARG
     assert lib.tfmoe_forward_host(None, None, 1, None, None) == tf.ERR_INVALID_ARG
+    assert lib.tfmoe_forward_add_norm(None, None, 1, None, None, None, None, None) == tf.ERR_INVALID_ARG
     assert lib.tfmoe_load_weights(None, None) == tf.ERR_INVALID_ARG
     assert lib.tfmoe_sync_status(None, None) == tf.ERR_INVALID_ARG
     p, n = ctypes.c_void_p(), ctypes.c_size_t()
