@@ -65,6 +65,7 @@ void carve_workspace(Layer &L, uint8_t *base, size_t *total) {
     Carver c;
     c.take(&w.logits, T * L.desc.num_experts, base);
     c.take(&w.xnorm, T, base);
+    c.take(&w.xexp, T, base);
     c.take(&w.cand_cnt, T, base);
     c.take(&w.cand, T * kRouterMaxCand, base);
     c.take(&w.ids, P, base);
@@ -103,6 +104,7 @@ void carve_weights(Layer &L, uint8_t *base, size_t *total) {
     Carver c;
     c.take(&w.router_w, ER * H, base);
     c.take(&w.router_cst, ER, base);
+    c.take(&w.router_wexp, 2, base);
     c.take(&w.router_bias, ER, base);
     c.take(&w.gu_codes, E * 2 * I * H / 2, base);
     c.take(&w.gu_scales, E * 2 * I * H / 16, base);

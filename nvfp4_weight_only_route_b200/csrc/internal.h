@@ -62,6 +62,7 @@ __host__ __device__ constexpr size_t max_mma_entries(size_t P, size_t E) { retur
 struct Workspace {
     float *logits = nullptr;        // [maxT][E]
     float *xnorm = nullptr;         // [maxT] upper bound of ||x_t||_2 (router, T > 16)
+    int32_t *xexp = nullptr;        // [maxT] smallest | largest << 16 exponent field of x_t's nonzero elements
     int32_t *cand_cnt = nullptr;    // [maxT] router candidates per token, -1 = every expert
     uint16_t *cand = nullptr;       // [maxT][kRouterMaxCand] router candidate experts
     int32_t *ids = nullptr;         // [maxT][k]
@@ -96,6 +97,7 @@ struct Workspace {
 struct Weights {
     uint16_t *router_w = nullptr;   // [E][H] bf16
     float4 *router_cst = nullptr;   // [E] router bound constants {bias, C_e, B_e, 0} (router_tc.cu)
+    int32_t *router_wexp = nullptr; // [2] smallest and largest exponent field of the router weights' nonzero elements
     float *router_bias = nullptr;   // [E]
     // Expert-slot arrays hold the E routed experts, then the shared expert's m = Is/I slots.
     uint8_t *gu_codes = nullptr;    // [E+m][2I/128][H/64] tiles (gate row j -> 2j, up row j -> 2j+1)

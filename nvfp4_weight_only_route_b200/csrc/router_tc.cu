@@ -23,9 +23,11 @@
 // are the candidates. A token whose approximations are not finite, or that has more
 // candidates than the list holds, takes the exact path over every expert.
 //
-// Kernels: xprep (the row norms of x, and the GEMV regime's block-scaled x), the tensor-core
-// kernel (approximate logits, candidate lists), refine (exact candidates, top k, softmax
-// weights, the large-batch plan's segment histograms).
+// Kernels: xprep (the row norms of x and the exponent range of each row, and the GEMV
+// regime's block-scaled x), the tensor-core kernel (approximate logits, candidate lists),
+// refine (exact candidates, top k, softmax weights, the shared slots, the large-batch plan's
+// segment histograms). At weight load, router_consts_kernel computes each expert's bound
+// constants and the exponent range of the router weights.
 #include <algorithm>
 #include <new>
 
@@ -41,7 +43,7 @@ constexpr int kRtThreads = 256;     // warp 0: TMA, warp 1: TMEM + MMA issue, wa
 constexpr int kRtMaxN = 256;        // experts (MMA N, E rounded up to 16)
 
 struct RtArgs {
-    int T, H, E, k, n_pad;
+    int T, H, E, n_pad;
     const float *xnorm;             // [T]  upper bound of ||x_t||_2
     const float4 *cst;              // [E]  {bias, C_e, B_e, 0}: eps(t, e) = fma(xnorm_t, C_e, B_e)
     float *logits;                  // [T][E] approximations; the exact pass overwrites candidates
@@ -277,13 +279,28 @@ __global__ void __launch_bounds__(kRtThreads, 1) router_tc_kernel(const __grid_c
 
 // One warp per token: ||x_t||_2 (fp64 sum of squares, rounded up to fp32) and, for the
 // GEMV regime, x in f16 with a power of two per 16-element block.
+// The exponent field of a bf16 value folded into a running (smallest, largest) over nonzero
+// values (a subnormal counts as 0, an infinity or NaN as 255).
+__device__ __forceinline__ void exp_range(uint32_t b, uint32_t &emin, uint32_t &emax) {
+    if (b & 0x7FFFu) {
+        const uint32_t e = (b >> 7) & 0xFFu;
+        emin = min(emin, e);
+        emax = max(emax, e);
+    }
+}
+
+// One warp per token: ||x_t||_2 (fp64 sum of squares, rounded up to fp32), the exponent range
+// of x_t's nonzero elements, and, for the GEMV regime, x in f16 with a power of two per
+// 16-element block.
 __global__ void __launch_bounds__(256) xprep_kernel(const uint16_t *__restrict__ x, int T, int H,
-                                                    float *__restrict__ xnorm, uint16_t *xq, float *xq_inv)
+                                                    float *__restrict__ xnorm, int32_t *__restrict__ xexp, uint16_t *xq,
+                                                    float *xq_inv)
 {
     const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (t >= T) return;
     const uint16_t *row = x + (size_t)t * H;
     double ss = 0.0;
+    uint32_t emin = 255u, emax = 0u;
     for (int c = lane * 8; c < H; c += 256) {
         const uint4 v = *reinterpret_cast<const uint4 *>(row + c);
         const uint32_t u[4] = {v.x, v.y, v.z, v.w};
@@ -292,11 +309,18 @@ __global__ void __launch_bounds__(256) xprep_kernel(const uint16_t *__restrict__
             const double lo = bf16_bits_to_float(u[j] & 0xFFFFu), hi = bf16_bits_to_float(u[j] >> 16);
             ss = fma(lo, lo, ss);
             ss = fma(hi, hi, ss);
+            exp_range(u[j] & 0xFFFFu, emin, emax);
+            exp_range(u[j] >> 16, emin, emax);
         }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) xnorm[t] = (float)(sqrt(ss) * (1.0 + 0x1p-18));
+    emin = __reduce_min_sync(0xffffffffu, emin);
+    emax = __reduce_max_sync(0xffffffffu, emax);
+    if (lane == 0) {
+        xnorm[t] = (float)(sqrt(ss) * (1.0 + 0x1p-18));
+        xexp[t] = (int32_t)(emin | (emax << 16));
+    }
     if (xq)
         for (int b = lane; b < H / 16; b += 32) {
             const size_t off = (size_t)t * H + (size_t)b * 16;
@@ -308,18 +332,26 @@ __global__ void __launch_bounds__(256) xprep_kernel(const uint16_t *__restrict__
 // C_e = (H + 34) 2^-22 ||w_e|| and B_e = 2^-21 |b_e| + 2^-126, both rounded up (the
 // factor 1 + 2^-18 also covers the rounding of the fma that forms eps).
 __global__ void __launch_bounds__(256) router_consts_kernel(const uint16_t *__restrict__ w, const float *bias,
-                                                            int E, int H, float4 *__restrict__ cst)
+                                                            int E, int H, float4 *__restrict__ cst,
+                                                            int32_t *__restrict__ wexp)
 {
     const int e = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
     if (e >= E) return;
     double ss = 0.0;
+    uint32_t emin = 255u, emax = 0u;
     for (int c = lane; c < H; c += 32) {
-        const double v = bf16_bits_to_float(w[(size_t)e * H + c]);
+        const uint16_t b = w[(size_t)e * H + c];
+        const double v = bf16_bits_to_float(b);
         ss = fma(v, v, ss);
+        exp_range(b, emin, emax);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    emin = __reduce_min_sync(0xffffffffu, emin);
+    emax = __reduce_max_sync(0xffffffffu, emax);
     if (lane == 0) {
+        atomicMin(wexp, (int32_t)emin);
+        atomicMax(wexp + 1, (int32_t)emax);
         const double up = 1.0 + 0x1p-18;
         const double wn = sqrt(ss) * up;
         const float b = bias ? bias[e] : 0.f;
@@ -344,7 +376,7 @@ __global__ void __launch_bounds__(256) router_refine_kernel(
     const uint16_t *__restrict__ x, const uint16_t *__restrict__ wr, const float *__restrict__ bias, int T, int H,
     int E, int k, int m, float *__restrict__ logits, const int32_t *__restrict__ cand_cnt,
     const uint16_t *__restrict__ cand, int32_t *__restrict__ ids, float *__restrict__ wts, int32_t *err_word,
-    int debug, int32_t *seg_cnt)
+    int debug, int32_t *seg_cnt, const int32_t *__restrict__ xexp, const int32_t *__restrict__ wexp)
 {
     __shared__ int32_t ids_s[kRefTokens * 32];
     __shared__ int32_t cnt_s[256];
@@ -358,6 +390,15 @@ __global__ void __launch_bounds__(256) router_refine_kernel(
         const bool all = n < 0 || n > kRouterMaxCand;
         if (all) n = E;
         const uint16_t *xrow = x + (size_t)t * H;
+        // Every product of a bf16 x element and a bf16 weight is exact in fp32 (16 significant
+        // bits) when it lies in fp32's normal range: nonzero elements normal, and the exponent
+        // fields with ex + ew in [128, 380] for every pair. Then the fp64 accumulation of the fp32
+        // product, acc + (double)(x * w), rounds exactly like fma((double)x, (double)w, acc) and
+        // needs one fp32 -> fp64 conversion instead of two.
+        const int32_t xr = __ldg(xexp + t);
+        const int xmin = xr & 0xFFFF, xmax = xr >> 16, wmin = __ldg(wexp), wmax = __ldg(wexp + 1);
+        const bool fast = xmin >= 1 && wmin >= 1 && xmax <= 254 && wmax <= 254 && xmin + wmin >= 128 &&
+                          xmax + wmax <= 380;
         // candidate j sits in lane j % 32, slot j / 32 (n <= 256)
         uint32_t key[8];
         int eid[8];
@@ -368,14 +409,29 @@ __global__ void __launch_bounds__(256) router_refine_kernel(
             const int e = all ? j : min((int)__ldg(cand + (size_t)t * kRouterMaxCand + j), E - 1);
             const uint16_t *wrow = wr + (size_t)e * H;
             double acc = 0.0;
-            for (int c = lane * 8; c < H; c += 256) {
-                const uint4 xv = *reinterpret_cast<const uint4 *>(xrow + c);
-                const uint4 wv = *reinterpret_cast<const uint4 *>(wrow + c);
-                const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w}, wu[4] = {wv.x, wv.y, wv.z, wv.w};
+            if (fast) {
+#pragma unroll 4
+                for (int c = lane * 8; c < H; c += 256) {
+                    const uint4 xv = *reinterpret_cast<const uint4 *>(xrow + c);
+                    const uint4 wv = *reinterpret_cast<const uint4 *>(wrow + c);
+                    const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w}, wu[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    acc = fma((double)bf16_bits_to_float(xu[i] & 0xFFFFu), (double)bf16_bits_to_float(wu[i] & 0xFFFFu), acc);
-                    acc = fma((double)bf16_bits_to_float(xu[i] >> 16), (double)bf16_bits_to_float(wu[i] >> 16), acc);
+                    for (int i = 0; i < 4; ++i) {
+                        acc += (double)__fmul_rn(bf16_bits_to_float(xu[i] & 0xFFFFu), bf16_bits_to_float(wu[i] & 0xFFFFu));
+                        acc += (double)__fmul_rn(bf16_bits_to_float(xu[i] >> 16), bf16_bits_to_float(wu[i] >> 16));
+                    }
+                }
+            } else {
+#pragma unroll 4
+                for (int c = lane * 8; c < H; c += 256) {
+                    const uint4 xv = *reinterpret_cast<const uint4 *>(xrow + c);
+                    const uint4 wv = *reinterpret_cast<const uint4 *>(wrow + c);
+                    const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w}, wu[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        acc = fma((double)bf16_bits_to_float(xu[i] & 0xFFFFu), (double)bf16_bits_to_float(wu[i] & 0xFFFFu), acc);
+                        acc = fma((double)bf16_bits_to_float(xu[i] >> 16), (double)bf16_bits_to_float(wu[i] >> 16), acc);
+                    }
                 }
             }
 #pragma unroll
@@ -470,9 +526,13 @@ void router_teardown(Layer &L)
 
 cudaError_t launch_router_norms(const Layer &L, cudaStream_t s)
 {
+    // exponent range of the weights: smallest starts at 0x7F7F7F7F, largest at 0
+    cudaError_t e = cudaMemsetAsync(L.w.router_wexp, 0x7F, sizeof(int32_t), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(L.w.router_wexp + 1, 0, sizeof(int32_t), s);
+    if (e != cudaSuccess) return e;
     router_consts_kernel<<<(L.desc.num_experts + 7) / 8, 256, 0, s>>>(
         L.w.router_w, L.desc.has_router_bias ? L.w.router_bias : nullptr, L.desc.num_experts, L.desc.hidden,
-        L.w.router_cst);
+        L.w.router_cst, L.w.router_wexp);
     return cudaGetLastError();
 }
 
@@ -489,9 +549,10 @@ cudaError_t launch_router_tc(Layer &L, const uint16_t *x, int T, bool gemv, int3
     const float *bias = L.desc.has_router_bias ? L.w.router_bias : nullptr;
     {
         StageTimer timer(L, TFMOE_STAGE_ROUTER, s);
-        xprep_kernel<<<(T + 7) / 8, 256, 0, s>>>(x, T, H, L.ws.xnorm, gemv ? L.ws.xq : nullptr, L.ws.xq_inv);
+        xprep_kernel<<<(T + 7) / 8, 256, 0, s>>>(x, T, H, L.ws.xnorm, L.ws.xexp, gemv ? L.ws.xq : nullptr,
+                                                 L.ws.xq_inv);
         RtArgs a{};
-        a.T = T; a.H = H; a.E = E; a.k = k; a.n_pad = n_pad;
+        a.T = T; a.H = H; a.E = E; a.n_pad = n_pad;
         a.xnorm = L.ws.xnorm;
         a.cst = L.w.router_cst;
         a.logits = L.ws.logits;
@@ -519,7 +580,7 @@ cudaError_t launch_router_tc(Layer &L, const uint16_t *x, int T, bool gemv, int3
         router_refine_kernel<<<(T + kRefTokens - 1) / kRefTokens, 256, 0, s>>>(
             x, L.w.router_w, bias, T, H, E, k, shared_slots(L), L.ws.logits, L.ws.cand_cnt, L.ws.cand, L.ws.ids,
             L.ws.topk_w,
-            L.ws.err_word, (L.desc.flags & TFMOE_FLAG_DEBUG_CHECKS) ? 1 : 0, seg_cnt);
+            L.ws.err_word, (L.desc.flags & TFMOE_FLAG_DEBUG_CHECKS) ? 1 : 0, seg_cnt, L.ws.xexp, L.w.router_wexp);
     }
     *launches += 3;
     return cudaGetLastError();

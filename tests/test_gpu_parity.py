@@ -106,6 +106,41 @@ def test_wide_dynamic_range_activations(oracle_mod, regime, H, I, E, k, T):
     _full_check(oracle_mod, layer, x, H, I, E, k, REGIMES[regime])
 
 
+def test_router_exact_path_for_extreme_exponents(oracle_mod):
+    """The exact router recomputation forms bf16 x bf16 products in fp32 when every product is
+    a normal fp32 number, and in fp64 otherwise. Token 3 holds one element of 2^-120 (its
+    products would be fp32 subnormals) and token 11 one of 2^126 (they could overflow); both
+    must take the fp64 path, every other token the fp32-product one, and the routing of all
+    40 tokens must equal the oracle's routing step bit for bit (ids and selected logits)."""
+    import torch
+    from nvfp4_weight_only_route_b200 import tfmoe
+    H, I, E, k, T = 512, 256, 16, 4, 40
+    shape = synth.custom_shape(H, I, E, k, global_scale=0.05, router_std=1.0)
+    layer = synth.make_layer(shape, 77)
+    # column 7 of the router weights at +-0.5, so that 2^126 there keeps every logit finite
+    rw = layer["router_w"].copy()
+    rw[:, 7] = np.where(rw[:, 7] & 0x8000, 0xBF00, 0x3F00).astype(np.uint16)
+    layer["router_w"] = rw
+    xf = (synth.make_x(shape, 77, T).astype(np.uint32) << 16).view(np.float32).copy()
+    xf[3, 5] = np.float32(2.0 ** -120)
+    xf[11, 7] = np.float32(2.0 ** 126)
+    x = bf16_bits(xf).reshape(T, H)
+    L = tfmoe.MoELayer(H, I, E, k, T)
+    try:
+        L.load_weights(tfmoe.layer_to_device(layer))
+        xd = torch.from_numpy(x.view(np.int16)).cuda()
+        out = torch.empty_like(xd)
+        L.forward(xd, out)
+        torch.cuda.synchronize()
+        ids = L.buffer_tensor(tfmoe.BUF_TOPK_IDS, torch.int32, (T, k)).cpu().numpy()
+        logits = L.buffer_tensor(tfmoe.BUF_LOGITS, torch.float32, (T, E)).cpu().numpy()
+    finally:
+        L.close()
+    r = oracle_mod.route(layer, x, top_k=k)
+    assert np.array_equal(ids, r["ids"])
+    assert np.array_equal(np.take_along_axis(logits, r["ids"], 1), np.take_along_axis(r["logits"], r["ids"], 1))
+
+
 @pytest.mark.parametrize("regime", sorted(REGIMES))
 def test_single_expert_holds_every_token(oracle_mod, regime):
     H, I, E, k, T = 256, 128, 8, 2, 40
