@@ -65,10 +65,15 @@ WORKLOADS = {
     "sweep_t256": (4, 256, SWEEP_SEEDS),
     "sweep_t2048": (4, 2048, SWEEP_SEEDS),
     "sweep_t7234": (4, 7234, SWEEP_SEEDS),
+    "decode_shared_norm": (1, 8, (1, 2, 3)),
 }
+# Workloads whose layer has a shared expert of m slots (width m * I) and that run through
+# tfmoe_forward_add_norm (shared expert + residual add + RMS norm: the add_moe_norm step).
+SHARED_NORM = {"decode_shared_norm": 1}
+NORM_EPS = 1e-6
 HEADLINE = "sweep_t7234"
 PER_CONFIG = ["tiny", "decode_t1", "decode", "zipf", "prefill", "sweep_t1", "sweep_t32", "sweep_t256",
-              "sweep_t2048"]
+              "sweep_t2048", "decode_shared_norm"]
 # Tokens of the workload per oracle call, for the CPU baseline and the reference arm.
 ORACLE_SAMPLE_TOKENS = {"tiny": 4, "decode_t1": 1, "decode": 8, "zipf": 16, "prefill": 8}
 
@@ -189,7 +194,27 @@ def ncu_traffic(workload: str, stage: str):
 
 def workload_label(name: str, H: int, I: int, E: int, k: int, T: int, seeds) -> str:
     """config.workload of both arms: the workload named by what it is, with its sizes."""
-    return f"{name}: H={H} I={I} E={E} top-{k} T={T} tokens/forward, seeds {list(seeds)} rotated"
+    extra = ""
+    if name in SHARED_NORM:
+        extra = f", shared expert Is={SHARED_NORM[name] * I}, residual add and RMS norm (tfmoe_forward_add_norm)"
+    return f"{name}: H={H} I={I} E={E} top-{k} T={T} tokens/forward{extra}, seeds {list(seeds)} rotated"
+
+
+class AddNormLayer:
+    """A layer with a shared expert whose forward_raw runs tfmoe_forward_add_norm with this
+    object's device residual, norm weights and out_norm buffers, so that every measurement
+    below drives the whole add_moe_norm step; everything else goes to the layer."""
+
+    def __init__(self, layer, residual, norm_w, out_norm):
+        self.layer, self.residual, self.norm_w, self.out_norm = layer, residual, norm_w, out_norm
+
+    def forward_raw(self, x_ptr: int, T: int, out_ptr: int, stream_handle: int) -> int:
+        return self.layer.lib.tfmoe_forward_add_norm(self.layer.handle, x_ptr, T, self.residual.data_ptr(),
+                                                     self.norm_w.data_ptr(), out_ptr, self.out_norm.data_ptr(),
+                                                     stream_handle)
+
+    def __getattr__(self, name):
+        return getattr(self.layer, name)
 
 
 def work_per_forward(mean_active: float, T: int, H: int, I: int, E: int, k: int):
@@ -376,24 +401,36 @@ class Bench:
             si, T, _ = WORKLOADS[n]
             self.max_tokens[si] = max(self.max_tokens.get(si, 0), T)
 
-    def layer(self, si, seed):
-        key = (si, seed)
+    def layer(self, si, seed, m=0):
+        key = (si, seed, m)
         if key not in self.layers:
+            torch = self.torch
             shape = self.synth.SHAPES[si]
             t0 = time.perf_counter()
-            lnp = self.synth.make_layer(shape, replica_seed(seed, self.rank))
+            rs = replica_seed(seed, self.rank)
+            lnp = self.synth.make_layer(shape, rs)
+            if m:
+                lnp.update(self.synth.make_shared(shape, rs, m * shape.I))
             L = self.tfmoe.MoELayer(shape.H, shape.I, shape.E, shape.k, self.max_tokens[si],
                                     has_router_bias=lnp["router_bias"] is not None, flags=self.args.flags,
-                                    gemv_max_tokens=self.args.gemv_max_tokens)
+                                    gemv_max_tokens=self.args.gemv_max_tokens, shared_intermediate=m * shape.I,
+                                    norm_eps=NORM_EPS)
             L.load_weights(self.tfmoe.layer_to_device(lnp, self.dev))
-            self.torch.cuda.synchronize()
+            if m:
+                T = self.max_tokens[si]
+                res = self.synth.make_residual(shape, rs, T)
+                gam = self.synth.make_norm_weight(shape, rs)
+                dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(self.dev)
+                L = AddNormLayer(L, dev(res), dev(gam), torch.empty((T, shape.H), dtype=torch.int16, device=self.dev))
+                lnp["_residual"], lnp["_norm_w"] = res, gam
+            torch.cuda.synchronize()
             self.gen_s += time.perf_counter() - t0
             self.layers[key] = [lnp, L]
         return self.layers[key]
 
-    def slim(self, si, seed):
+    def slim(self, si, seed, m=0):
         """Keep only the router of a host layer whose expert weights no check reads again."""
-        lnp = self.layers[(si, seed)][0]
+        lnp = self.layers[(si, seed, m)][0]
         for k in list(lnp):
             if k not in ("router_w", "router_bias"):
                 lnp[k] = None
@@ -412,15 +449,20 @@ class Bench:
         torch, tfmoe = self.torch, self.tfmoe
         si, T, _ = WORKLOADS[name]
         k, E = self.synth.SHAPES[si].k, self.synth.SHAPES[si].E
+        m = SHARED_NORM.get(name, 0)
         out = torch.empty((T, self.synth.SHAPES[si].H), dtype=torch.int16, device=self.dev)
         worst = 0.0
+        norm_note = ""
         for li, L in enumerate(Ls):
             with torch.cuda.stream(self.stream):
                 tfmoe.check(L.forward_raw(xs[li][0].data_ptr(), T, out.data_ptr(), self.stream.cuda_stream))
             self.stream.synchronize()
             tfmoe.check(L.sync_status(self.stream))
             x_np = xs[li][0].cpu().numpy().view(np.uint16)
-            ids_g = L.buffer_tensor(tfmoe.BUF_TOPK_IDS, torch.int32, (T, k)).cpu().numpy()
+            ids_all = L.buffer_tensor(tfmoe.BUF_TOPK_IDS, torch.int32, (T, k + m)).cpu().numpy()
+            if m and not np.array_equal(ids_all[:, k:], np.tile(E + np.arange(m), (T, 1))):
+                raise SystemExit(f"parity gate ({name}): shared-expert slots missing from the routing")
+            ids_g = ids_all[:, :k]
             log_g = L.buffer_tensor(tfmoe.BUF_LOGITS, torch.float32, (T, E)).cpu().numpy()
             r = oracle.route(lnps[li], x_np, top_k=k)
             if not (np.array_equal(ids_g, r["ids"]) and
@@ -437,7 +479,20 @@ class Bench:
                 continue
             got = out.cpu().numpy().view(np.uint16)
             idx = np.arange(T) if T <= n_sample else np.unique(np.linspace(0, T - 1, n_sample).astype(int))
-            ref = oracle.forward(lnps[li], x_np[idx], top_k=k, intermediates=False)
+            if m:
+                res_np, gam_np = lnps[li]["_residual"][:T], lnps[li]["_norm_w"]
+                ref = oracle.forward(lnps[li], x_np[idx], top_k=k, intermediates=False, residual=res_np[idx],
+                                     norm_w=gam_np, eps=NORM_EPS)
+                got_n = L.out_norm[:T].cpu().numpy().view(np.uint16)[idx]
+                want_n = oracle.rms_norm(got[idx], gam_np, NORM_EPS)
+                gv = (got_n.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+                wv = (want_n.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+                if not np.all(np.abs(gv - wv) <= 2.0 ** -7 * np.abs(wv)):
+                    raise SystemExit(f"parity gate ({name}): RMS norm differs from the oracle's norm of the same row")
+                norm_note = (f"; RMS norm of the output equal to the oracle's norm of the same rows on "
+                             f"{int(np.sum(got_n == want_n))}/{got_n.size} elements, the rest within one ulp")
+            else:
+                ref = oracle.forward(lnps[li], x_np[idx], top_k=k, intermediates=False)
             g64 = (got[idx].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
             half_ulp = 0.5 * 2.0 ** (np.floor(np.log2(np.maximum(np.maximum(np.abs(g64), np.abs(ref["out64"])),
                                                                  2.0 ** -126))) - 7)
@@ -448,12 +503,12 @@ class Bench:
             worst = max(worst, float(np.max(err / tol)))
         return (f"ok: ids and selected logits bit-exact (others within the stated bound) for all {T} tokens x {len(Ls)} layer(s); output within "
                 f"4e-3*S+1e-3 on {min(T, n_sample)} sampled tokens x {min(len(Ls), sample_layers)} layer(s), "
-                f"worst |err|/tol {worst:.3f}")
+                f"worst |err|/tol {worst:.3f}{norm_note}")
 
     def routing_stats(self, name, Ls, xs):
         torch, tfmoe = self.torch, self.tfmoe
         si, T, _ = WORKLOADS[name]
-        E = self.synth.SHAPES[si].E
+        E = self.synth.SHAPES[si].E + SHARED_NORM.get(name, 0)      # expert slots
         out = torch.empty((T, self.synth.SHAPES[si].H), dtype=torch.int16, device=self.dev)
         st = {"active": [], "gemv": [], "mma_pairs": [], "mma": []}
         launches = 0
@@ -602,6 +657,10 @@ class Bench:
         si, T, _ = WORKLOADS[name]
         sh = self.synth.SHAPES[si]
         nbytes, flops = work_per_forward(stats["active"], T, sh.H, sh.I, sh.E, sh.k)
+        m = SHARED_NORM.get(name, 0)
+        if m:   # the shared slots count in "active"; add the residual read and the normed output written
+            nbytes += T * sh.H * 2 * 2
+            flops += 2.0 * T * m * 3 * sh.H * sh.I
         t = ms_per_fwd * 1e-3
         gbs, tfl = nbytes / t / 1e9, flops / t / 1e12
         d = {"algorithmic_bytes_per_forward": nbytes, "hbm_gbs": gbs, "hbm_frac_of_8tbs": gbs / NOMINAL_HBM_GBS,
@@ -630,13 +689,14 @@ class Bench:
 
     def measure(self, name, steps, warmup, graph, n_sample, sample_layers, clocks=False, target_s=None):
         si, T, seeds = WORKLOADS[name]
-        entries = [self.layer(si, sd) for sd in seeds]
+        m = SHARED_NORM.get(name, 0)
+        entries = [self.layer(si, sd, m) for sd in seeds]
         lnps, Ls = [e[0] for e in entries], [e[1] for e in entries]
         n_x = 8 if T <= 256 else 2
         xs = self.inputs(name, n_x)
         parity = self.parity(name, Ls, lnps, xs, n_sample, sample_layers) if self.rank == 0 else "rank 0 only"
         for sd in seeds[max(1, sample_layers):]:
-            self.slim(si, sd)
+            self.slim(si, sd, m)
         log(f"{name}: parity {parity}")
         stats, launches = self.routing_stats(name, Ls, xs)
         per_forward = T >= 1024
@@ -680,7 +740,7 @@ class Bench:
 
     def cpu_baseline(self, name, seconds, one_thread: bool = False):
         si, T, _ = WORKLOADS[name]
-        lnp = self.layers[(si, WORKLOADS[name][2][0])][0]
+        lnp = self.layers[(si, WORKLOADS[name][2][0], SHARED_NORM.get(name, 0))][0]
         x_np = self.synth.make_x(self.synth.SHAPES[si], WORKLOADS[name][2][0], T)
         n = oracle_tokens_per_call(name)
         from oracle import oracle
@@ -736,11 +796,16 @@ def main():
         pcs = {}
         for pc in PER_CONFIG:
             big = WORKLOADS[pc][1] > 256
-            r, _, _, _, _ = b.measure(pc, 0, 3, args.graph, n_sample=8 if big else 64, sample_layers=1,
-                                      target_s=0.3)
-            log(f"{pc}: {r['tok_s']:.0f} tok/s, {r['ms_per_forward'] * 1e3:.1f} us per forward")
-            if not args.no_cpu_baseline:
-                r["cpu_baseline"] = b.cpu_baseline(pc, 2.0, one_thread=pc in ("tiny", "decode_t1", "decode", "zipf"))
+            try:
+                r, _, _, _, _ = b.measure(pc, 0, 3, args.graph, n_sample=8 if big else 64, sample_layers=1,
+                                          target_s=0.3)
+                log(f"{pc}: {r['tok_s']:.0f} tok/s, {r['ms_per_forward'] * 1e3:.1f} us per forward")
+                if not args.no_cpu_baseline:
+                    r["cpu_baseline"] = b.cpu_baseline(pc, 2.0,
+                                                       one_thread=pc in ("tiny", "decode_t1", "decode", "zipf"))
+            except (Exception, SystemExit) as exc:     # a per-config line fails alone, visibly
+                log(f"{pc}: failed: {exc!r}")
+                r = {"error": repr(exc)}
             pcs[pc] = r
 
     if rank == 0:
