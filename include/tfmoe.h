@@ -267,7 +267,8 @@ typedef enum {
  * intermediates) and rewriting that stage's outputs; a measurement aid for
  * timing one kernel in isolation. T must equal the last forward's T and x
  * must be its input (read by the gate/up stages); out receives the combine
- * stage's result. Supported stages: GEMV_GATE_UP, GEMV_DOWN, MMA_GATE_UP,
+ * stage's result (the plain weighted combine, also after a
+ * tfmoe_forward_add_norm: no residual, no norm). Supported stages: GEMV_GATE_UP, GEMV_DOWN, MMA_GATE_UP,
  * MMA_DOWN, GATHER, COMBINE (others return TFMOE_ERR_UNSUPPORTED); a stage
  * whose kernels the forward did not use enqueues nothing. Stage kernels are
  * launched in plain stream order (tfmoe_forward lets the down projection and

@@ -106,6 +106,17 @@ def test_wide_dynamic_range_activations(oracle_mod, regime, H, I, E, k, T):
     _full_check(oracle_mod, layer, x, H, I, E, k, REGIMES[regime])
 
 
+@pytest.mark.parametrize("H,I,E,k,T", [(256, 128, 32, 12, 40), (256, 128, 64, 20, 33)])
+def test_large_top_k_on_the_tensor_core_router(oracle_mod, H, I, E, k, T):
+    """k above 8 with more than 16 tokens: the tensor-core router's epilogue keeps 16 or 32 lower
+    bounds (a looser, still valid threshold than the k-th), and the refinement selects k of the
+    exact candidates."""
+    shape = synth.custom_shape(H, I, E, k, global_scale=0.05, router_std=1.0)
+    layer = synth.make_layer(shape, 300 + k)
+    x = synth.make_x(shape, 300 + k, T)
+    _full_check(oracle_mod, layer, x, H, I, E, k, REGIMES["auto"])
+
+
 def test_router_exact_path_for_extreme_exponents(oracle_mod):
     """The exact router recomputation forms bf16 x bf16 products in fp32 when every product is
     a normal fp32 number, and in fp64 otherwise. Token 3 holds one element of 2^-120 (its
