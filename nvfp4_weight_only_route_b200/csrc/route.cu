@@ -528,9 +528,6 @@ __global__ void __launch_bounds__(kFusedThreads) route_fused_kernel(
     __shared__ int is_last;
     // one CTA per routed expert; the plan (pa.E) also covers the m shared slots
     const int E = (int)gridDim.x, e = blockIdx.x, kx = k + m;
-    // the GEMV gate/up grid may launch now: its CTAs take their places and wait for this
-    // grid to complete before they read anything
-    grid_dep_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // logits of expert e: warp w takes tokens w, w + 8 (T <= 16); lane l covers 8 columns per
     // 256-column step, and the warp adds its lanes in a fixed shuffle order
