@@ -69,3 +69,45 @@ def test_both_arms_name_the_workload_alike():
     b = _load_bench()
     assert (b.workload_label("decode", 2048, 768, 128, 8, 8, (1, 2, 3))
             == "decode: H=2048 I=768 E=128 top-8 T=8 tokens/forward, seeds [1, 2, 3] rotated")
+
+
+def test_shared_norm_workload_is_registered_and_labelled():
+    b = _load_bench()
+    assert "decode_shared_norm" in b.PER_CONFIG and b.SHARED_NORM["decode_shared_norm"] == 1
+    si, T, seeds = b.WORKLOADS["decode_shared_norm"]
+    assert (si, T) == b.WORKLOADS["decode"][:2]
+    label = b.workload_label("decode_shared_norm", 2048, 768, 128, 8, T, seeds)
+    assert "shared expert Is=768" in label and "tfmoe_forward_add_norm" in label
+    assert "shared" not in b.workload_label("decode", 2048, 768, 128, 8, T, seeds)
+    assert b.regime_of("decode_shared_norm") == "hbm"
+
+
+def test_add_norm_layer_passes_its_buffers_and_delegates():
+    """The bench's wrapper drives tfmoe_forward_add_norm with its own residual, norm weights and
+    out_norm, and hands every other attribute to the layer (no GPU: a recording fake)."""
+    b = _load_bench()
+
+    class Buf:
+        def __init__(self, p):
+            self.p = p
+
+        def data_ptr(self):
+            return self.p
+
+    calls = []
+
+    class Lib:
+        def tfmoe_forward_add_norm(self, *a):
+            calls.append(a)
+            return 0
+
+    class Layer:
+        lib, handle = Lib(), 77
+
+        def last_launch_count(self):
+            return 5
+
+    w = b.AddNormLayer(Layer(), Buf(100), Buf(200), Buf(300))
+    assert w.forward_raw(1000, 8, 2000, 9) == 0
+    assert calls == [(77, 1000, 8, 100, 200, 2000, 300, 9)]
+    assert w.last_launch_count() == 5 and w.handle == 77
