@@ -64,7 +64,7 @@ typedef enum {
     TFMOE_ERR_OOM = 2,           /* device allocation failed in create / load_weights */
     TFMOE_ERR_CUDA = 3,          /* a CUDA call or kernel launch failed; see tfmoe_last_error() */
     TFMOE_ERR_NOT_LOADED = 4,    /* forward before load_weights */
-    TFMOE_ERR_UNSUPPORTED = 5,   /* valid arguments this build does not handle (e.g. H % 128 != 0) */
+    TFMOE_ERR_UNSUPPORTED = 5,   /* valid arguments the library does not handle (e.g. H % 128 != 0) */
     TFMOE_ERR_TIMEOUT = 6,       /* a bounded device-side wait gave up (reported by tfmoe_sync_status) */
     TFMOE_ERR_DEVICE = 7         /* a kernel's own check set the device error word */
 } tfmoe_status;
@@ -85,7 +85,7 @@ typedef struct tfmoe_layer tfmoe_layer;   /* opaque */
  * Layer shape. Requirements (else TFMOE_ERR_INVALID_ARG):
  *   hidden H and intermediate I positive multiples of 16; 1 <= top_k <= num_experts;
  *   max_tokens >= 1.
- * This build additionally needs H % 128 == 0, I % 64 == 0 and num_experts <= 256
+ * The library additionally needs H % 128 == 0, I % 64 == 0 and num_experts <= 256
  * (else TFMOE_ERR_UNSUPPORTED).
  * shared_intermediate: 0, or the shared expert's width Is, a multiple of I; the
  * library runs it as m = Is / I extra expert slots that every token takes with

@@ -161,10 +161,10 @@ tfmoe_status tfmoe_create(const tfmoe_layer_desc *desc, tfmoe_layer **out)
     if (d.flags & ~(TFMOE_FLAG_FORCE_GEMV | TFMOE_FLAG_FORCE_MMA | TFMOE_FLAG_DEBUG_CHECKS | TFMOE_FLAG_TEST_TIMEOUT))
         return fail(TFMOE_ERR_INVALID_ARG, "unknown flag bits 0x%x", d.flags);
     if (d.hidden % 128 || d.intermediate % 64)
-        return fail(TFMOE_ERR_UNSUPPORTED, "this build needs hidden %% 128 == 0 and intermediate %% 64 == 0 (got %d, %d)",
+        return fail(TFMOE_ERR_UNSUPPORTED, "libtfmoe needs hidden %% 128 == 0 and intermediate %% 64 == 0 (got %d, %d)",
                     d.hidden, d.intermediate);
     if (d.hidden > kMaxReduction || d.intermediate > kMaxReduction)
-        return fail(TFMOE_ERR_UNSUPPORTED, "this build supports hidden and intermediate up to %d (got %d, %d)",
+        return fail(TFMOE_ERR_UNSUPPORTED, "libtfmoe supports hidden and intermediate up to %d (got %d, %d)",
                     kMaxReduction, d.hidden, d.intermediate);
     if (d.shared_intermediate < 0 || d.shared_intermediate % d.intermediate)
         return fail(TFMOE_ERR_INVALID_ARG, "shared_intermediate (%d) must be 0 or a multiple of intermediate (%d)",
@@ -173,7 +173,7 @@ tfmoe_status tfmoe_create(const tfmoe_layer_desc *desc, tfmoe_layer **out)
         return fail(TFMOE_ERR_INVALID_ARG, "norm_eps must be finite and >= 0");
     const long long m = d.shared_intermediate / d.intermediate;
     if (d.num_experts + m > 256 || d.top_k + m > 32)
-        return fail(TFMOE_ERR_UNSUPPORTED, "this build supports num_experts + m <= 256 and top_k + m <= 32 "
+        return fail(TFMOE_ERR_UNSUPPORTED, "libtfmoe supports num_experts + m <= 256 and top_k + m <= 32 "
                     "(m = shared_intermediate / intermediate = %lld)", m);
     const long long kx = d.top_k + m;
     if ((long long)d.max_tokens * kx > (1LL << 30))

@@ -26,7 +26,7 @@ __host__ __device__ __forceinline__ size_t scale_offset(size_t row_tile_index, i
     return (row_tile_index * (size_t)KT + (size_t)kt) * kTileScaleBytes;
 }
 
-// Largest reduction length (hidden or intermediate) of this build: a GEMV task
+// Largest reduction length (hidden or intermediate) the library supports: a GEMV task
 // stages the scales of all its column tiles with one tensor copy, whose box
 // extent is limited to 256 tiles.
 constexpr int kMaxReduction = 256 * kTileK;

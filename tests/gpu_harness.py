@@ -14,7 +14,7 @@ def bf16_to_f64(bits):
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-class GpuRun:
+class GpuLayerRun:
     def __init__(self, layer_np, H, I, E, k, max_tokens, flags=0, gemv_max_tokens=0):
         import torch
         from nvfp4_weight_only_route_b200 import tfmoe

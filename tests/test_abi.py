@@ -76,7 +76,7 @@ def _create(tf, **kw):
     (dict(hidden=500), 1), (dict(intermediate=0), 1), (dict(top_k=9), 1), (dict(top_k=0), 1),
     (dict(max_tokens=0), 1), (dict(flags=3), 1), (dict(flags=0x100), 1),
     (dict(hidden=528), 5), (dict(intermediate=80), 5), (dict(num_experts=300, top_k=2), 5),
-    # limits of this build: the reduction length a GEMV task's scale copy covers (256 tiles of 64),
+    # limits of the library: the reduction length a GEMV task's scale copy covers (256 tiles of 64),
     # top_k <= 32 (one warp per token in top-k), 32-bit offsets of the permuted activation rows
     (dict(hidden=16384 + 128), 5), (dict(intermediate=16384 + 64), 5),
     (dict(num_experts=64, top_k=33), 5),

@@ -12,7 +12,7 @@ import pytest
 
 from nvfp4_weight_only_route_b200 import synth
 
-from gpu_harness import GpuRun, check_intermediates, check_logits, check_output, check_routing, logit_bound
+from gpu_harness import GpuLayerRun, check_intermediates, check_logits, check_output, check_routing, logit_bound
 from layer_builders import bf16_bits
 
 pytestmark = pytest.mark.gpu
@@ -31,7 +31,7 @@ def _cuda():
 
 def _full_check(oracle_mod, layer, x, H, I, E, k, flags, max_tokens=None):
     T = x.shape[0]
-    run = GpuRun(layer, H, I, E, k, max_tokens or max(T, 1), flags=flags)
+    run = GpuLayerRun(layer, H, I, E, k, max_tokens or max(T, 1), flags=flags)
     try:
         g = run.forward(x)
     finally:
@@ -181,7 +181,7 @@ def test_exact_logit_ties(oracle_mod, regime):
 def test_zero_tokens_launches_nothing(oracle_mod):
     import torch
     s = synth.SHAPES[0]
-    run = GpuRun(synth.make_layer(s, 0), s.H, s.I, s.E, s.k, 4)
+    run = GpuLayerRun(synth.make_layer(s, 0), s.H, s.I, s.E, s.k, 4)
     try:
         x = torch.zeros((1, s.H), dtype=torch.int16, device="cuda")
         out = torch.full((1, s.H), 7, dtype=torch.int16, device="cuda")
@@ -199,7 +199,7 @@ def test_max_tokens_and_over_limit(oracle_mod):
     layer = synth.make_layer(s, 0)
     x = synth.make_x(s, 0, 6)
     _full_check(oracle_mod, layer, x, s.H, s.I, s.E, s.k, 0, max_tokens=6)
-    run = GpuRun(layer, s.H, s.I, s.E, s.k, 6)
+    run = GpuLayerRun(layer, s.H, s.I, s.E, s.k, 6)
     try:
         xt = torch.zeros((7, s.H), dtype=torch.int16, device="cuda")
         out = torch.zeros((7, s.H), dtype=torch.int16, device="cuda")
@@ -233,7 +233,7 @@ def test_deterministic_bytes(oracle_mod):
     s = synth.SHAPES[2]
     layer = synth.make_layer(s, 4)
     x = synth.make_x(s, 4, 256)
-    run = GpuRun(layer, s.H, s.I, s.E, s.k, 256)
+    run = GpuLayerRun(layer, s.H, s.I, s.E, s.k, 256)
     try:
         a = run.forward(x, intermediates=False)["out"]
         b = run.forward(x, intermediates=False)["out"]
@@ -247,7 +247,7 @@ def test_forward_host_matches_device(oracle_mod):
     s = synth.SHAPES[1]
     layer = synth.make_layer(s, 1)
     x = synth.make_x(s, 1, 8)
-    run = GpuRun(layer, s.H, s.I, s.E, s.k, 8)
+    run = GpuLayerRun(layer, s.H, s.I, s.E, s.k, 8)
     try:
         dev = run.forward(x, intermediates=False)["out"]
         xh = torch.from_numpy(x.view(np.int16)).pin_memory()
@@ -272,7 +272,7 @@ def test_debug_checks_report_clean(oracle_mod):
     s = synth.SHAPES[1]
     layer = synth.make_layer(s, 2)
     x = synth.make_x(s, 2, 8)
-    run = GpuRun(layer, s.H, s.I, s.E, s.k, 8, flags=4)
+    run = GpuLayerRun(layer, s.H, s.I, s.E, s.k, 8, flags=4)
     try:
         g = run.forward(x)
     finally:
@@ -310,7 +310,7 @@ def test_prefill_layer_sampled(oracle_mod):
     s = synth.SHAPES[3]
     layer = synth.make_layer(s, 5)
     x = synth.make_x(s, 5, 8192)
-    run = GpuRun(layer, s.H, s.I, s.E, s.k, 8192)
+    run = GpuLayerRun(layer, s.H, s.I, s.E, s.k, 8192)
     try:
         _sampled_check(oracle_mod, run, layer, x, s.k, 24, 5)
     finally:
@@ -322,7 +322,7 @@ def test_large_layer_sweep_sampled(oracle_mod, seed):
     """One large-sweep layer per seed (6..10), every T of the sweep."""
     s = synth.SHAPES[4]
     layer = synth.make_layer(s, seed)
-    run = GpuRun(layer, s.H, s.I, s.E, s.k, max(s.T))
+    run = GpuLayerRun(layer, s.H, s.I, s.E, s.k, max(s.T))
     try:
         for T in s.T:
             x = synth.make_x(s, seed, T)
@@ -340,7 +340,7 @@ def test_large_batch_plan(oracle_mod, regime):
     s = synth.custom_shape(H=256, I=128, E=64, k=8)
     layer = synth.make_layer(s, 21)
     x = synth.make_x(s, 21, 601)
-    run = GpuRun(layer, s.H, s.I, s.E, s.k, 601, flags=REGIMES[regime])
+    run = GpuLayerRun(layer, s.H, s.I, s.E, s.k, 601, flags=REGIMES[regime])
     try:
         g = run.forward(x, intermediates=True)
         o = oracle_mod.forward(layer, x, top_k=s.k, intermediates=True)
@@ -385,7 +385,7 @@ def test_debug_checks_flag_non_finite_logits(oracle_mod, value):
     from nvfp4_weight_only_route_b200 import tfmoe
     s = synth.SHAPES[1]
     layer = synth.make_layer(s, 2)
-    run = GpuRun(layer, s.H, s.I, s.E, s.k, 8, flags=tfmoe.FLAG_DEBUG_CHECKS)
+    run = GpuLayerRun(layer, s.H, s.I, s.E, s.k, 8, flags=tfmoe.FLAG_DEBUG_CHECKS)
     try:
         for T in (8, 40):                     # the fused decode routing and the split router + top-k
             x = synth.make_x(s, 2, T)
@@ -397,7 +397,7 @@ def test_debug_checks_flag_non_finite_logits(oracle_mod, value):
             out = torch.empty_like(xd)
             if T > 8:
                 run.close()
-                run = GpuRun(layer, s.H, s.I, s.E, s.k, T, flags=tfmoe.FLAG_DEBUG_CHECKS)
+                run = GpuLayerRun(layer, s.H, s.I, s.E, s.k, T, flags=tfmoe.FLAG_DEBUG_CHECKS)
             run.layer.forward(xd, out)
             assert run.layer.sync_status() == tfmoe.ERR_DEVICE
             assert "0x8" in tfmoe.last_error()
@@ -416,8 +416,8 @@ def test_handles_of_different_shapes_coexist(oracle_mod):
     big_s = synth.custom_shape(H=512, I=1024, E=8, k=2, global_scale=0.05, router_std=1.0)
     small_s = synth.custom_shape(H=128, I=64, E=4, k=1, global_scale=0.05, router_std=1.0)
     big_l, small_l = synth.make_layer(big_s, 41), synth.make_layer(small_s, 42)
-    big = GpuRun(big_l, 512, 1024, 8, 2, 40, flags=REGIMES["gemv"])
-    small = GpuRun(small_l, 128, 64, 4, 1, 40, flags=REGIMES["gemv"])
+    big = GpuLayerRun(big_l, 512, 1024, 8, 2, 40, flags=REGIMES["gemv"])
+    small = GpuLayerRun(small_l, 128, 64, 4, 1, 40, flags=REGIMES["gemv"])
     try:
         for T in (5, 33):
             for run, layer, s in ((big, big_l, big_s), (small, small_l, small_s)):
