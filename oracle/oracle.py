@@ -41,7 +41,7 @@ class _Layer(ctypes.Structure):
 
 
 class _Epilogue(ctypes.Structure):
-    _fields_ = [("residual", _u16p), ("norm_w", _u16p), ("eps", ctypes.c_double)]
+    _fields_ = [("residual", _u16p), ("norm_w", _u16p), ("eps", ctypes.c_double), ("act_fp4", ctypes.c_int32)]
 
 
 class _Outputs(ctypes.Structure):
@@ -85,6 +85,12 @@ def lib():
         _lib.oracle_forward.argtypes = [ctypes.POINTER(_Layer), _u16p, ctypes.c_int32,
                                         ctypes.c_int32, ctypes.POINTER(_Epilogue), ctypes.POINTER(_Outputs)]
         _lib.oracle_rms_norm.restype = ctypes.c_int
+        _lib.oracle_e2m1_rne.restype = ctypes.c_uint
+        _lib.oracle_e2m1_rne.argtypes = [ctypes.c_double]
+        _lib.oracle_e4m3_rne.restype = ctypes.c_uint
+        _lib.oracle_e4m3_rne.argtypes = [ctypes.c_double]
+        _lib.oracle_quant_act_row.restype = ctypes.c_int
+        _lib.oracle_quant_act_row.argtypes = [_f64p, ctypes.c_int32, _u8p, _u8p, _f32p, _f64p]
         _lib.oracle_rms_norm.argtypes = [_u16p, _u16p, ctypes.c_int32, ctypes.c_int32, ctypes.c_double, _u16p]
         _lib.oracle_route.restype = ctypes.c_int
         _lib.oracle_route.argtypes = [ctypes.POINTER(_Layer), _u16p, ctypes.c_int32, ctypes.c_int32,
@@ -120,6 +126,29 @@ def _ptr(a: Optional[np.ndarray], t):
     return a.ctypes.data_as(t)
 
 
+def e2m1_rne(v: float) -> int:
+    return int(lib().oracle_e2m1_rne(v))
+
+
+def e4m3_rne(v: float) -> int:
+    return int(lib().oracle_e4m3_rne(v))
+
+
+def quant_act_row(v: np.ndarray):
+    """The oracle's NVFP4 quantisation of one activation row (values exactly representable in
+    fp32, length a multiple of 16): (codes uint8 [K], scales uint8 [K/16], g fp32, deq fp64 [K])."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    K = v.shape[0]
+    codes, scales = np.zeros(K, np.uint8), np.zeros(K // 16, np.uint8)
+    g = ctypes.c_float()
+    deq = np.zeros(K, np.float64)
+    rc = lib().oracle_quant_act_row(_ptr(v, _f64p), K, _ptr(codes, _u8p), _ptr(scales, _u8p), ctypes.byref(g),
+                                    _ptr(deq, _f64p))
+    if rc != 0:
+        raise RuntimeError(f"oracle_quant_act_row failed with code {rc}")
+    return codes, scales, float(g.value), deq
+
+
 def rms_norm(v: np.ndarray, gamma: np.ndarray, eps: float) -> np.ndarray:
     """The oracle's RMS norm of bf16 rows v [T][H] with bf16 gamma [H] (bf16 bits out)."""
     v = np.ascontiguousarray(v, dtype=np.uint16)
@@ -134,7 +163,7 @@ def rms_norm(v: np.ndarray, gamma: np.ndarray, eps: float) -> np.ndarray:
 
 def forward(layer: Dict[str, Optional[np.ndarray]], x: np.ndarray, *, top_k: int,
             nthreads: int = 0, intermediates: bool = False, residual: Optional[np.ndarray] = None,
-            norm_w: Optional[np.ndarray] = None, eps: float = 1e-6) -> Dict[str, np.ndarray]:
+            norm_w: Optional[np.ndarray] = None, eps: float = 1e-6, act_fp4: bool = False) -> Dict[str, np.ndarray]:
     """Run the oracle on host arrays in the canonical layout.
 
     ``x`` is bf16 bits [T][H]. Returns out (bf16 bits), out64, S, and with
@@ -143,6 +172,8 @@ def forward(layer: Dict[str, Optional[np.ndarray]], x: np.ndarray, *, top_k: int
     [H][Is/2], [H][Is/16], globals as one-element fp32 arrays) adds the shared expert
     (``a_sh``, ``y_sh`` with ``intermediates``). ``residual`` (bf16 bits [T][H]) is added
     to the output; ``norm_w`` (bf16 bits [H]) adds ``out_norm``, the RMS norm of ``out``.
+    ``act_fp4`` selects the W4A4 variant: the routed experts read NVFP4-quantised x (gate/up)
+    and a (down) rows (see quant_act_row).
     """
     E, H = layer["router_w"].shape
     I = layer["gate_codes"].shape[1]
@@ -178,7 +209,7 @@ def forward(layer: Dict[str, Optional[np.ndarray]], x: np.ndarray, *, top_k: int
         L.sh_down_codes = _ptr(arr("shared_down_codes", np.uint8), _u8p)
         L.sh_down_scales = _ptr(arr("shared_down_scales", np.uint8), _u8p)
         L.sh_down_global = float(np.float32(layer["shared_down_global"].reshape(-1)[0]))
-    epi = _Epilogue(_ptr(None, _u16p), _ptr(None, _u16p), float(eps))
+    epi = _Epilogue(_ptr(None, _u16p), _ptr(None, _u16p), float(eps), 1 if act_fp4 else 0)
     if residual is not None:
         residual = np.ascontiguousarray(residual, dtype=np.uint16)
         assert residual.shape == (T, H)

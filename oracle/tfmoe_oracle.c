@@ -44,6 +44,8 @@
  *   out = bf16_RNE( sum over slots s=0..k-1 of g_s * y_s
  *                   (+ y_shared) (+ residual) )                   in fp64
  *   out_norm = bf16_RNE( out * gamma / sqrt(mean over h of out^2 + eps) )
+ *   W4A4 variant (act_fp4): gate/up read NVFP4-quantised x rows and down reads
+ *   NVFP4-quantised a rows (the quantiser and its reading are defined below)
  *
  * Parity pins live in the repository's CPU test-suite; every function below
  * is pinned there (format tables, a hand-worked block, closed-form chains,
@@ -125,6 +127,89 @@ static void dequant_row(const uint8_t *codes, const uint8_t *scales, float globa
 static double silu(double z) { return z / (1.0 + exp(-z)); }
 
 /* ------------------------------------------------------------------ */
+/* NVFP4 activations (the W4A4 variant)                                 */
+/* ------------------------------------------------------------------ */
+/*
+ * The pages name an all-FP4 prefill (FP4 tensor cores) beside the W4A16 path but give no
+ * recipe for quantising activations. The reading taken here quantises an activation row the
+ * way the weights are stored: E2M1 codes, one E4M3 scale per 16 consecutive elements, one
+ * fp32 multiplier per row (per token for x, per routed pair for a), every decision in fp32:
+ *   g   = fl32(amax_row / 2688)             (2688 = 6 * 448; g = 1 for an all-zero row)
+ *   s_b = E4M3_RNE(min(fl32(amax_b / fl32(6 g)), 448))
+ *   q_i = E2M1_RNE(fl32(v_i / fl32(s_b g)))  (saturating at +-6; 0 when s_b g = 0)
+ *   deq_i = E2M1(q_i) * s_b * g             (exact in fp64)
+ */
+
+/* E2M1 code of the value nearest to v, ties to the code with an even mantissa bit,
+ * saturating at +-6; the sign bit is set for every v < 0 (so tiny negatives give -0). */
+unsigned oracle_e2m1_rne(double v)
+{
+    const double a = fabs(v);
+    unsigned c;
+    if (a <= 0.25) c = 0;            /* 0.25: between 0 (m=0) and 0.5 (m=1) -> 0 */
+    else if (a < 0.75) c = 1;
+    else if (a <= 1.25) c = 2;       /* 0.75 -> 1.0 (m=0); 1.25: 1.0 (m=0) against 1.5 (m=1) */
+    else if (a < 1.75) c = 3;
+    else if (a <= 2.5) c = 4;        /* 1.75 -> 2.0; 2.5: 2.0 (m=0) against 3.0 (m=1) */
+    else if (a < 3.5) c = 5;
+    else if (a <= 5.0) c = 6;        /* 3.5 -> 4.0; 5.0: 4.0 (m=0) against 6.0 (m=1) */
+    else c = 7;                      /* up to 6 and beyond: saturate */
+    return (v < 0.0 ? 8u : 0u) | c;
+}
+
+/* E4M3 byte of the value nearest to v >= 0 (ties to even), values above 448 clamped to 448.
+ * The quantum is 2^(e-3) for v in [2^e, 2^(e+1)), e >= -6, and 2^-9 below 2^-6. */
+unsigned oracle_e4m3_rne(double v)
+{
+    if (!(v > 0.0)) return 0;
+    if (v >= 448.0) return 0x7Eu;
+    int e;
+    (void)frexp(v, &e);              /* v = f 2^e, f in [0.5, 1): leading bit 2^(e-1) */
+    int q_exp = (e - 1) - 3;
+    if (q_exp < -9) q_exp = -9;
+    double r = ldexp(rint(ldexp(v, -q_exp)), q_exp);
+    if (r > 448.0) r = 448.0;
+    for (unsigned b = 0; b < 0x7Fu; ++b)
+        if (oracle_e4m3(b) == r) return b;
+    return 0x7Eu;                    /* not reached: every rounded value is an E4M3 value */
+}
+
+/* One activation row of K values (each exactly a float) in NVFP4, as the comment above
+ * defines: codes [K] (one per byte here), scales [K/16], the row's fp32 multiplier and the
+ * dequantised values [K]. */
+int oracle_quant_act_row(const double *v, int32_t K, uint8_t *codes, uint8_t *scales, float *g_out, double *deq)
+{
+    if (!v || K <= 0 || K % 16) return 1;
+    float amax = 0.0f;
+    for (int i = 0; i < K; ++i) {
+        const float a = fabsf((float)v[i]);
+        if (a > amax) amax = a;
+    }
+    const float g = amax > 0.0f ? amax / 2688.0f : 1.0f;
+    const float six_g = 6.0f * g;
+    for (int b = 0; b < K / 16; ++b) {
+        float amax_b = 0.0f;
+        for (int i = 16 * b; i < 16 * b + 16; ++i) {
+            const float a = fabsf((float)v[i]);
+            if (a > amax_b) amax_b = a;
+        }
+        float ratio = amax_b / six_g;
+        if (ratio > 448.0f) ratio = 448.0f;
+        const unsigned sb = oracle_e4m3_rne((double)ratio);
+        const double sbv = oracle_e4m3(sb);
+        const float S = (float)sbv * g;
+        if (scales) scales[b] = (uint8_t)sb;
+        for (int i = 16 * b; i < 16 * b + 16; ++i) {
+            const unsigned c = (S > 0.0f) ? oracle_e2m1_rne((double)((float)v[i] / S)) : 0u;
+            if (codes) codes[i] = (uint8_t)c;
+            if (deq) deq[i] = oracle_e2m1(c) * sbv * (double)g;
+        }
+    }
+    if (g_out) *g_out = g;
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
 /* The layer                                                            */
 /* ------------------------------------------------------------------ */
 
@@ -153,6 +238,7 @@ typedef struct {
     const uint16_t *residual;   /* bf16 [T][H], added to the layer output */
     const uint16_t *norm_w;     /* bf16 [H], gamma of the RMS norm of the layer output */
     double eps;                 /* the norm's epsilon */
+    int32_t act_fp4;            /* 1: the W4A4 variant, x and a quantised to NVFP4 (routed experts) */
 } oracle_epilogue;
 
 /* Outputs. Every pointer except out may be NULL. Per-pair arrays are indexed
@@ -310,6 +396,17 @@ int oracle_forward(const oracle_layer *L, const uint16_t *x, int32_t T, int32_t 
         route_token(L, x + (size_t)t * H, logits + (size_t)t * E, ids + (size_t)t * k, g + (size_t)t * k);
 
     for (size_t i = 0; i < (size_t)T * H; ++i) xd[i] = oracle_bf16_to_double(x[i]);
+    const int fp4 = epi && epi->act_fp4;
+    if (fp4 && Is > 0) return 1;      /* the W4A4 variant covers the routed experts */
+    if (fp4) {                        /* gate/up read the NVFP4-quantised token rows */
+        double *row = (double *)malloc(sizeof(double) * H);
+        if (!row) return 2;
+        for (int t = 0; t < T; ++t) {
+            oracle_quant_act_row(xd + (size_t)t * H, H, NULL, NULL, NULL, row);
+            memcpy(xd + (size_t)t * H, row, sizeof(double) * H);
+        }
+        free(row);
+    }
 
     /* Step 2: per-expert pair lists, in (token, slot) order. */
     for (size_t p = 0; p < P; ++p) count[ids[p]]++;
@@ -350,7 +447,21 @@ int oracle_forward(const oracle_layer *L, const uint16_t *x, int32_t T, int32_t 
         }
     }
 
-    /* Step 4: down projection, rows in parallel; y stays in fp64. */
+    /* Step 4: down projection, rows in parallel; y stays in fp64. Its activation is a, or for
+     * the W4A4 variant a's NVFP4-quantised rows. */
+    double *ad = NULL;                /* W4A4: the dequantised NVFP4 rows of a */
+    if (fp4) {
+        ad = (double *)malloc(sizeof(double) * P * I);
+        if (!ad) return 2;
+        for (size_t i = 0; i < P * I; ++i) ad[i] = oracle_bf16_to_double(a[i]);
+        double *row = (double *)malloc(sizeof(double) * I);
+        if (!row) return 2;
+        for (size_t p = 0; p < P; ++p) {
+            oracle_quant_act_row(ad + p * I, I, NULL, NULL, NULL, row);
+            memcpy(ad + p * I, row, sizeof(double) * I);
+        }
+        free(row);
+    }
     for (int e = 0; e < E; ++e) {
         if (count[e] == 0) continue;
 #pragma omp parallel num_threads(nthreads)
@@ -363,9 +474,10 @@ int oracle_forward(const oracle_layer *L, const uint16_t *x, int32_t T, int32_t 
                 for (int q = start[e]; q < start[e + 1]; ++q) {
                     int p = pairs[q];
                     const uint16_t *ar = a + (size_t)p * I;
+                    const double *aq = ad ? ad + (size_t)p * I : NULL;
                     double s = 0.0, sa = 0.0;
                     for (int j = 0; j < I; ++j) {
-                        double term = oracle_bf16_to_double(ar[j]) * dd[j];
+                        double term = (aq ? aq[j] : oracle_bf16_to_double(ar[j])) * dd[j];
                         s += term;
                         sa += fabs(term);
                     }
@@ -419,7 +531,7 @@ int oracle_forward(const oracle_layer *L, const uint16_t *x, int32_t T, int32_t 
     if (O->y) memcpy(O->y, y, sizeof(double) * P * H);
     if (O->yabs) memcpy(O->yabs, yabs, sizeof(double) * P * H);
 
-    free(logits); free(ids); free(g); free(a); free(y); free(yabs); free(xd);
+    free(logits); free(ids); free(g); free(a); free(y); free(yabs); free(xd); free(ad);
     free(count); free(start); free(pairs);
     return 0;
 }

@@ -17,6 +17,7 @@ import test_oracle_bruteforce as bf
 import test_oracle_closed_form as cf
 import test_oracle_epilogue as ep
 import test_oracle_formats as ff
+import test_oracle_w4a4 as w4
 
 MUTATIONS = {
     "nibble_order": ("(c % 2 == 0) ? (byte & 0x0Fu) : (byte >> 4)", "(c % 2 == 0) ? (byte >> 4) : (byte & 0x0Fu)"),
@@ -46,6 +47,11 @@ MUTATIONS = {
     "norm_eps_outside_root": ("1.0 / sqrt(ss / (double)H + eps)", "1.0 / (sqrt(ss / (double)H) + eps)"),
     "norm_gamma_column_0": ("oracle_bf16_to_double(gamma[h])", "oracle_bf16_to_double(gamma[0])"),
     "norm_mean_off_by_one": ("sqrt(ss / (double)H + eps)", "sqrt(ss / (double)(H - 1) + eps)"),
+    "act_e2m1_tie_away_from_zero": ("if (a <= 0.25) c = 0;", "if (a < 0.25) c = 0;"),
+    "act_global_over_448": ("amax / 2688.0f", "amax / 448.0f"),
+    "act_block_scale_from_row_amax": ("float ratio = amax_b / six_g;", "float ratio = amax / six_g;"),
+    "act_e4m3_truncates": ("rint(ldexp(v, -q_exp))", "floor(ldexp(v, -q_exp))"),
+    "w4a4_down_reads_unquantised_a": ("const double *aq = ad ? ad + (size_t)p * I : NULL;", "const double *aq = NULL;"),
 }
 
 
@@ -71,6 +77,10 @@ def _all_pins(mod):
             cases.append(lambda n=name: getattr(ep, n)(mod))
     cases.append(lambda: ep.test_shared_expert_residual_and_norm_match_dense(mod, 64, 32, 4, 2, 32, 3, 21))
     cases.append(lambda: ep.test_norm_of_constant_row_is_sign_when_eps_is_zero(mod, 0.75))
+    for name in dir(w4):
+        if name.startswith("test_") and name != "test_w4a4_forward_matches_dense":
+            cases.append(lambda n=name: getattr(w4, n)(mod))
+    cases.append(lambda: w4.test_w4a4_forward_matches_dense(mod, 64, 32, 4, 2, 3, 61))
     for c in cases:
         try:
             c()
